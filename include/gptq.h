@@ -1,0 +1,207 @@
+/*
+ * gptq.h -- C ABI of the B200 GPTQ layer solver (libgptq.so).
+ *
+ * The library turns one linear layer's weights W (out x in) and its
+ * calibration activations X (in x tokens) into 2/3/4/8-bit group-quantized
+ * integer codes with one scale and one zero per group, the act-order
+ * permutation and g_idx.  Three calls make one layer solve:
+ *
+ *   gptq_hessian_accumulate  S += X X^T            (once per calibration chunk)
+ *   gptq_prepare_hinv        H = 2 S / n, dead-channel fix, dampening,
+ *                            act-order permutation, U = upper Cholesky
+ *                            factor of H^-1
+ *   gptq_quantize_layer      the blocked column sweep with error
+ *                            compensation, group quantization and packing
+ *
+ * What is computed follows the GPTQ pages: "gptq" glossary page (Method and
+ * Algorithm: layer-wise, Hessian from calibration data, quantize each weight
+ * in order and compensate the error with H^-1; Group quantization), "Using
+ * AutoGPTQ in Practice" (Hessian computation, Cholesky factorization, group
+ * quantization; Key Parameters: bits, group_size, desc_act, damp_percent),
+ * "gptq" agent-skill page (Group-wise quantization: own scale and zero per
+ * group; group_size -1 = per column) and the AutoGPTQ artifact page (2/3/4/8
+ * bits, symmetric and asymmetric schemes, config validation).
+ *
+ * Conventions for every call
+ *   - Pointers named "device" are CUDA device (or managed) memory owned by the
+ *     caller; the library never keeps them after the call returns and never
+ *     allocates device memory itself: scratch space is the caller's
+ *     workspace, sized by gptq_workspace_bytes().
+ *   - stream is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream).  Work is enqueued on it; only gptq_prepare_hinv waits for it.
+ *   - Matrices are row-major unless stated otherwise; leading dimensions are
+ *     in elements.
+ *   - Every call returns a gptq_status_t.  Nothing aborts or traps.  On an
+ *     error, gptq_last_error() returns a message for the calling thread.
+ *   - The kernels are built for sm_100a only; on any other device the calls
+ *     return GPTQ_ERR_UNSUPPORTED.  There is no CPU fallback.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GPTQ_ABI_VERSION 1
+
+typedef enum gptq_status {
+  GPTQ_OK = 0,
+  GPTQ_ERR_INVALID_ARG = 1,  /* rejected on the host before any launch        */
+  GPTQ_ERR_NOT_PD = 2,       /* damped Hessian has no Cholesky factor          */
+  GPTQ_ERR_NONFINITE = 3,    /* NaN or Inf met in S                            */
+  GPTQ_ERR_WORKSPACE = 4,    /* workspace missing, misaligned or too small     */
+  GPTQ_ERR_CUDA = 5,         /* a CUDA runtime call failed (message says which)*/
+  GPTQ_ERR_TIMEOUT = 6,      /* a bounded device-side wait gave up             */
+  GPTQ_ERR_UNSUPPORTED = 7   /* valid request this build does not implement    */
+} gptq_status_t;
+
+typedef enum gptq_dtype {
+  GPTQ_F16 = 0,
+  GPTQ_BF16 = 1,
+  GPTQ_F32 = 2
+} gptq_dtype_t;
+
+/*
+ * Quantization settings, the fields of the pages' BaseQuantizeConfig
+ * ("gptq" agent-skill page, Quantization configurations; "Using AutoGPTQ in
+ * Practice", Key Parameters) plus the symmetric flag (AutoGPTQ artifact page)
+ * and the lazy-batch width.
+ *   bits          2, 3, 4 or 8.
+ *   group_size    -1 (one group per output row) or a positive divisor of in.
+ *                 This build also needs 128 % group_size == 0 or
+ *                 group_size % 128 == 0 (else GPTQ_ERR_UNSUPPORTED).
+ *   sym           0: asymmetric grid over [min(0, min w), max(0, max w)],
+ *                    zero = rint(-lo / scale);
+ *                 1: symmetric, scale = 2 max|w| / maxq, zero = (maxq+1)/2.
+ *   desc_act      1: process columns by decreasing diag(H) (ActOrder).
+ *   damp_percent  >= 0, finite: damp_percent * mean(diag H) is added to the
+ *                 diagonal.
+ *   block_size    > 0; with group_size != -1 it must divide group_size or be
+ *                 a multiple of it.  It is the lazy-batch width: it changes
+ *                 only the order of floating-point rounding, never the
+ *                 result in exact arithmetic.  The kernels sweep 128 columns
+ *                 at a time and apply the deferred update of later columns
+ *                 every max(128, block_size rounded down to 128) columns.
+ * maxq = 2^bits - 1.  code = clamp(rint(w / scale) + zero, 0, maxq), the
+ * division and rint in IEEE float32 (round half to even).
+ */
+typedef struct gptq_config {
+  int32_t bits;
+  int32_t group_size;
+  int32_t sym;
+  int32_t desc_act;
+  float damp_percent;
+  int32_t block_size;
+} gptq_config_t;
+
+/* GPTQ_ABI_VERSION of the loaded library. */
+int gptq_abi_version(void);
+
+/* Message for the last error on the calling thread ("" if none).  The
+ * pointer stays valid until the thread's next gptq_* call. */
+const char* gptq_last_error(void);
+
+/* Host-only check of a configuration for a layer of out x in (the pages'
+ * config validator, AutoGPTQ artifact page).  out may be 0. */
+gptq_status_t gptq_validate_config(const gptq_config_t* cfg, int64_t out,
+                                   int64_t in);
+
+/* Bytes of device workspace that gptq_prepare_hinv (out = 0) or both
+ * gptq_prepare_hinv and gptq_quantize_layer (out > 0) need for a layer of
+ * out x in.  Returns 0 for invalid sizes.  The workspace must be 256-byte
+ * aligned; its contents need no initialisation and are not preserved. */
+size_t gptq_workspace_bytes(int64_t out, int64_t in, const gptq_config_t* cfg);
+
+/*
+ * S += X X^T: accumulate the Gram matrix of one chunk of calibration tokens
+ * ("gptq" glossary page, Algorithm (1): the Hessian comes from calibration
+ * data).
+ *   S        device fp32, in x in, row-major.  Only the upper triangle with
+ *            the diagonal (S[i][j], j >= i) is read and written; the strictly
+ *            lower triangle is left untouched.  Zero it before the first
+ *            chunk.  (S, n) is additive: chunks may come in any number of
+ *            calls, and a saved (S, n) resumes accumulation.
+ *   in       channels, >= 1.
+ *   X        device, in x tokens, element type xt, row stride ldx >= tokens
+ *            (row i = channel i, tokens contiguous).  Read only.
+ *   tokens   >= 0; 0 is a no-op.
+ *   n_accum  host pointer or NULL; *n_accum += tokens on success.
+ * fp16/bf16 X with a 16-byte aligned base and (ldx * 2) % 16 == 0 runs on the
+ * tensor cores (fp32 accumulation); fp32 X and other layouts run on CUDA
+ * cores in fp32.  Asynchronous.  Accumulation order is fixed for a given
+ * (in, tokens, device), so repeated calls give identical S.
+ */
+gptq_status_t gptq_hessian_accumulate(float* S, int64_t in, const void* X,
+                                      gptq_dtype_t xt, int64_t tokens,
+                                      int64_t ldx, int64_t* n_accum,
+                                      void* stream);
+
+/*
+ * From the accumulated S (upper triangle) and token count n:
+ *   H = 2 S / n;  dead channels (H_ii == 0) get H_ii = 1;
+ *   perm = stable descending argsort of diag(H) if desc_act, else identity
+ *          ("Using AutoGPTQ in Practice", Key Parameters, desc_act);
+ *   H += damp_percent * mean(diag H) * I (same section, damp_percent);
+ *   U = upper Cholesky factor of (H[perm][:, perm])^-1, i.e. U upper
+ *       triangular with positive diagonal and U^T U = H_perm^-1 ("Using
+ *       AutoGPTQ in Practice": Cholesky factorization).
+ * Outputs (device, caller-owned):
+ *   U     fp32 in x in, COLUMN-major: element (i, j) of U at U[j*in + i].
+ *         Entries with i > j are written as 0.
+ *   perm  int32[in]: perm[p] = original column processed at position p.
+ *   dead  uint8[in], by original column: 1 if the channel never fired.
+ * ws / ws_bytes: workspace from gptq_workspace_bytes(0, in, cfg) or larger.
+ * Waits for the stream once, to read the device status word:
+ *   GPTQ_ERR_NONFINITE if S holds NaN/Inf, GPTQ_ERR_NOT_PD if a pivot of the
+ *   factorisation is not positive, GPTQ_ERR_TIMEOUT if a bounded device wait
+ *   gave up.  Only bits/group_size/sym/block_size are not used here.
+ */
+gptq_status_t gptq_prepare_hinv(const float* S, int64_t n, int64_t in,
+                                const gptq_config_t* cfg, float* U,
+                                int32_t* perm, uint8_t* dead, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/*
+ * The column sweep ("gptq" glossary page, Algorithm (2): for each weight in
+ * order, quantize it, compute the error, adjust the remaining weights with
+ * H^-1), in processing order perm, with one scale/zero per group of
+ * group_size consecutive processed columns ("gptq" agent-skill page,
+ * Group-wise quantization).  For processed column j of row r:
+ *   at a group start, scale/zero from the group's current (updated) weights;
+ *   q = clamp(rint(w / scale) + zero, 0, maxq);   deq = scale * (q - zero);
+ *   e = (w - deq) / U[j][j];   w[r][c] -= e * U[j][c] for all later c.
+ * Inputs (device): W out x in, element type wt, row stride ldw >= in, not
+ *   modified (dead columns are zeroed in the library's working copy);
+ *   U, perm, dead as written by gptq_prepare_hinv.
+ * Outputs (device, caller-owned; NULL allowed where marked):
+ *   codes    int32 out x in, original column order (NULL: skipped).
+ *   qweight  uint32 [out][in*bits/32]: row r's codes in original column
+ *            order as an LSB-first stream of bits-wide fields in
+ *            little-endian words (fields may straddle words).  Needs
+ *            (in*bits) % 32 == 0 (NULL: skipped).
+ *   scales   fp32 [out][ngroups], ngroups = in/group_size or 1 for -1;
+ *            group index in processing order.
+ *   zeros    int32 [out][ngroups], same indexing.
+ *   g_idx    int32[in]: group of original column c (0 for group_size -1).
+ *   loss     fp32[out] or NULL: sum over columns of e^2 for each row (the
+ *            quadratic error (W - deq) H (W - deq)^T with the damped H).
+ * ws / ws_bytes: workspace from gptq_workspace_bytes(out, in, cfg).
+ * Asynchronous.  out == 0 is a no-op.
+ */
+gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out,
+                                  int64_t in, int64_t ldw, const float* U,
+                                  const int32_t* perm, const uint8_t* dead,
+                                  const gptq_config_t* cfg, int32_t* codes,
+                                  uint32_t* qweight, float* scales,
+                                  int32_t* zeros, int32_t* g_idx, float* loss,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

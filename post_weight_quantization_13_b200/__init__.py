@@ -1,0 +1,204 @@
+"""Python binding of libgptq.so, the B200 GPTQ layer solver.
+
+Argument marshalling only: every step of the solve runs in the library's
+CUDA kernels.  PyTorch provides device memory and the stream.  The functions
+carry the C ABI's names (``include/gptq.h``):
+
+    gptq_hessian_accumulate(S, X, n_accum=None, stream=None)
+    gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, stream=None)
+    gptq_quantize_layer(W, U, perm, dead, cfg, scales, zeros, g_idx, ws, ...)
+
+plus ``solve_layer`` which allocates the outputs and workspace and makes the
+three calls in order.  If the shared library is missing the import fails: there
+is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+__all__ = [
+    "GptqConfig", "GptqError", "LIB_PATH", "lib", "GPTQ_OK",
+    "gptq_abi_version", "gptq_last_error", "gptq_validate_config",
+    "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
+    "gptq_quantize_layer", "solve_layer", "STATUS_NAMES",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
+
+GPTQ_OK = 0
+STATUS_NAMES = {
+    0: "GPTQ_OK", 1: "GPTQ_ERR_INVALID_ARG", 2: "GPTQ_ERR_NOT_PD",
+    3: "GPTQ_ERR_NONFINITE", 4: "GPTQ_ERR_WORKSPACE", 5: "GPTQ_ERR_CUDA",
+    6: "GPTQ_ERR_TIMEOUT", 7: "GPTQ_ERR_UNSUPPORTED",
+}
+_DTYPES = {"float16": 0, "bfloat16": 1, "float32": 2}
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with "
+        "`python -m post_weight_quantization_13_b200.build` (there is no CPU fallback)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32),
+                ("sym", ctypes.c_int32), ("desc_act", ctypes.c_int32),
+                ("damp_percent", ctypes.c_float), ("block_size", ctypes.c_int32)]
+
+
+_p = ctypes.c_void_p
+_i64 = ctypes.c_int64
+lib.gptq_abi_version.restype = ctypes.c_int
+lib.gptq_last_error.restype = ctypes.c_char_p
+lib.gptq_validate_config.argtypes = [ctypes.POINTER(_Config), _i64, _i64]
+lib.gptq_validate_config.restype = ctypes.c_int
+lib.gptq_workspace_bytes.argtypes = [_i64, _i64, ctypes.POINTER(_Config)]
+lib.gptq_workspace_bytes.restype = ctypes.c_size_t
+lib.gptq_hessian_accumulate.argtypes = [_p, _i64, _p, ctypes.c_int, _i64, _i64,
+                                        ctypes.POINTER(_i64), _p]
+lib.gptq_hessian_accumulate.restype = ctypes.c_int
+lib.gptq_prepare_hinv.argtypes = [_p, _i64, _i64, ctypes.POINTER(_Config), _p, _p, _p,
+                                  _p, ctypes.c_size_t, _p]
+lib.gptq_prepare_hinv.restype = ctypes.c_int
+lib.gptq_quantize_layer.argtypes = [_p, ctypes.c_int, _i64, _i64, _i64, _p, _p, _p,
+                                    ctypes.POINTER(_Config), _p, _p, _p, _p, _p, _p,
+                                    _p, ctypes.c_size_t, _p]
+lib.gptq_quantize_layer.restype = ctypes.c_int
+
+
+class GptqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+
+
+@dataclass
+class GptqConfig:
+    """The pages' BaseQuantizeConfig fields plus ``sym`` and ``block_size``."""
+    bits: int = 4
+    group_size: int = 128
+    sym: bool = False
+    desc_act: bool = False
+    damp_percent: float = 0.01
+    block_size: int = 128
+
+    def c(self) -> _Config:
+        return _Config(int(self.bits), int(self.group_size), int(bool(self.sym)),
+                       int(bool(self.desc_act)), float(self.damp_percent), int(self.block_size))
+
+    @classmethod
+    def of(cls, cfg) -> "GptqConfig":
+        if isinstance(cfg, GptqConfig):
+            return cfg
+        if isinstance(cfg, dict):
+            return cls(**cfg)
+        return cls(**{k: getattr(cfg, k) for k in cls.__dataclass_fields__})
+
+
+def _check(status: int):
+    if status != GPTQ_OK:
+        raise GptqError(status, lib.gptq_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dt(t) -> int:
+    name = str(t.dtype).replace("torch.", "")
+    if name not in _DTYPES:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return _DTYPES[name]
+
+
+def _rowmajor(t, name):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with contiguous rows")
+
+
+def gptq_abi_version() -> int:
+    return lib.gptq_abi_version()
+
+
+def gptq_last_error() -> str:
+    return lib.gptq_last_error().decode()
+
+
+def gptq_validate_config(cfg, out: int, in_: int) -> None:
+    c = GptqConfig.of(cfg).c()
+    _check(lib.gptq_validate_config(ctypes.byref(c), out, in_))
+
+
+def gptq_workspace_bytes(out: int, in_: int, cfg) -> int:
+    c = GptqConfig.of(cfg).c()
+    return int(lib.gptq_workspace_bytes(out, in_, ctypes.byref(c)))
+
+
+def gptq_hessian_accumulate(S, X, n_accum=None, stream=None) -> int:
+    """S (in x in fp32, upper triangle) += X X^T for X (in x tokens).
+    Returns the updated token count (n_accum + tokens)."""
+    _rowmajor(S, "S")
+    _rowmajor(X, "X")
+    n = _i64(0 if n_accum is None else int(n_accum))
+    _check(lib.gptq_hessian_accumulate(_ptr(S), S.shape[0], _ptr(X), _dt(X), X.shape[1],
+                                       X.stride(0), ctypes.byref(n), _stream(stream)))
+    return n.value
+
+
+def gptq_prepare_hinv(S, n: int, cfg, U, perm, dead, ws, stream=None) -> None:
+    c = GptqConfig.of(cfg).c()
+    _check(lib.gptq_prepare_hinv(_ptr(S), int(n), S.shape[0], ctypes.byref(c), _ptr(U),
+                                 _ptr(perm), _ptr(dead), _ptr(ws), ws.numel() * ws.element_size(),
+                                 _stream(stream)))
+
+
+def gptq_quantize_layer(W, U, perm, dead, cfg, scales, zeros, g_idx, ws, codes=None,
+                        qweight=None, loss=None, stream=None) -> None:
+    _rowmajor(W, "W")
+    c = GptqConfig.of(cfg).c()
+    _check(lib.gptq_quantize_layer(_ptr(W), _dt(W), W.shape[0], W.shape[1], W.stride(0),
+                                   _ptr(U), _ptr(perm), _ptr(dead), ctypes.byref(c),
+                                   _ptr(codes), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                                   _ptr(g_idx), _ptr(loss), _ptr(ws),
+                                   ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def solve_layer(W, X=None, cfg=None, S=None, n=None, with_codes=True, stream=None):
+    """One layer solve on the GPU: Hessian from X (or the given (S, n)),
+    prepare, quantize.  Allocates outputs and workspace with torch and
+    returns a dict of device tensors."""
+    import torch
+    cfg = GptqConfig.of(cfg or GptqConfig())
+    dev = W.device
+    out, in_ = W.shape
+    if S is None:
+        S = torch.zeros((in_, in_), dtype=torch.float32, device=dev)
+        n = gptq_hessian_accumulate(S, X, 0, stream)
+    ws = torch.empty(gptq_workspace_bytes(out, in_, cfg), dtype=torch.uint8, device=dev)
+    U = torch.empty((in_, in_), dtype=torch.float32, device=dev)
+    perm = torch.empty(in_, dtype=torch.int32, device=dev)
+    dead = torch.empty(in_, dtype=torch.uint8, device=dev)
+    gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, stream)
+    ng = 1 if cfg.group_size == -1 else in_ // cfg.group_size
+    scales = torch.empty((out, ng), dtype=torch.float32, device=dev)
+    zeros = torch.empty((out, ng), dtype=torch.int32, device=dev)
+    g_idx = torch.empty(in_, dtype=torch.int32, device=dev)
+    loss = torch.empty(out, dtype=torch.float32, device=dev)
+    codes = torch.empty((out, in_), dtype=torch.int32, device=dev) if with_codes else None
+    qweight = None
+    if (in_ * cfg.bits) % 32 == 0:
+        qweight = torch.empty((out, in_ * cfg.bits // 32), dtype=torch.int32, device=dev)
+    gptq_quantize_layer(W, U, perm, dead, cfg, scales, zeros, g_idx, ws, codes=codes,
+                        qweight=qweight, loss=loss, stream=stream)
+    return dict(S=S, n=n, U=U, perm=perm, dead=dead, scales=scales, zeros=zeros, g_idx=g_idx,
+                loss=loss, codes=codes, qweight=qweight)

@@ -1,0 +1,57 @@
+// Host-side internals shared by the library's translation units.
+#pragma once
+
+#include <cstdarg>
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace gptq {
+
+// First 256 bytes of every workspace.
+struct PrepHeader {
+  uint32_t status;  // ST_* flags OR-ed by kernels
+  float lambda;     // damping added to the diagonal
+  uint32_t pad[62];
+};
+constexpr int64_t kHeaderBytes = 256;
+static_assert(sizeof(PrepHeader) == kHeaderBytes, "header size");
+
+inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+struct DeviceInfo {
+  int id = -1;
+  int sms = 0;
+  int major = 0, minor = 0;
+};
+// Properties of the current device (cached per device).
+const DeviceInfo& device_info();
+
+// Record a message for gptq_last_error() and return s.
+gptq_status_t fail(gptq_status_t s, const char* fmt, ...);
+void clear_error();
+
+#define CUDA_TRY(x)                                                                           \
+  do {                                                                                        \
+    cudaError_t e_ = (x);                                                                     \
+    if (e_ != cudaSuccess) return ::gptq::fail(GPTQ_ERR_CUDA, "%s: %s", #x, cudaGetErrorString(e_)); \
+  } while (0)
+
+// Workspace needs of the two workspace-using calls.
+size_t prepare_ws_bytes(int64_t in);
+size_t quantize_ws_bytes(int64_t out, int64_t in, const gptq_config_t* cfg);
+
+gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_config_t* cfg, float* U,
+                           int32_t* perm, uint8_t* dead, void* ws, size_t ws_bytes, cudaStream_t st);
+gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_t in, int64_t ldw, const float* U,
+                             const int32_t* perm, const uint8_t* dead, const gptq_config_t* cfg, int32_t* codes,
+                             uint32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, float* loss, void* ws,
+                             size_t ws_bytes, cudaStream_t st);
+gptq_status_t hessian_accumulate(float* S, int64_t in, const void* X, gptq_dtype_t xt, int64_t tokens, int64_t ldx,
+                                 cudaStream_t st);
+
+// Lazy-batch width actually used for a configuration (multiple of 128,
+// compatible with group_size, at most 1024).
+int64_t outer_block(const gptq_config_t* cfg);
+
+}  // namespace gptq

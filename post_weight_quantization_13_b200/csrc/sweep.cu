@@ -1,0 +1,525 @@
+// gptq_quantize_layer: the column sweep with error compensation ("gptq"
+// glossary page, Algorithm (2) and Key innovation) and group quantization
+// ("gptq" agent-skill page, Group-wise quantization), then unpermute and
+// bit-packing.
+//
+// Data flow on the device (all in the caller's workspace):
+//   Wp   fp32 working copy of W in processing order (dead columns zeroed).
+//   U    split into tf32 hi + fp32 remainder for the tensor-core updates.
+//   for each 128-column block k:
+//     sweep_kernel   rows in parallel; the block's columns in registers
+//                    (4 lanes per row, interleaved columns), U's diagonal
+//                    block in shared memory.  For each column: group
+//                    parameters at a group start, code, error
+//                    e = (w - deq) / U_jj, eager update of the block's later
+//                    columns.  Writes codes, scales, zeros, and E (split).
+//     tc_gemm        lazy update of later columns, W -= E U_blk (3xTF32).
+//   pack_kernel      codes back to original column order, g_idx, LSB-first
+//                    bit packing.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cstdlib>
+
+#include "gemm.cuh"
+#include "internal.cuh"
+
+namespace gptq {
+namespace {
+
+constexpr int BW = 128;          // columns per sweep block
+constexpr int ROWS = 32;         // rows per sweep CTA
+constexpr int UPITCH = 36;       // floats per (j, lane) slice of U in smem
+constexpr int EPITCH = BW + 1;
+
+struct SweepParams {
+  const float* Wp;
+  int64_t ldw;  // = np_
+  int64_t out, in;
+  int64_t kB;    // first processing column of this block
+  int ncols;     // columns of this block that exist (<= 128)
+  const float* Uh;
+  const float* Ul;
+  int64_t ldu;
+  int maxq;
+  int sym;
+  int gs;         // group size (-1: one group per row)
+  int ngroups;
+  int gstart0;    // GSB == 128: a group starts at column 0 of this block
+  int gbeyond;    // GSB == 128: group columns past this block (read from Wp)
+  float* scales;
+  int32_t* zeros;
+  uint8_t* codes_p;
+  float* Eh;
+  float* El;
+  int64_t lde;
+  int64_t e_col0;
+  float* loss;
+};
+
+__device__ __forceinline__ void group_params(float lo, float hi, float amax, int sym, float fmaxq, float& s,
+                                             float& z) {
+  if (sym) {
+    const float a = amax == 0.f ? 1.f : amax;
+    s = __fdiv_rn(2.f * a, fmaxq);
+    z = (fmaxq + 1.f) * 0.5f;
+  } else {
+    lo = fminf(lo, 0.f);
+    hi = fmaxf(hi, 0.f);
+    if (lo == 0.f && hi == 0.f) {
+      lo = -1.f;
+      hi = 1.f;
+    }
+    s = __fdiv_rn(hi - lo, fmaxq);
+    z = rintf(__fdiv_rn(-lo, s));
+  }
+}
+
+template <int GSB, int J>
+struct Step {
+  template <typename Ctx>
+  static __device__ __forceinline__ void run(Ctx& c) {
+    c.template step<J>();
+    Step<GSB, J + 1>::run(c);
+  }
+};
+template <int GSB>
+struct Step<GSB, BW> {
+  template <typename Ctx>
+  static __device__ __forceinline__ void run(Ctx&) {}
+};
+
+template <int GSB>
+struct SweepCtx {
+  const SweepParams& sp;
+  float (&w)[32];
+  const float* Us;  // [128][4][UPITCH]
+  const float* rd;  // [128]
+  float* Esh;       // [ROWS][EPITCH]
+  float* Esl;
+  uint8_t* Cs;      // [ROWS][BW]
+  int64_t row;
+  int rl, lane, q;
+  float s, z, fmaxq, lsum;
+
+  template <int J>
+  __device__ __forceinline__ void step() {
+    constexpr int I = J / 4, Q = J % 4;
+    if (J >= sp.ncols) return;
+    const bool gstart = (GSB < BW) ? (J % GSB == 0) : (J == 0 && sp.gstart0);
+    if (gstart) {
+      float lo = INFINITY, hi = -INFINITY, am = 0.f;
+#pragma unroll
+      for (int i = I; i < 32; ++i) {
+        const int col = 4 * i + q;
+        const bool in_group = (GSB < BW) ? (col < J + GSB) : (col < sp.ncols);
+        if (in_group) {
+          lo = fminf(lo, w[i]);
+          hi = fmaxf(hi, w[i]);
+          am = fmaxf(am, fabsf(w[i]));
+        }
+      }
+      if (GSB == BW && sp.gbeyond > 0 && row < sp.out) {
+        const float* src = sp.Wp + row * sp.ldw + sp.kB + BW;
+        for (int cidx = q; cidx < sp.gbeyond; cidx += 4) {
+          const float v = src[cidx];
+          lo = fminf(lo, v);
+          hi = fmaxf(hi, v);
+          am = fmaxf(am, fabsf(v));
+        }
+      }
+#pragma unroll
+      for (int m = 1; m <= 2; m <<= 1) {
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, m));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, m));
+        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
+      }
+      group_params(lo, hi, am, sp.sym, fmaxq, s, z);
+      if (q == 0 && row < sp.out) {
+        const int64_t g = sp.gs == -1 ? 0 : (sp.kB + J) / sp.gs;
+        sp.scales[row * sp.ngroups + g] = s;
+        sp.zeros[row * sp.ngroups + g] = (int32_t)z;
+      }
+    }
+    float e = 0.f;
+    if (q == Q) {
+      const float x = w[I];
+      float qf = rintf(__fdiv_rn(x, s)) + z;
+      qf = fminf(fmaxf(qf, 0.f), fmaxq);
+      const float deq = s * (qf - z);
+      e = (x - deq) * rd[J];
+      lsum = fmaf(e, e, lsum);
+      Cs[rl * BW + J] = (uint8_t)qf;
+      float eh, el;
+      split_tf32(e, eh, el);
+      Esh[rl * EPITCH + J] = eh;
+      Esl[rl * EPITCH + J] = el;
+    }
+    e = __shfl_sync(0xffffffffu, e, (lane & ~3) | Q);
+    const float* urow = Us + (J * 4 + q) * UPITCH;
+#pragma unroll
+    for (int m = I / 4; m < 8; ++m) {
+      const float4 u = *reinterpret_cast<const float4*>(urow + 4 * m);
+      if (4 * m + 0 >= I) w[4 * m + 0] = fmaf(-e, u.x, w[4 * m + 0]);
+      if (4 * m + 1 >= I) w[4 * m + 1] = fmaf(-e, u.y, w[4 * m + 1]);
+      if (4 * m + 2 >= I) w[4 * m + 2] = fmaf(-e, u.z, w[4 * m + 2]);
+      if (4 * m + 3 >= I) w[4 * m + 3] = fmaf(-e, u.w, w[4 * m + 3]);
+    }
+  }
+};
+
+template <int GSB>
+__global__ void __launch_bounds__(128) sweep_kernel(const SweepParams sp) {
+  extern __shared__ __align__(16) float smf[];
+  float* Us = smf;                                 // 128 * 4 * UPITCH
+  float* rd = Us + BW * 4 * UPITCH;                // 128
+  float* Esh = rd + BW;                            // ROWS * EPITCH
+  float* Esl = Esh + ROWS * EPITCH;                // ROWS * EPITCH
+  uint8_t* Cs = reinterpret_cast<uint8_t*>(Esl + ROWS * EPITCH);  // ROWS * BW
+  const int tid = threadIdx.x;
+  // U's diagonal block: Us[j][c % 4][c / 4] = U[kB+j][kB+c] = Ucm[kB+c][kB+j]
+  for (int e = tid; e < BW * BW; e += blockDim.x) {
+    const int c = e / BW, j = e % BW;
+    float v = 0.f;
+    if (c < sp.ncols && j < sp.ncols) {
+      const int64_t g = (sp.kB + c) * sp.ldu + sp.kB + j;
+      v = sp.Uh[g] + sp.Ul[g];
+    }
+    Us[(j * 4 + (c & 3)) * UPITCH + (c >> 2)] = v;
+    if (c == j) rd[j] = (j < sp.ncols) ? 1.f / v : 0.f;
+  }
+  for (int e = tid; e < ROWS * EPITCH; e += blockDim.x) {
+    Esh[e] = 0.f;
+    Esl[e] = 0.f;
+  }
+  const int warp = tid >> 5, lane = tid & 31;
+  const int rl = warp * 8 + (lane >> 2);
+  const int q = lane & 3;
+  const int64_t row = (int64_t)blockIdx.x * ROWS + rl;
+  float w[32];
+  {
+    const float* src = sp.Wp + row * sp.ldw + sp.kB;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w[i] = (row < sp.out) ? src[4 * i + q] : 0.f;
+  }
+  __syncthreads();
+  SweepCtx<GSB> ctx{sp, w, Us, rd, Esh, Esl, Cs, row, rl, lane, q, 1.f, 0.f, (float)sp.maxq, 0.f};
+  // a group that started in an earlier block keeps that block's scale/zero
+  if (GSB == BW && !sp.gstart0 && row < sp.out) {
+    const int64_t g = sp.gs == -1 ? 0 : sp.kB / sp.gs;
+    ctx.s = sp.scales[row * sp.ngroups + g];
+    ctx.z = (float)sp.zeros[row * sp.ngroups + g];
+  }
+  Step<GSB, 0>::run(ctx);
+  float l = ctx.lsum;
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
+  if (q == 0 && row < sp.out && sp.loss) sp.loss[row] += l;
+  __syncthreads();
+  for (int e = tid; e < ROWS * BW; e += blockDim.x) {
+    const int r = e / BW, c = e % BW;
+    const int64_t gr = (int64_t)blockIdx.x * ROWS + r;
+    if (gr >= sp.out) continue;
+    sp.Eh[gr * sp.lde + sp.e_col0 + c] = Esh[r * EPITCH + c];
+    sp.El[gr * sp.lde + sp.e_col0 + c] = Esl[r * EPITCH + c];
+    if (c < sp.ncols) sp.codes_p[gr * sp.ldw + sp.kB + c] = Cs[r * BW + c];
+  }
+}
+
+// Wp[r][p] = W[r][perm[p]] (0 for dead channels and the padding).
+template <typename T>
+__global__ void __launch_bounds__(256) gather_w_kernel(const T* __restrict__ W, int64_t ldw_in, int64_t out,
+                                                       int64_t in, int64_t np_, const int32_t* __restrict__ perm,
+                                                       const uint8_t* __restrict__ dead, float* __restrict__ Wp) {
+  const int64_t r = blockIdx.y;
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < np_; p += (int64_t)gridDim.x * blockDim.x) {
+    float v = 0.f;
+    if (p < in) {
+      const int32_t c = perm[p];
+      if (!dead[c]) v = static_cast<float>(W[r * ldw_in + c]);
+    }
+    Wp[r * np_ + p] = v;
+  }
+}
+template <>
+__global__ void __launch_bounds__(256) gather_w_kernel<__half>(const __half* __restrict__ W, int64_t ldw_in,
+                                                               int64_t out, int64_t in, int64_t np_,
+                                                               const int32_t* __restrict__ perm,
+                                                               const uint8_t* __restrict__ dead,
+                                                               float* __restrict__ Wp) {
+  const int64_t r = blockIdx.y;
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < np_; p += (int64_t)gridDim.x * blockDim.x) {
+    float v = 0.f;
+    if (p < in) {
+      const int32_t c = perm[p];
+      if (!dead[c]) v = __half2float(W[r * ldw_in + c]);
+    }
+    Wp[r * np_ + p] = v;
+  }
+}
+template <>
+__global__ void __launch_bounds__(256) gather_w_kernel<__nv_bfloat16>(const __nv_bfloat16* __restrict__ W,
+                                                                      int64_t ldw_in, int64_t out, int64_t in,
+                                                                      int64_t np_, const int32_t* __restrict__ perm,
+                                                                      const uint8_t* __restrict__ dead,
+                                                                      float* __restrict__ Wp) {
+  const int64_t r = blockIdx.y;
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < np_; p += (int64_t)gridDim.x * blockDim.x) {
+    float v = 0.f;
+    if (p < in) {
+      const int32_t c = perm[p];
+      if (!dead[c]) v = __bfloat162float(W[r * ldw_in + c]);
+    }
+    Wp[r * np_ + p] = v;
+  }
+}
+
+// Uh/Ul[c][j] = split(Ucm[c][j]) with the padding zero.
+__global__ void __launch_bounds__(256) split_u_kernel(const float* __restrict__ U, int64_t in, int64_t np_,
+                                                      float* __restrict__ Uh, float* __restrict__ Ul) {
+  const int64_t c = blockIdx.y;
+  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < np_; j += (int64_t)gridDim.x * blockDim.x) {
+    const float v = (c < in && j < in) ? U[c * in + j] : 0.f;
+    float h, l;
+    split_tf32(v, h, l);
+    Uh[c * np_ + j] = h;
+    Ul[c * np_ + j] = l;
+  }
+}
+
+__global__ void invperm_kernel(const int32_t* __restrict__ perm, int64_t in, int gs, int32_t* __restrict__ inv,
+                               int32_t* __restrict__ g_idx) {
+  const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (p < in) {
+    const int32_t c = perm[p];
+    inv[c] = (int32_t)p;
+    g_idx[c] = gs == -1 ? 0 : (int32_t)(p / gs);
+  }
+}
+
+// One thread per packed word: gathers the (at most 32/bits + 1) codes whose
+// fields overlap it, in original column order.  Also writes the unpacked
+// int32 codes when requested (each column exactly once, by the word holding
+// its first bit).
+__global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ codes_p, int64_t ldc_p, int64_t out,
+                                                   int64_t in, int bits, const int32_t* __restrict__ inv,
+                                                   uint32_t* __restrict__ qweight, int32_t* __restrict__ codes) {
+  const int64_t r = blockIdx.y;
+  const int64_t nwords = (in * bits + 31) / 32;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nwords; w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t bit0 = w * 32;
+    int64_t c = bit0 / bits;
+    uint64_t acc = 0;
+    for (; c < in && c * bits < bit0 + 32; ++c) {
+      const uint32_t v = codes_p[r * ldc_p + inv[c]];
+      const int64_t off = c * bits - bit0;  // may be negative for the field straddling in
+      if (off >= 0) {
+        acc |= (uint64_t)v << off;
+        if (codes) codes[r * in + c] = (int32_t)v;
+      } else {
+        acc |= (uint64_t)v >> (-off);
+      }
+    }
+    if (qweight) qweight[r * nwords + w] = (uint32_t)acc;
+  }
+}
+
+cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
+  if (!force_simt && tc_gemm_supported(g)) return tc_gemm(g, st, sms);
+  return simt_gemm(g, st);
+}
+
+template <int GSB>
+cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st) {
+  const size_t smem = (size_t)(BW * 4 * UPITCH + BW + 2 * ROWS * EPITCH) * sizeof(float) + ROWS * BW;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(sweep_kernel<GSB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const unsigned grid = (unsigned)((sp.out + ROWS - 1) / ROWS);
+  sweep_kernel<GSB><<<grid, 128, smem, st>>>(sp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int64_t outer_block(const gptq_config_t* cfg) {
+  const int64_t gs = cfg->group_size;
+  int64_t bo = std::min<int64_t>(cfg->block_size, 1024) / 128 * 128;
+  for (; bo > 128; bo -= 128) {
+    if (gs == -1 || gs % bo == 0 || bo % gs == 0) break;
+  }
+  return std::max<int64_t>(bo, 128);
+}
+
+size_t quantize_ws_bytes(int64_t out, int64_t in, const gptq_config_t* cfg) {
+  const int64_t np_ = round_up(in, BW);
+  const int64_t bo = outer_block(cfg);
+  size_t b = kHeaderBytes;
+  b += round_up(4 * out * np_, 256);       // Wp
+  b += 2 * round_up(4 * np_ * np_, 256);   // Uh, Ul
+  b += 2 * round_up(4 * out * bo, 256);    // Eh, El
+  b += round_up(out * np_, 256);           // codes_p
+  b += round_up(4 * in, 256);              // inverse permutation
+  return b;
+}
+
+gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_t in, int64_t ldw, const float* U,
+                             const int32_t* perm, const uint8_t* dead, const gptq_config_t* cfg, int32_t* codes,
+                             uint32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, float* loss, void* ws,
+                             size_t ws_bytes, cudaStream_t st) {
+  const DeviceInfo& dev = device_info();
+  const int64_t np_ = round_up(in, BW);
+  const int64_t bo = outer_block(cfg);
+  uint8_t* p = (uint8_t*)ws;
+  PrepHeader* hdr = (PrepHeader*)p;
+  p += kHeaderBytes;
+  float* Wp = (float*)p;
+  p += round_up(4 * out * np_, 256);
+  float* Uh = (float*)p;
+  p += round_up(4 * np_ * np_, 256);
+  float* Ul = (float*)p;
+  p += round_up(4 * np_ * np_, 256);
+  float* Eh = (float*)p;
+  p += round_up(4 * out * bo, 256);
+  float* El = (float*)p;
+  p += round_up(4 * out * bo, 256);
+  uint8_t* codes_p = p;
+  p += round_up(out * np_, 256);
+  int32_t* inv = (int32_t*)p;
+  const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
+
+  CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
+  if (loss) CUDA_TRY(cudaMemsetAsync(loss, 0, sizeof(float) * out, st));
+  {
+    dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 32), (unsigned)out);
+    switch (wt) {
+      case GPTQ_F16:
+        gather_w_kernel<__half><<<grid, 256, 0, st>>>((const __half*)W, ldw, out, in, np_, perm, dead, Wp);
+        break;
+      case GPTQ_BF16:
+        gather_w_kernel<__nv_bfloat16>
+            <<<grid, 256, 0, st>>>((const __nv_bfloat16*)W, ldw, out, in, np_, perm, dead, Wp);
+        break;
+      default:
+        gather_w_kernel<float><<<grid, 256, 0, st>>>((const float*)W, ldw, out, in, np_, perm, dead, Wp);
+        break;
+    }
+    CUDA_TRY(cudaGetLastError());
+  }
+  {
+    dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 32), (unsigned)np_);
+    split_u_kernel<<<grid, 256, 0, st>>>(U, in, np_, Uh, Ul);
+    CUDA_TRY(cudaGetLastError());
+  }
+  const int gs = cfg->group_size;
+  const int ngroups = gs == -1 ? 1 : (int)(in / gs);
+  const int gsb = (gs == -1 || gs >= BW) ? BW : gs;
+  for (int64_t o0 = 0; o0 < in; o0 += bo) {
+    const int64_t o1 = std::min(in, o0 + bo);
+    for (int64_t k = o0; k < o1; k += BW) {
+      SweepParams sp;
+      sp.Wp = Wp;
+      sp.ldw = np_;
+      sp.out = out;
+      sp.in = in;
+      sp.kB = k;
+      sp.ncols = (int)std::min<int64_t>(BW, in - k);
+      sp.Uh = Uh;
+      sp.Ul = Ul;
+      sp.ldu = np_;
+      sp.maxq = (1 << cfg->bits) - 1;
+      sp.sym = cfg->sym;
+      sp.gs = gs;
+      sp.ngroups = ngroups;
+      if (gsb == BW) {
+        sp.gstart0 = (gs == -1) ? (k == 0) : (k % gs == 0);
+        const int64_t gend = (gs == -1) ? in : k + gs;
+        sp.gbeyond = sp.gstart0 ? (int)std::max<int64_t>(0, gend - (k + BW)) : 0;
+      } else {
+        sp.gstart0 = 0;
+        sp.gbeyond = 0;
+      }
+      sp.scales = scales;
+      sp.zeros = zeros;
+      sp.codes_p = codes_p;
+      sp.Eh = Eh;
+      sp.El = El;
+      sp.lde = bo;
+      sp.e_col0 = k - o0;
+      sp.loss = loss;
+      cudaError_t e;
+      switch (gsb) {
+        case 32:
+          e = launch_sweep<32>(sp, st);
+          break;
+        case 64:
+          e = launch_sweep<64>(sp, st);
+          break;
+        default:
+          e = launch_sweep<128>(sp, st);
+          break;
+      }
+      CUDA_TRY(e);
+      // inner lazy update: the rest of this outer block
+      const int64_t c0 = k + BW;
+      if (c0 < o1) {
+        GemmArgs g;
+        g.op = OP_TF32X3;
+        g.P = {Eh, El, out, bo, bo};
+        g.Q = {Uh, Ul, np_, np_, np_};
+        g.R = out;
+        g.Cn = o1 - c0;
+        g.K = BW;
+        g.p_row0 = 0;
+        g.p_k0 = k - o0;
+        g.q_row0 = c0;
+        g.q_k0 = k;
+        g.C = Wp;
+        g.ldc = np_;
+        g.c_row0 = 0;
+        g.c_col0 = c0;
+        g.alpha = -1.f;
+        g.beta = 1.f;
+        g.status = &hdr->status;
+        CUDA_TRY(run_gemm(g, st, dev.sms, force_simt));
+      }
+    }
+    // outer lazy update: every later column
+    if (o1 < in) {
+      GemmArgs g;
+      g.op = OP_TF32X3;
+      g.P = {Eh, El, out, bo, bo};
+      g.Q = {Uh, Ul, np_, np_, np_};
+      g.R = out;
+      g.Cn = in - o1;
+      g.K = o1 - o0;
+      g.p_row0 = 0;
+      g.p_k0 = 0;
+      g.q_row0 = o1;
+      g.q_k0 = o0;
+      g.C = Wp;
+      g.ldc = np_;
+      g.c_row0 = 0;
+      g.c_col0 = o1;
+      g.alpha = -1.f;
+      g.beta = 1.f;
+      g.status = &hdr->status;
+      CUDA_TRY(run_gemm(g, st, dev.sms, force_simt));
+    }
+  }
+  invperm_kernel<<<(unsigned)((in + 255) / 256), 256, 0, st>>>(perm, in, gs, inv, g_idx);
+  CUDA_TRY(cudaGetLastError());
+  if (qweight || codes) {
+    const int64_t nwords = (in * cfg->bits + 31) / 32;
+    dim3 grid((unsigned)std::min<int64_t>((nwords + 255) / 256, 32), (unsigned)out);
+    pack_kernel<<<grid, 256, 0, st>>>(codes_p, np_, out, in, cfg->bits, inv, qweight, codes);
+    CUDA_TRY(cudaGetLastError());
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

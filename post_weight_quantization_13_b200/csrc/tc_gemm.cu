@@ -1,0 +1,571 @@
+// tcgen05 tensor-core kernel for C (+)= alpha * P Q^T (see gemm.cuh).
+//
+// One persistent CTA per SM, warp-specialised:
+//   warp 0      TMA producer: fills a ring of shared-memory stages with
+//               K-major operand tiles (64-byte rows, 64-byte swizzle).
+//   warp 1      owns the tensor memory (all 512 columns) and issues
+//               tcgen05.mma from one thread; completion is signalled back to
+//               the producer (stage free) and to the epilogue (accumulator
+//               ready) through tcgen05.commit on mbarriers.
+//   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulators, then a
+//               coalesced read-modify-write of C (lane = column of C).
+//
+// The MMA shape is M = 128 (C columns, tensor-memory lanes) by N <= 256
+// (C rows, tensor-memory columns).  A CTA "round" owns up to four such
+// pieces whose accumulators fit together in the 512 tensor-memory columns.
+// Two schedules:
+//   tri   the upper triangle of a symmetric S = X X^T.  Column strip b
+//         (128 columns) needs rows [0, 128(b+1)).  All strips' rows, in
+//         16-row units, are laid end to end and cut into equal segments, one
+//         per CTA and round, so every CTA gets the same work (+-16 rows) and
+//         all CTAs stream the same k-window of X at the same time, which
+//         keeps X reads L2-resident.
+//   grid  regular 128 x 256 tiles (optionally batched), one per round, with
+//         two tensor-memory buffers so a tile's epilogue overlaps the next
+//         tile's main loop.
+// Every wait is bounded: a wait that gives up records ST_TIMEOUT in the
+// status word, stops the CTA's work, lets in-flight copies and MMAs drain
+// (bounded again), frees the tensor memory and returns.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "gemm.cuh"
+
+namespace gptq {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kMaxPieces = 4;
+constexpr int kMaxQSlots = 3;
+constexpr uint32_t kRowBytes = 64;                 // one K-major row per stage
+constexpr uint32_t kQTileBytes = 128 * kRowBytes;  // 8 KB per component
+constexpr int kTriMaxUnits = 29;                   // 464 rows per CTA round
+
+struct Piece {
+  int q0, p0, np;     // first C column, first C row, rows (multiple of 16)
+  int qslot;          // which Q tile of the stage
+  int prow;           // first row inside the stage's P region
+  int tcol;           // first tensor-memory column inside the buffer
+  int batch;
+};
+
+struct KParams {
+  int tri;
+  int kbc;                       // k-tiles per round
+  int p_row0, p_k0, q_row0, q_k0;
+  int R, Cn;
+  // grid schedule
+  int nq, npt, ntiles;
+  int64_t bs_p_row, bs_p_k, bs_q_row, bs_q_k, bs_c_row, bs_c_col;
+  // tri schedule
+  int n_in, nstrips, utot, T;
+  int grid, rounds;
+  // epilogue
+  float* C;
+  float* C_lo;
+  int64_t ldc, c_row0, c_col0;
+  float alpha, beta;
+  int mask;
+  int64_t mask_off;
+  int transpose;
+  uint32_t* status;
+  // shared-memory plan
+  int stages, stage_bytes, qslots, p_rows_max;
+};
+
+// 16-row units before strip b (every strip before the last is full).
+__host__ __device__ __forceinline__ int tri_prefix(int b) { return 4 * b * (b + 1); }
+
+__host__ __device__ int round_pieces(const KParams& kp, int cta, int round, Piece* pc) {
+  int n = 0;
+  if (kp.tri) {
+    const int s = round * kp.grid + cta;
+    int x = s * kp.T;
+    const int x1 = min(x + kp.T, kp.utot);
+    if (x >= x1) return 0;
+    int qstrip[kMaxQSlots];
+    int nslots = 0;
+    int prow = 0;
+    while (x < x1) {
+      int b = (int)((sqrtf(1.0f + (float)x) - 1.0f) * 0.5f);
+      if (b < 0) b = 0;
+      while (b + 1 < kp.nstrips && tri_prefix(b + 1) <= x) ++b;
+      while (b > 0 && tri_prefix(b) > x) --b;
+      const int send = (b == kp.nstrips - 1) ? kp.utot : tri_prefix(b + 1);
+      const int a = min(x1, send) - x;
+      const int nsplit = (a + 15) / 16;
+      const int base = a / nsplit, extra = a % nsplit;
+      int slot = -1;
+      for (int i = 0; i < nslots; ++i)
+        if (qstrip[i] == b) slot = i;
+      if (slot < 0) {
+        if (nslots == kMaxQSlots) return -1;
+        qstrip[nslots] = b;
+        slot = nslots++;
+      }
+      for (int k = 0; k < nsplit; ++k) {
+        const int u = base + (k < extra ? 1 : 0);
+        if (n == kMaxPieces) return -1;
+        pc[n].q0 = 128 * b;
+        pc[n].p0 = (x - tri_prefix(b)) * 16;
+        pc[n].np = u * 16;
+        pc[n].qslot = slot;
+        pc[n].prow = prow;
+        pc[n].tcol = prow;
+        pc[n].batch = 0;
+        prow += u * 16;
+        x += u;
+        ++n;
+      }
+    }
+    return n;
+  }
+  const int t = round * kp.grid + cta;
+  if (t >= kp.ntiles) return 0;
+  const int per = kp.nq * kp.npt;
+  const int batch = t / per;
+  const int rem = t - batch * per;
+  const int pt = rem / kp.nq;
+  const int qt = rem - pt * kp.nq;
+  pc[0].q0 = qt * 128;
+  pc[0].p0 = pt * 256;
+  int rows = min(256, kp.R - pc[0].p0);
+  pc[0].np = (rows + 15) & ~15;
+  pc[0].qslot = 0;
+  pc[0].prow = 0;
+  pc[0].tcol = 0;
+  pc[0].batch = batch;
+  return 1;
+}
+
+template <int OP>
+struct OpTraits;
+template <>
+struct OpTraits<OP_F16> {
+  static constexpr int kSplit = 1, kBK = 32, kFmt = 0;
+};
+template <>
+struct OpTraits<OP_BF16> {
+  static constexpr int kSplit = 1, kBK = 32, kFmt = 1;
+};
+template <>
+struct OpTraits<OP_TF32X3> {
+  static constexpr int kSplit = 2, kBK = 16, kFmt = 2;
+};
+
+template <int OP>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmPlo,
+                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQlo,
+                   const __grid_constant__ KParams kp) {
+  constexpr int SPLIT = OpTraits<OP>::kSplit;
+  constexpr int BK = OpTraits<OP>::kBK;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint64_t* full = (uint64_t*)(smem + (size_t)kp.stages * kp.stage_bytes);
+  uint64_t* empty = full + kp.stages;
+  uint64_t* acc_full = empty + kp.stages;  // [2]
+  uint64_t* acc_empty = acc_full + 2;      // [2]
+  uint64_t* drain = acc_empty + 2;         // [1]
+  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nbuf = kp.tri ? 1 : 2;
+  const uint32_t buf_cols = 512u / nbuf;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kp.stages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmP);
+    tma_prefetch_desc(&tmQ);
+    if (SPLIT == 2) {
+      tma_prefetch_desc(&tmPlo);
+      tma_prefetch_desc(&tmQlo);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+
+  const uint32_t q_region = (uint32_t)kp.qslots * kQTileBytes * SPLIT;
+  const uint32_t p_comp = (uint32_t)kp.p_rows_max * kRowBytes;  // one component of P region
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      Piece pc[kMaxPieces];
+      for (int round = 0; round < kp.rounds && !*abort_flag; ++round) {
+        const int npc = round_pieces(kp, blockIdx.x, round, pc);
+        if (npc <= 0) break;
+        int nslot = 0;
+        int rows = 0;
+        for (int i = 0; i < npc; ++i) {
+          nslot = max(nslot, pc[i].qslot + 1);
+          rows += pc[i].np;
+        }
+        const uint32_t bytes = (uint32_t)(nslot * kQTileBytes + rows * kRowBytes) * SPLIT;
+        for (int kb = 0; kb < kp.kbc; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1)) {
+            raise_status(kp.status, ST_TIMEOUT);
+            *abort_flag = 1;
+            break;
+          }
+          if (*abort_flag) break;
+          uint8_t* sb = smem + (size_t)stage * kp.stage_bytes;
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          int done_slots = 0;
+          for (int i = 0; i < npc; ++i) {
+            const Piece& p = pc[i];
+            const int bq = p.batch;
+            if (p.qslot >= done_slots) {  // first piece of a new Q tile
+              const int x = (int)(kp.q_k0 + bq * kp.bs_q_k) + kb * BK;
+              const int y = (int)(kp.q_row0 + bq * kp.bs_q_row) + p.q0;
+              uint8_t* dq = sb + p.qslot * kQTileBytes * SPLIT;
+              tma_load_2d(dq, &tmQ, &full[stage], x, y);
+              if (SPLIT == 2) tma_load_2d(dq + kQTileBytes, &tmQlo, &full[stage], x, y);
+              done_slots = p.qslot + 1;
+            }
+            const int x = (int)(kp.p_k0 + bq * kp.bs_p_k) + kb * BK;
+            const int y0 = (int)(kp.p_row0 + bq * kp.bs_p_row) + p.p0;
+            for (int r = 0; r < p.np; r += 16) {
+              uint8_t* dp = sb + q_region + (uint32_t)(p.prow + r) * kRowBytes;
+              tma_load_2d(dp, &tmP, &full[stage], x, y0 + r);
+              if (SPLIT == 2) tma_load_2d(dp + p_comp, &tmPlo, &full[stage], x, y0 + r);
+            }
+          }
+          if (++stage == kp.stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      Piece pc[kMaxPieces];
+      for (int round = 0; round < kp.rounds && !*abort_flag; ++round) {
+        const int npc = round_pieces(kp, blockIdx.x, round, pc);
+        if (npc <= 0) break;
+        const int buf = round % nbuf;
+        const int use = round / nbuf;
+        if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) {
+          raise_status(kp.status, ST_TIMEOUT);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t tacc = tbase + buf * buf_cols;
+        bool ok = true;
+        for (int kb = 0; kb < kp.kbc; ++kb) {
+          if (!mbar_wait(&full[stage], phase)) {
+            raise_status(kp.status, ST_TIMEOUT);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(smem + (size_t)stage * kp.stage_bytes);
+          for (int i = 0; i < npc; ++i) {
+            const Piece& p = pc[i];
+            const uint32_t idesc = make_idesc(OpTraits<OP>::kFmt, 128, (uint32_t)p.np);
+            const uint32_t qa = sb + p.qslot * kQTileBytes * SPLIT;
+            const uint32_t pb = sb + q_region + (uint32_t)p.prow * kRowBytes;
+            const uint32_t d = tacc + (uint32_t)p.tcol;
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+              const uint64_t ad = smem_desc_k_sw64(qa + kk * 32);
+              const uint64_t bd = smem_desc_k_sw64(pb + kk * 32);
+              if (SPLIT == 1) {
+                umma_f16(d, ad, bd, idesc, acc);
+              } else {
+                const uint64_t ad_lo = smem_desc_k_sw64(qa + kQTileBytes + kk * 32);
+                const uint64_t bd_lo = smem_desc_k_sw64(pb + p_comp + kk * 32);
+                umma_tf32(d, ad, bd, idesc, acc);
+                umma_tf32(d, ad, bd_lo, idesc, 1u);
+                umma_tf32(d, ad_lo, bd, idesc, 1u);
+              }
+            }
+          }
+          umma_commit(&empty[stage]);
+          if (++stage == kp.stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2-5)
+    const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
+    Piece pc[kMaxPieces];
+    for (int round = 0; round < kp.rounds; ++round) {
+      const int npc = round_pieces(kp, blockIdx.x, round, pc);
+      if (npc <= 0) break;
+      const int buf = round % nbuf;
+      const int use = round / nbuf;
+      if (!mbar_wait(&acc_full[buf], use & 1)) {
+        raise_status(kp.status, ST_TIMEOUT);
+        *abort_flag = 1;
+        break;
+      }
+      if (*abort_flag) break;
+      tc_fence_after();
+      for (int i = 0; i < npc; ++i) {
+        const Piece& p = pc[i];
+        const int c = p.q0 + quarter * 32 + lane;
+        const int64_t cr = kp.c_row0 + (int64_t)p.batch * kp.bs_c_row;
+        const int64_t cc = kp.c_col0 + (int64_t)p.batch * kp.bs_c_col;
+        const uint32_t taddr = tbase + buf * buf_cols + (uint32_t)p.tcol + ((uint32_t)(quarter * 32) << 16);
+        for (int n0 = 0; n0 < p.np; n0 += 16) {
+          float v[16];
+          tmem_ld16(taddr + (uint32_t)n0, v);
+          if (c >= kp.Cn) continue;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int r = p.p0 + n0 + j;
+            if (r >= kp.R) break;
+            if (kp.mask == 1 && (int64_t)c - r < kp.mask_off) continue;
+            if (kp.mask == 2 && (int64_t)c - r > kp.mask_off) continue;
+            const int64_t idx = kp.transpose ? (cr + c) * kp.ldc + (cc + r) : (cr + r) * kp.ldc + (cc + c);
+            float val = kp.alpha * v[j];
+            if (kp.beta != 0.f) {
+              float old = kp.C[idx];
+              if (kp.C_lo) old += kp.C_lo[idx];
+              val = fmaf(kp.beta, old, val);
+            }
+            if (kp.C_lo) {
+              float hi, lo;
+              split_tf32(val, hi, lo);
+              kp.C[idx] = hi;
+              kp.C_lo[idx] = lo;
+            } else {
+              kp.C[idx] = val;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  __syncthreads();
+  if (*abort_flag) {
+    // Let copies and MMAs that were already issued finish before the shared
+    // and tensor memory go away (both bounded).
+    if (threadIdx.x == 32) {
+      umma_commit(drain);
+      mbar_wait(drain, 0);
+    }
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer();
+      while (globaltimer() - t0 < 1000000ull) {
+      }
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld, int esize, int op,
+              int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  CUtensorMapDataType dt = op == OP_F16    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                           : op == OP_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)(ld * esize)};
+  cuuint32_t box[2] = {(cuuint32_t)(kRowBytes / esize), (cuuint32_t)box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = enc(m, dt, 2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int esize_of(int op) { return op == OP_TF32X3 ? 4 : 2; }
+int bk_of(int op) { return op == OP_TF32X3 ? 16 : 32; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+template <int OP>
+cudaError_t launch(const CUtensorMap& mp, const CUtensorMap& mpl, const CUtensorMap& mq, const CUtensorMap& mql,
+                   const KParams& kp, int grid, size_t smem, cudaStream_t st) {
+  static int configured = 0;  // the attribute is per function, set it once per process
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
+    if (e != cudaSuccess) return e;
+    configured = 1;
+  }
+  tc_gemm_kernel<OP><<<grid, kThreads, smem, st>>>(mp, mpl, mq, mql, kp);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_gemm_supported(const GemmArgs& a) {
+  const int es = esize_of(a.op);
+  const Operand* ops[2] = {&a.P, &a.Q};
+  for (const Operand* o : ops) {
+    if (!o->hi || !aligned16(o->hi) || (o->ld * es) % 16) return false;
+    if (a.op == OP_TF32X3 && (!o->lo || !aligned16(o->lo))) return false;
+    if (o->rows <= 0 || o->cols <= 0) return false;
+  }
+  if (a.tri) return a.batch == 1 && a.P.hi == a.Q.hi && a.R == a.Cn;
+  // the k range of each product must end on a k-tile or at the stored edge
+  const int bk = bk_of(a.op);
+  if (a.K % bk) {
+    for (int b = 0; b < a.batch; ++b) {
+      if (a.p_k0 + b * a.bs_p_k + a.K != a.P.cols) return false;
+      if (a.q_k0 + b * a.bs_q_k + a.K != a.Q.cols) return false;
+    }
+  }
+  return true;
+}
+
+cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
+  if (a.R <= 0 || a.Cn <= 0 || a.K <= 0 || a.batch <= 0) return cudaSuccess;
+  const int es = esize_of(a.op);
+  const int split = a.op == OP_TF32X3 ? 2 : 1;
+  CUtensorMap mp, mpl, mq, mql;
+  std::memset(&mpl, 0, sizeof(mpl));
+  std::memset(&mql, 0, sizeof(mql));
+  if (!make_map(&mp, a.P.hi, a.P.rows, a.P.cols, a.P.ld, es, a.op, 16)) return cudaErrorInvalidValue;
+  if (!make_map(&mq, a.Q.hi, a.Q.rows, a.Q.cols, a.Q.ld, es, a.op, 128)) return cudaErrorInvalidValue;
+  if (split == 2) {
+    if (!make_map(&mpl, a.P.lo, a.P.rows, a.P.cols, a.P.ld, es, a.op, 16)) return cudaErrorInvalidValue;
+    if (!make_map(&mql, a.Q.lo, a.Q.rows, a.Q.cols, a.Q.ld, es, a.op, 128)) return cudaErrorInvalidValue;
+  }
+  KParams kp;
+  std::memset(&kp, 0, sizeof(kp));
+  kp.tri = a.tri;
+  kp.kbc = (int)((a.K + bk_of(a.op) - 1) / bk_of(a.op));
+  kp.p_row0 = (int)a.p_row0;
+  kp.p_k0 = (int)a.p_k0;
+  kp.q_row0 = (int)a.q_row0;
+  kp.q_k0 = (int)a.q_k0;
+  kp.R = (int)a.R;
+  kp.Cn = (int)a.Cn;
+  kp.C = a.C;
+  kp.C_lo = a.C_lo;
+  kp.ldc = a.ldc;
+  kp.c_row0 = a.c_row0;
+  kp.c_col0 = a.c_col0;
+  kp.alpha = a.alpha;
+  kp.beta = a.beta;
+  kp.mask = a.mask;
+  kp.mask_off = a.mask_off;
+  kp.transpose = a.transpose;
+  kp.status = a.status;
+  int grid;
+  if (a.tri) {
+    const int n = (int)a.R;
+    kp.n_in = n;
+    kp.nstrips = (n + 127) / 128;
+    kp.utot = tri_prefix(kp.nstrips - 1) + (n + 15) / 16;
+    grid = num_sms;
+    int rounds = (kp.utot + grid * kTriMaxUnits - 1) / (grid * kTriMaxUnits);
+    int T = (kp.utot + grid * rounds - 1) / (grid * rounds);
+    // check the packing on the host with the same function the kernel uses
+    while (true) {
+      kp.grid = grid;
+      kp.rounds = (kp.utot + grid * T - 1) / (grid * T);
+      kp.T = T;
+      bool ok = true;
+      int slots = 1;
+      Piece pc[kMaxPieces];
+      for (int s = 0; s < grid * kp.rounds && ok; ++s) {
+        const int np = round_pieces(kp, s % grid, s / grid, pc);
+        if (np < 0) ok = false;
+        for (int i = 0; i < np; ++i) slots = std::max(slots, pc[i].qslot + 1);
+      }
+      if (ok) {
+        kp.qslots = slots;
+        break;
+      }
+      if (--T < 1) return cudaErrorInvalidValue;
+    }
+    kp.p_rows_max = kp.T * 16;
+  } else {
+    kp.nq = (int)((a.Cn + 127) / 128);
+    kp.npt = (int)((a.R + 255) / 256);
+    kp.ntiles = kp.nq * kp.npt * a.batch;
+    kp.bs_p_row = a.bs_p_row;
+    kp.bs_p_k = a.bs_p_k;
+    kp.bs_q_row = a.bs_q_row;
+    kp.bs_q_k = a.bs_q_k;
+    kp.bs_c_row = a.bs_c_row;
+    kp.bs_c_col = a.bs_c_col;
+    grid = std::min(num_sms, kp.ntiles);
+    kp.grid = grid;
+    kp.rounds = (kp.ntiles + grid - 1) / grid;
+    kp.qslots = 1;
+    kp.p_rows_max = 256;
+  }
+  kp.stage_bytes = (int)((kp.qslots * kQTileBytes + kp.p_rows_max * kRowBytes) * split);
+  kp.stage_bytes = (kp.stage_bytes + 1023) & ~1023;
+  const int budget = 232448 - 1024 - 256;
+  kp.stages = std::min(8, budget / kp.stage_bytes);
+  if (kp.stages < 2) return cudaErrorInvalidValue;
+  const size_t smem = 1024 + (size_t)kp.stages * kp.stage_bytes + 256;
+  switch (a.op) {
+    case OP_F16:
+      return launch<OP_F16>(mp, mpl, mq, mql, kp, grid, smem, st);
+    case OP_BF16:
+      return launch<OP_BF16>(mp, mpl, mq, mql, kp, grid, smem, st);
+    default:
+      return launch<OP_TF32X3>(mp, mpl, mq, mql, kp, grid, smem, st);
+  }
+}
+
+}  // namespace gptq
