@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 GPTQ layer solver.
+
+One step = one whole layer solve through the C ABI on inputs resident in HBM:
+S = 0; S += X X^T over all calibration tokens (gptq_hessian_accumulate);
+gptq_prepare_hinv; gptq_quantize_layer (codes packed, scales, zeros, g_idx).
+The metric is weights quantized per second (out * in per step), with the
+per-step split and the roofline of the dominant kernel (the Hessian SYRK on
+the tensor cores).  Inputs are seeded synthetic stand-ins for the pages'
+calibration set (128 sequences x 2048 tokens) and a Llama-7B-shaped layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the CPU oracle, timed on the host
+
+With N > 1 (torchrun, one process per GPU) every rank solves its own
+independent copy of the layer (layers are independent problems; there is no
+data-path collective): value = all ranks' weights / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ layer-solve weights/sec and ms/layer (4096×4096, 4-bit g128), % of roofline"
+UNIT = "weights/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=150)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama7b_q_proj")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str, enabled=True):
+        self.proc = None
+        self.path = None
+        if not enabled:
+            return
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 8:
+                    continue
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[4:8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+def gpu_id_for(dev):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev)
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((p.get("num_threads", 1) for p in threadpool_info()), default=1)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def oracle_setup(wl, layer, q, W, X):
+    """Untimed setup for the sampled oracle: a full-size U and perm."""
+    import numpy as np
+    import oracle as O
+    S, nt = O.hessian([np.asarray(X[:, :2048])])
+    prep = O.prepare(S, nt, q.damp_percent, q.desc_act)
+    return dict(S=S, nt=nt, U=prep["U"], perm=prep["perm"])
+
+
+def oracle_sample(wl, layer, q, W, X, setup, tokens, prep_n, rows):
+    """The float64 oracle, as it stands, on a bounded sample of one layer
+    solve, scaled to the whole layer: the Hessian over ``tokens`` tokens
+    (x all/tokens), the prepare on a ``prep_n`` x ``prep_n`` principal block
+    (x (in/prep_n)^3, its cost being cubic) and the column sweep of ``rows``
+    rows over all columns (x out/rows).  Returns (weights/s, detail)."""
+    import numpy as np
+    import oracle as O
+    n = wl.tokens
+    t0 = time.perf_counter()
+    O.hessian([np.asarray(X[:, :tokens])])
+    t_h = time.perf_counter() - t0
+    pn = min(prep_n, layer.in_)
+    t0 = time.perf_counter()
+    O.prepare(setup["S"][:pn, :pn], setup["nt"], q.damp_percent, q.desc_act)
+    t_p = time.perf_counter() - t0
+    r = min(rows, layer.out)
+    Wp = np.asarray(W[:r], dtype=np.float64)[:, setup["perm"]]
+    t0 = time.perf_counter()
+    O.sweep_blocked(Wp, setup["U"], q.bits, q.group_size, q.sym, q.block_size)
+    t_s = time.perf_counter() - t0
+    sh, sp, ss = n / tokens, (layer.in_ / pn) ** 3, layer.out / r
+    total = t_h * sh + t_p * sp + t_s * ss
+    sample = (f"Hessian over {tokens} of {n} tokens (x{sh:.0f}), prepare on a {pn}x{pn} block "
+              f"(x{sp:.0f}), sweep of {r} of {layer.out} rows (x{ss:.0f}); "
+              f"{t_h + t_p + t_s:.2f} s measured")
+    return layer.out * layer.in_ / total, dict(
+        cores=_blas_threads(), sample=sample, est_s_per_layer=total,
+        split_s=dict(hessian=t_h * sh, prepare=t_p * sp, sweep=t_s * ss))
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle (float64 numpy) on the host cores,
+    each step a bounded sample of the same layer solve."""
+    import gen
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = gen.WORKLOADS[args.workload]
+    layer = wl.layers[0]
+    q = wl.quant[0]
+    W = gen.weight(wl, layer)
+    X = gen.x_full(wl, layer.site, tokens=2048)
+    setup = oracle_setup(wl, layer, q, W, X)
+    vals, detail = [], None
+    for i in range(args.warmup + args.steps):
+        v, detail = oracle_sample(wl, layer, q, W, X, setup, tokens=512, prep_n=1024, rows=16)
+        if i >= args.warmup:
+            vals.append(v)
+    v = statistics.median(vals)
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * layer.out * layer.in_ / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": wl.name, "out": layer.out, "in": layer.in_, "tokens": wl.tokens,
+                       "bits": q.bits, "group_size": q.group_size, "desc_act": q.desc_act},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": detail["cores"], "kind": "oracle",
+                             "sample": detail["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU
+def run_ours(args):
+    import numpy as np
+    import torch
+
+    import gen
+    import post_weight_quantization_13_b200 as g
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    wl = gen.WORKLOADS[args.workload]
+    layer = wl.layers[0]
+    q = wl.quant[0]
+    cfg = g.GptqConfig(**q.as_dict())
+    out, in_ = layer.out, layer.in_
+    n_tok = wl.tokens
+
+    # inputs: generated on the host (pinned), copied once; resident in HBM
+    Wh = torch.from_numpy(gen.weight(wl, layer)).pin_memory()
+    tdt = {"float16": torch.float16, "float32": torch.float32}[wl.x_dtype]
+    Xh = torch.empty((in_, n_tok), dtype=tdt, pin_memory=True)
+    gen.x_full(wl, layer.site, out=Xh.numpy())
+    W = Wh.to(dev)
+    X = Xh.to(dev)
+    S = torch.zeros((in_, in_), dtype=torch.float32, device=dev)
+    ws = torch.empty(g.gptq_workspace_bytes(out, in_, cfg), dtype=torch.uint8, device=dev)
+    U = torch.empty((in_, in_), dtype=torch.float32, device=dev)
+    perm = torch.empty(in_, dtype=torch.int32, device=dev)
+    dead = torch.empty(in_, dtype=torch.uint8, device=dev)
+    ng = 1 if q.group_size == -1 else in_ // q.group_size
+    scales = torch.empty((out, ng), dtype=torch.float32, device=dev)
+    zeros = torch.empty((out, ng), dtype=torch.int32, device=dev)
+    g_idx = torch.empty(in_, dtype=torch.int32, device=dev)
+    qweight = torch.empty((out, in_ * q.bits // 32), dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    phase_ms = {"hessian": [], "prepare": [], "quantize": []}
+
+    def step(record=False):
+        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
+        e0.record(stream)
+        S.zero_()
+        n = g.gptq_hessian_accumulate(S, X, 0, stream)
+        e1.record(stream)
+        g.gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, stream)
+        e2.record(stream)
+        g.gptq_quantize_layer(W, U, perm, dead, cfg, scales, zeros, g_idx, ws, qweight=qweight,
+                              stream=stream)
+        e3.record(stream)
+        return (e0, e1, e2, e3) if record else None
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(gpu_id_for(local), enabled=not args.no_clocks)
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = g.gptq_kernel_launches()
+    start, end = ev(), ev()
+    marks = []
+    start.record(stream)
+    for _ in range(args.steps):
+        marks.append(step(record=True))
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    if pg:
+        pg.barrier()
+    launches = g.gptq_kernel_launches() - launches0
+    clocks = sampler.stop()
+    elapsed = start.elapsed_time(end)  # ms
+    for e0, e1, e2, e3 in marks:
+        phase_ms["hessian"].append(e0.elapsed_time(e1))
+        phase_ms["prepare"].append(e1.elapsed_time(e2))
+        phase_ms["quantize"].append(e2.elapsed_time(e3))
+    if pg:
+        t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        elapsed = float(t.item())
+    ms_step = elapsed / args.steps
+    value = world * out * in_ * args.steps / (elapsed / 1e3)
+
+    # the dominant kernel: one tcgen05 SYRK launch per step (plus S.zero_)
+    hess_ms = statistics.mean(phase_ms["hessian"])
+    flops = in_ * (in_ + 1) * n_tok
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    achieved = flops / (hess_ms / 1e3) / 1e12
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            t = json.load(f).get(f"hessian_syrk:{wl.name}")
+        traffic = t.get("bytes_per_launch") if t else None
+
+    # e2e: host buffers in, results out, every step, through the same ABI calls
+    e2e = None
+    if not args.no_e2e:
+        outs_h = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                  for t in (qweight, scales, zeros, g_idx, perm)]
+        outs_d = [qweight, scales, zeros, g_idx, perm]
+        step()
+        torch.cuda.synchronize(dev)
+        if pg:
+            pg.barrier()
+        s0, s1 = ev(), ev()
+        s0.record(stream)
+        for _ in range(args.e2e_steps):
+            X.copy_(Xh, non_blocking=True)
+            W.copy_(Wh, non_blocking=True)
+            step()
+            for h, d in zip(outs_h, outs_d):
+                h.copy_(d, non_blocking=True)
+        s1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = s0.elapsed_time(s1)
+        if pg:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in outs_d)
+        e2e = {"value": world * out * in_ * args.e2e_steps / (e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        setup = oracle_setup(wl, layer, q, Wh.numpy(), Xh.numpy())
+        v, d = oracle_sample(wl, layer, q, Wh.numpy(), Xh.numpy(), setup, tokens=4096,
+                             prep_n=layer.in_, rows=64)
+        cpu = {"value": v, "unit": UNIT, "cores": d["cores"], "kind": "oracle", "sample": d["sample"],
+               "est_s_per_layer": d["est_s_per_layer"], "split_s": d["split_s"]}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": wl.name, "out": out, "in": in_, "tokens": n_tok,
+                       "bits": q.bits, "group_size": q.group_size, "sym": q.sym,
+                       "desc_act": q.desc_act, "damp_percent": q.damp_percent,
+                       "block_size": q.block_size, "x_dtype": wl.x_dtype,
+                       "l2": f"inputs larger than L2 (X {Xh.numel() * Xh.element_size() / 2**30:.2f} GiB)",
+                       "parallelism": f"replicas x{world}"},
+            "split_ms": {k: statistics.mean(v) for k, v in phase_ms.items()},
+            "roofline": {"kernel": "tc_gemm_kernel<f16> (Hessian S += X X^T, tcgen05)",
+                         "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16)",
+                         "flops_per_launch": flops},
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -72,8 +72,9 @@ typedef enum gptq_dtype {
  * and the lazy-batch width.
  *   bits          2, 3, 4 or 8.
  *   group_size    -1 (one group per output row) or a positive divisor of in.
- *                 This build also needs 128 % group_size == 0 or
- *                 group_size % 128 == 0 (else GPTQ_ERR_UNSUPPORTED).
+ *                 This build also needs group_size >= 8 and either
+ *                 128 % group_size == 0 or group_size % 128 == 0 (else
+ *                 GPTQ_ERR_UNSUPPORTED).
  *   sym           0: asymmetric grid over [min(0, min w), max(0, max w)],
  *                    zero = rint(-lo / scale);
  *                 1: symmetric, scale = 2 max|w| / maxq, zero = (maxq+1)/2.
@@ -88,6 +89,8 @@ typedef enum gptq_dtype {
  *                 every max(128, block_size rounded down to 128) columns.
  * maxq = 2^bits - 1.  code = clamp(rint(w / scale) + zero, 0, maxq), the
  * division and rint in IEEE float32 (round half to even).
+ * Layer size limits of this build: 1 <= in <= 32768, 0 <= out <= 65535
+ * (larger layers return GPTQ_ERR_UNSUPPORTED).
  */
 typedef struct gptq_config {
   int32_t bits;
@@ -100,6 +103,11 @@ typedef struct gptq_config {
 
 /* GPTQ_ABI_VERSION of the loaded library. */
 int gptq_abi_version(void);
+
+/* Number of CUDA kernels this library has launched in this process, over
+ * all calls and threads (a diagnostic: callers can count the launches of a
+ * region by differencing two reads). */
+uint64_t gptq_kernel_launches(void);
 
 /* Message for the last error on the calling thread ("" if none).  The
  * pointer stays valid until the thread's next gptq_* call. */
@@ -131,9 +139,11 @@ size_t gptq_workspace_bytes(int64_t out, int64_t in, const gptq_config_t* cfg);
  *   tokens   >= 0; 0 is a no-op.
  *   n_accum  host pointer or NULL; *n_accum += tokens on success.
  * fp16/bf16 X with a 16-byte aligned base and (ldx * 2) % 16 == 0 runs on the
- * tensor cores (fp32 accumulation); fp32 X and other layouts run on CUDA
- * cores in fp32.  Asynchronous.  Accumulation order is fixed for a given
- * (in, tokens, device), so repeated calls give identical S.
+ * tensor cores (exact products, fp32 accumulation, drained into S every 8192
+ * tokens so the accumulation error stays near 2e-5 relative for any token
+ * count); fp32 X and other layouts run on CUDA cores in fp32.  Asynchronous.
+ * Accumulation order is fixed for a given (in, tokens, device), so repeated
+ * calls give identical S.
  */
 gptq_status_t gptq_hessian_accumulate(float* S, int64_t in, const void* X,
                                       gptq_dtype_t xt, int64_t tokens,

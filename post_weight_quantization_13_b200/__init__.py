@@ -20,7 +20,7 @@ from dataclasses import dataclass
 
 __all__ = [
     "GptqConfig", "GptqError", "LIB_PATH", "lib", "GPTQ_OK",
-    "gptq_abi_version", "gptq_last_error", "gptq_validate_config",
+    "gptq_abi_version", "gptq_last_error", "gptq_kernel_launches", "gptq_validate_config",
     "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
     "gptq_quantize_layer", "solve_layer", "STATUS_NAMES",
 ]
@@ -38,7 +38,7 @@ _DTYPES = {"float16": 0, "bfloat16": 1, "float32": 2}
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build it with "
-        "`python -m post_weight_quantization_13_b200.build` (there is no CPU fallback)")
+        "`python post_weight_quantization_13_b200/build.py` (there is no CPU fallback)")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -53,6 +53,7 @@ _p = ctypes.c_void_p
 _i64 = ctypes.c_int64
 lib.gptq_abi_version.restype = ctypes.c_int
 lib.gptq_last_error.restype = ctypes.c_char_p
+lib.gptq_kernel_launches.restype = ctypes.c_uint64
 lib.gptq_validate_config.argtypes = [ctypes.POINTER(_Config), _i64, _i64]
 lib.gptq_validate_config.restype = ctypes.c_int
 lib.gptq_workspace_bytes.argtypes = [_i64, _i64, ctypes.POINTER(_Config)]
@@ -128,6 +129,10 @@ def _rowmajor(t, name):
 
 def gptq_abi_version() -> int:
     return lib.gptq_abi_version()
+
+
+def gptq_kernel_launches() -> int:
+    return int(lib.gptq_kernel_launches())
 
 
 def gptq_last_error() -> str:

@@ -1,6 +1,9 @@
 """Build libgptq.so in-tree for sm_100a with nvcc (no torch involved).
 
-    python -m post_weight_quantization_13_b200.build [--force]
+    python post_weight_quantization_13_b200/build.py [--force]
+
+(run as a file, not as a module of the package: importing the package loads
+the library this script builds)
 
 Objects go to ``post_weight_quantization_13_b200/_build/``; the shared
 library lands next to this file.  Translation units compile in parallel and

@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -30,6 +31,11 @@ gptq_status_t fail(gptq_status_t s, const char* fmt, ...) {
 }
 
 void clear_error() { g_last_error.clear(); }
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 const DeviceInfo& device_info() {
   static DeviceInfo infos[64];
@@ -106,6 +112,8 @@ extern "C" {
 
 int gptq_abi_version(void) { return GPTQ_ABI_VERSION; }
 
+uint64_t gptq_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
 const char* gptq_last_error(void) { return g_last_error.c_str(); }
 
 gptq_status_t gptq_validate_config(const gptq_config_t* cfg, int64_t out, int64_t in) {
@@ -127,8 +135,9 @@ gptq_status_t gptq_validate_config(const gptq_config_t* cfg, int64_t out, int64_
     return fail(GPTQ_ERR_INVALID_ARG, "damp_percent must be finite and >= 0");
   if (cfg->sym != 0 && cfg->sym != 1) return fail(GPTQ_ERR_INVALID_ARG, "sym must be 0 or 1");
   if (cfg->desc_act != 0 && cfg->desc_act != 1) return fail(GPTQ_ERR_INVALID_ARG, "desc_act must be 0 or 1");
-  if (gs != -1 && gs % 128 != 0 && 128 % gs != 0)
-    return fail(GPTQ_ERR_UNSUPPORTED, "group_size %d: this build needs group_size | 128 or 128 | group_size", gs);
+  if (gs != -1 && ((gs % 128 != 0 && 128 % gs != 0) || gs < 8))
+    return fail(GPTQ_ERR_UNSUPPORTED,
+                "group_size %d: this build needs group_size >= 8 with group_size | 128 or 128 | group_size", gs);
   if (in > kMaxIn || out > kMaxOut)
     return fail(GPTQ_ERR_UNSUPPORTED, "layer %lld x %lld exceeds this build's limits (in <= %lld, out <= %lld)",
                 (long long)out, (long long)in, (long long)kMaxIn, (long long)kMaxOut);

@@ -48,6 +48,8 @@ struct GemmArgs {
   uint32_t* status = nullptr;                   // device status word (may be null)
 };
 
+void note_launch();
+
 // Returns cudaSuccess or the launch error.  Asynchronous.
 cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t stream, int num_sms);
 cudaError_t simt_gemm(const GemmArgs& a, cudaStream_t stream);

@@ -27,6 +27,9 @@ struct DeviceInfo {
 // Properties of the current device (cached per device).
 const DeviceInfo& device_info();
 
+// Process-wide count of kernels this library has launched (diagnostic).
+void note_launch();
+
 // Record a message for gptq_last_error() and return s.
 gptq_status_t fail(gptq_status_t s, const char* fmt, ...);
 void clear_error();

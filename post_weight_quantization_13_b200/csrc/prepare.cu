@@ -283,12 +283,15 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   CUDA_TRY(cudaMemsetAsync(Mh, 0, 4 * mat, st));  // M, Mt (hi, lo): strictly-off-triangle blocks stay 0
   const float scale = (float)(2.0 / (double)n);
   diag_kernel<<<1, 1024, 0, st>>>(S, in, scale, cfg->damp_percent, hd, dead, hdr);
+  note_launch();
   CUDA_TRY(cudaGetLastError());
   rank_kernel<<<(unsigned)((in + 255) / 256), 256, 0, st>>>(hd, in, cfg->desc_act, perm);
+  note_launch();
   CUDA_TRY(cudaGetLastError());
   {
     dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 16), (unsigned)np_);
     gather_kernel<<<grid, 256, 0, st>>>(S, in, np_, scale, perm, dead, hdr, Rh, Rl);
+    note_launch();
     CUDA_TRY(cudaGetLastError());
   }
   static bool leaf_cfg = false;
@@ -300,6 +303,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   const int KB = (int)(np_ / NB);
   for (int k = 0; k < KB; ++k) {
     leaf_kernel<<<1, 512, leaf_smem, st>>>(Rh, Rl, Mh, Ml, Mth, Mtl, np_, k, hdr);
+    note_launch();
     CUDA_TRY(cudaGetLastError());
     const int64_t r0 = (int64_t)(k + 1) * NB;
     const int64_t m = np_ - r0;
@@ -406,6 +410,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
       CUDA_TRY(run_gemm(b, st, dev.sms, force_simt));
       dim3 tg((unsigned)((s1 + 31) / 32), (unsigned)((s2 + 31) / 32), (unsigned)nb);
       transpose_blocks_kernel<<<tg, 256, 0, st>>>(Mh, Ml, Mth, Mtl, np_, o1, o2, s1, s2, stride);
+      note_launch();
       CUDA_TRY(cudaGetLastError());
       i = j;
     }
@@ -415,6 +420,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   {
     dim3 grid((unsigned)std::min<int64_t>((in + 255) / 256, 16), (unsigned)in);
     write_u_kernel<<<grid, 256, 0, st>>>(Mth, Mtl, np_, in, U);
+    note_launch();
     CUDA_TRY(cudaGetLastError());
   }
   uint32_t status = 0;

@@ -160,12 +160,15 @@ cudaError_t simt_gemm(const GemmArgs& a, cudaStream_t st) {
   switch (a.op) {
     case OP_F16:
       simt_gemm_kernel<__half><<<grid, 256, 0, st>>>(sp);
+      note_launch();
       break;
     case OP_BF16:
       simt_gemm_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(sp);
+      note_launch();
       break;
     default:
       simt_gemm_kernel<float><<<grid, 256, 0, st>>>(sp);
+      note_launch();
       break;
   }
   return cudaGetLastError();

@@ -341,6 +341,7 @@ cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st) {
   }
   const unsigned grid = (unsigned)((sp.out + ROWS - 1) / ROWS);
   sweep_kernel<GSB><<<grid, 128, smem, st>>>(sp);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -399,13 +400,16 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
     switch (wt) {
       case GPTQ_F16:
         gather_w_kernel<__half><<<grid, 256, 0, st>>>((const __half*)W, ldw, out, in, np_, perm, dead, Wp);
+        note_launch();
         break;
       case GPTQ_BF16:
         gather_w_kernel<__nv_bfloat16>
             <<<grid, 256, 0, st>>>((const __nv_bfloat16*)W, ldw, out, in, np_, perm, dead, Wp);
+            note_launch();
         break;
       default:
         gather_w_kernel<float><<<grid, 256, 0, st>>>((const float*)W, ldw, out, in, np_, perm, dead, Wp);
+        note_launch();
         break;
     }
     CUDA_TRY(cudaGetLastError());
@@ -413,6 +417,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
   {
     dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 32), (unsigned)np_);
     split_u_kernel<<<grid, 256, 0, st>>>(U, in, np_, Uh, Ul);
+    note_launch();
     CUDA_TRY(cudaGetLastError());
   }
   const int gs = cfg->group_size;
@@ -453,15 +458,23 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
       sp.loss = loss;
       cudaError_t e;
       switch (gsb) {
+        case 8:
+          e = launch_sweep<8>(sp, st);
+          break;
+        case 16:
+          e = launch_sweep<16>(sp, st);
+          break;
         case 32:
           e = launch_sweep<32>(sp, st);
           break;
         case 64:
           e = launch_sweep<64>(sp, st);
           break;
-        default:
+        case 128:
           e = launch_sweep<128>(sp, st);
           break;
+        default:
+          return fail(GPTQ_ERR_UNSUPPORTED, "group_size %d is not supported by the sweep kernel", gs);
       }
       CUDA_TRY(e);
       // inner lazy update: the rest of this outer block
@@ -512,11 +525,13 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
     }
   }
   invperm_kernel<<<(unsigned)((in + 255) / 256), 256, 0, st>>>(perm, in, gs, inv, g_idx);
+  note_launch();
   CUDA_TRY(cudaGetLastError());
   if (qweight || codes) {
     const int64_t nwords = (in * cfg->bits + 31) / 32;
     dim3 grid((unsigned)std::min<int64_t>((nwords + 255) / 256, 32), (unsigned)out);
     pack_kernel<<<grid, 256, 0, st>>>(codes_p, np_, out, in, cfg->bits, inv, qweight, codes);
+    note_launch();
     CUDA_TRY(cudaGetLastError());
   }
   return GPTQ_OK;

@@ -42,6 +42,7 @@ constexpr int kMaxQSlots = 3;
 constexpr uint32_t kRowBytes = 64;                 // one K-major row per stage
 constexpr uint32_t kQTileBytes = 128 * kRowBytes;  // 8 KB per component
 constexpr int kTriMaxUnits = 29;                   // 464 rows per CTA round
+constexpr int kChunkTiles = 256;                   // k-tiles per accumulator drain
 
 struct Piece {
   int q0, p0, np;     // first C column, first C row, rows (multiple of 16)
@@ -54,6 +55,7 @@ struct Piece {
 struct KParams {
   int tri;
   int kbc;                       // k-tiles per round
+  int kchunk, nchunks;           // k-tiles per accumulator drain, drains per round
   int p_row0, p_k0, q_row0, q_k0;
   int R, Cn;
   // grid schedule
@@ -267,113 +269,131 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0;
+      int step = 0;  // (round, chunk) counter: selects the accumulator buffer
       Piece pc[kMaxPieces];
-      for (int round = 0; round < kp.rounds && !*abort_flag; ++round) {
+      bool ok = true;
+      for (int round = 0; round < kp.rounds && ok && !*abort_flag; ++round) {
         const int npc = round_pieces(kp, blockIdx.x, round, pc);
         if (npc <= 0) break;
-        const int buf = round % nbuf;
-        const int use = round / nbuf;
-        if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) {
-          raise_status(kp.status, ST_TIMEOUT);
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t tacc = tbase + buf * buf_cols;
-        bool ok = true;
-        for (int kb = 0; kb < kp.kbc; ++kb) {
-          if (!mbar_wait(&full[stage], phase)) {
+        for (int ch = 0; ch < kp.nchunks && ok; ++ch, ++step) {
+          const int buf = step % nbuf;
+          const int use = step / nbuf;
+          if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) {
             raise_status(kp.status, ST_TIMEOUT);
             *abort_flag = 1;
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sb = smem_u32(smem + (size_t)stage * kp.stage_bytes);
-          for (int i = 0; i < npc; ++i) {
-            const Piece& p = pc[i];
-            const uint32_t idesc = make_idesc(OpTraits<OP>::kFmt, 128, (uint32_t)p.np);
-            const uint32_t qa = sb + p.qslot * kQTileBytes * SPLIT;
-            const uint32_t pb = sb + q_region + (uint32_t)p.prow * kRowBytes;
-            const uint32_t d = tacc + (uint32_t)p.tcol;
+          const uint32_t tacc = tbase + buf * buf_cols;
+          const int kb0 = ch * kp.kchunk;
+          const int kb1 = min(kp.kbc, kb0 + kp.kchunk);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait(&full[stage], phase)) {
+              raise_status(kp.status, ST_TIMEOUT);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sb = smem_u32(smem + (size_t)stage * kp.stage_bytes);
+            for (int i = 0; i < npc; ++i) {
+              const Piece& p = pc[i];
+              const uint32_t idesc = make_idesc(OpTraits<OP>::kFmt, 128, (uint32_t)p.np);
+              const uint32_t qa = sb + p.qslot * kQTileBytes * SPLIT;
+              const uint32_t pb = sb + q_region + (uint32_t)p.prow * kRowBytes;
+              const uint32_t d = tacc + (uint32_t)p.tcol;
 #pragma unroll
-            for (int kk = 0; kk < 2; ++kk) {
-              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-              const uint64_t ad = smem_desc_k_sw64(qa + kk * 32);
-              const uint64_t bd = smem_desc_k_sw64(pb + kk * 32);
-              if (SPLIT == 1) {
-                umma_f16(d, ad, bd, idesc, acc);
-              } else {
-                const uint64_t ad_lo = smem_desc_k_sw64(qa + kQTileBytes + kk * 32);
-                const uint64_t bd_lo = smem_desc_k_sw64(pb + p_comp + kk * 32);
-                umma_tf32(d, ad, bd, idesc, acc);
-                umma_tf32(d, ad, bd_lo, idesc, 1u);
-                umma_tf32(d, ad_lo, bd, idesc, 1u);
+              for (int kk = 0; kk < 2; ++kk) {
+                const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
+                const uint64_t ad = smem_desc_k_sw64(qa + kk * 32);
+                const uint64_t bd = smem_desc_k_sw64(pb + kk * 32);
+                if (SPLIT == 1) {
+                  umma_f16(d, ad, bd, idesc, acc);
+                } else {
+                  const uint64_t ad_lo = smem_desc_k_sw64(qa + kQTileBytes + kk * 32);
+                  const uint64_t bd_lo = smem_desc_k_sw64(pb + p_comp + kk * 32);
+                  umma_tf32(d, ad, bd, idesc, acc);
+                  umma_tf32(d, ad, bd_lo, idesc, 1u);
+                  umma_tf32(d, ad_lo, bd, idesc, 1u);
+                }
               }
             }
+            umma_commit(&empty[stage]);
+            if (++stage == kp.stages) {
+              stage = 0;
+              phase ^= 1;
+            }
           }
-          umma_commit(&empty[stage]);
-          if (++stage == kp.stages) {
-            stage = 0;
-            phase ^= 1;
-          }
+          if (!ok) break;
+          umma_commit(&acc_full[buf]);
         }
-        if (!ok) break;
-        umma_commit(&acc_full[buf]);
       }
     }
   } else {
     // ------------------------------------------------ epilogue (warps 2-5)
     const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
     Piece pc[kMaxPieces];
-    for (int round = 0; round < kp.rounds; ++round) {
+    int step = 0;
+    bool ok = true;
+    for (int round = 0; round < kp.rounds && ok; ++round) {
       const int npc = round_pieces(kp, blockIdx.x, round, pc);
       if (npc <= 0) break;
-      const int buf = round % nbuf;
-      const int use = round / nbuf;
-      if (!mbar_wait(&acc_full[buf], use & 1)) {
-        raise_status(kp.status, ST_TIMEOUT);
-        *abort_flag = 1;
-        break;
-      }
-      if (*abort_flag) break;
-      tc_fence_after();
-      for (int i = 0; i < npc; ++i) {
-        const Piece& p = pc[i];
-        const int c = p.q0 + quarter * 32 + lane;
-        const int64_t cr = kp.c_row0 + (int64_t)p.batch * kp.bs_c_row;
-        const int64_t cc = kp.c_col0 + (int64_t)p.batch * kp.bs_c_col;
-        const uint32_t taddr = tbase + buf * buf_cols + (uint32_t)p.tcol + ((uint32_t)(quarter * 32) << 16);
-        for (int n0 = 0; n0 < p.np; n0 += 16) {
-          float v[16];
-          tmem_ld16(taddr + (uint32_t)n0, v);
-          if (c >= kp.Cn) continue;
+      for (int ch = 0; ch < kp.nchunks; ++ch, ++step) {
+        const int buf = step % nbuf;
+        const int use = step / nbuf;
+        if (!mbar_wait(&acc_full[buf], use & 1)) {
+          raise_status(kp.status, ST_TIMEOUT);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the first chunk applies beta, later chunks accumulate onto C
+        const float beta = ch == 0 ? kp.beta : 1.f;
+        for (int i = 0; i < npc; ++i) {
+          const Piece& p = pc[i];
+          const int c = p.q0 + quarter * 32 + lane;
+          const int64_t cr = kp.c_row0 + (int64_t)p.batch * kp.bs_c_row;
+          const int64_t cc = kp.c_col0 + (int64_t)p.batch * kp.bs_c_col;
+          const uint32_t taddr =
+              tbase + buf * buf_cols + (uint32_t)p.tcol + ((uint32_t)(quarter * 32) << 16);
+          for (int n0 = 0; n0 < p.np; n0 += 16) {
+            float v[16];
+            tmem_ld16(taddr + (uint32_t)n0, v);
+            if (c >= kp.Cn) continue;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int r = p.p0 + n0 + j;
-            if (r >= kp.R) break;
-            if (kp.mask == 1 && (int64_t)c - r < kp.mask_off) continue;
-            if (kp.mask == 2 && (int64_t)c - r > kp.mask_off) continue;
-            const int64_t idx = kp.transpose ? (cr + c) * kp.ldc + (cc + r) : (cr + r) * kp.ldc + (cc + c);
-            float val = kp.alpha * v[j];
-            if (kp.beta != 0.f) {
-              float old = kp.C[idx];
-              if (kp.C_lo) old += kp.C_lo[idx];
-              val = fmaf(kp.beta, old, val);
-            }
-            if (kp.C_lo) {
-              float hi, lo;
-              split_tf32(val, hi, lo);
-              kp.C[idx] = hi;
-              kp.C_lo[idx] = lo;
-            } else {
-              kp.C[idx] = val;
+            for (int j = 0; j < 16; ++j) {
+              const int r = p.p0 + n0 + j;
+              if (r >= kp.R) break;
+              if (kp.mask == 1 && (int64_t)c - r < kp.mask_off) continue;
+              if (kp.mask == 2 && (int64_t)c - r > kp.mask_off) continue;
+              const int64_t idx =
+                  kp.transpose ? (cr + c) * kp.ldc + (cc + r) : (cr + r) * kp.ldc + (cc + c);
+              float val = kp.alpha * v[j];
+              if (beta != 0.f) {
+                float old = kp.C[idx];
+                if (kp.C_lo) old += kp.C_lo[idx];
+                val = fmaf(beta, old, val);
+              }
+              if (kp.C_lo) {
+                float hi, lo;
+                split_tf32(val, hi, lo);
+                kp.C[idx] = hi;
+                kp.C_lo[idx] = lo;
+              } else {
+                kp.C[idx] = val;
+              }
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
     }
   }
 
@@ -448,6 +468,7 @@ cudaError_t launch(const CUtensorMap& mp, const CUtensorMap& mpl, const CUtensor
     configured = 1;
   }
   tc_gemm_kernel<OP><<<grid, kThreads, smem, st>>>(mp, mpl, mq, mql, kp);
+  note_launch();
   return cudaGetLastError();
 }
 
@@ -490,6 +511,11 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
   std::memset(&kp, 0, sizeof(kp));
   kp.tri = a.tri;
   kp.kbc = (int)((a.K + bk_of(a.op) - 1) / bk_of(a.op));
+  // Drain the fp32 accumulators into C every kChunkTiles k-tiles: the tensor
+  // core's accumulation error grows with the number of MMAs summed in place,
+  // while C gets round-to-nearest adds.
+  kp.kchunk = std::min(kp.kbc, kChunkTiles);
+  kp.nchunks = (kp.kbc + kp.kchunk - 1) / kp.kchunk;
   kp.p_row0 = (int)a.p_row0;
   kp.p_k0 = (int)a.p_k0;
   kp.q_row0 = (int)a.q_row0;

@@ -18,8 +18,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def g():
-    from post_weight_quantization_13_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import post_weight_quantization_13_b200 as m
     return m
 

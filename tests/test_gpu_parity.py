@@ -49,7 +49,7 @@ def test_hessian_accumulate(lib, in_, tokens, dtype, seed):
     iu = np.triu_indices(in_)
     err = rel_fro(Sg[iu], ref[iu])
     assert err < 1e-3, err
-    assert err < 1e-5, err          # fp32 accumulation of exact products
+    assert err < 5e-5, err          # fp32 accumulation of exact products, <= 8192 per drain
     il = np.tril_indices(in_, -1)
     assert np.all(Sg[il] == -7.0)   # the strictly lower triangle is untouched
 
@@ -69,8 +69,8 @@ def test_hessian_chunked_equals_one_pass(lib):
     assert n == n2 == t
     iu = np.triu_indices(in_)
     ref = X64 @ X64.T
-    assert rel_fro(host(S1)[iu], ref[iu]) < 1e-5
-    assert rel_fro(host(S1)[iu], host(S2)[iu]) < 1e-5
+    assert rel_fro(host(S1)[iu], ref[iu]) < 5e-5
+    assert rel_fro(host(S1)[iu], host(S2)[iu]) < 5e-5
     # repeated calls are bitwise reproducible
     S3 = torch.zeros_like(S1)
     lib.gptq_hessian_accumulate(S3, Xd, 0)
