@@ -42,6 +42,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama7b_q_proj")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="calibration tokens (default: the workload's); smaller for profiling")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -220,6 +222,9 @@ def run_ours(args):
         pg = dist
 
     wl = gen.WORKLOADS[args.workload]
+    if args.tokens:
+        import dataclasses
+        wl = dataclasses.replace(wl, tokens=args.tokens)
     layer = wl.layers[0]
     q = wl.quant[0]
     cfg = g.GptqConfig(**q.as_dict())

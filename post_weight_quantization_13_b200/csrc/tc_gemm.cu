@@ -2,27 +2,34 @@
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: fills a ring of shared-memory stages with
-//               K-major operand tiles (64-byte rows, 64-byte swizzle).
+//               K-major operand tiles (64-byte rows, 64-byte swizzle).  Row
+//               ranges are cut into power-of-two boxes (256/128/64/32/16
+//               rows), so a stage needs only a handful of copies.
 //   warp 1      owns the tensor memory (all 512 columns) and issues
 //               tcgen05.mma from one thread; completion is signalled back to
 //               the producer (stage free) and to the epilogue (accumulator
 //               ready) through tcgen05.commit on mbarriers.
 //   warps 2-5   epilogue: tcgen05.ld of the fp32 accumulators, then a
-//               coalesced read-modify-write of C (lane = column of C).
+//               coalesced read-modify-write of C (lane = column of C), with
+//               32 loads in flight per thread.  They sleep while they wait,
+//               so they do not take issue slots from warps 0 and 1.
 //
-// The MMA shape is M = 128 (C columns, tensor-memory lanes) by N <= 256
-// (C rows, tensor-memory columns).  A CTA "round" owns up to four such
-// pieces whose accumulators fit together in the 512 tensor-memory columns.
-// Two schedules:
-//   tri   the upper triangle of a symmetric S = X X^T.  Column strip b
-//         (128 columns) needs rows [0, 128(b+1)).  All strips' rows, in
-//         16-row units, are laid end to end and cut into equal segments, one
-//         per CTA and round, so every CTA gets the same work (+-16 rows) and
-//         all CTAs stream the same k-window of X at the same time, which
-//         keeps X reads L2-resident.
+// One MMA is M = 128 (C columns = tensor-memory lanes) by N <= 256 (C rows =
+// tensor-memory columns).  A "piece" is a row range of up to 256 rows of C
+// against one or two 128-column Q tiles (two accumulators that share the P
+// tile: a 256 x N output from 256 + N operand rows per k).  Schedules:
+//   tri   the upper triangle of a symmetric S = X X^T, in 256-column
+//         super-strips; super-strip s needs rows [0, 256(s+1)).  All
+//         super-strips' rows, in 16-row units, are laid end to end and cut
+//         into equal segments, one per CTA and round: every CTA gets the
+//         same work (+-16 rows) and all CTAs stream the same k-window of X
+//         together, which keeps X L2-resident.
 //   grid  regular 128 x 256 tiles (optionally batched), one per round, with
 //         two tensor-memory buffers so a tile's epilogue overlaps the next
 //         tile's main loop.
+// Long k ranges are cut into chunks; after each chunk the accumulators are
+// drained into C with round-to-nearest adds, which bounds the error of the
+// tensor core's in-place fp32 accumulation.
 // Every wait is bounded: a wait that gives up records ST_TIMEOUT in the
 // status word, stops the CTA's work, lets in-flight copies and MMAs drain
 // (bounded again), frees the tensor memory and returns.
@@ -37,18 +44,20 @@ namespace gptq {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kMaxPieces = 4;
-constexpr int kMaxQSlots = 3;
+constexpr int kMaxPieces = 2;
 constexpr uint32_t kRowBytes = 64;                 // one K-major row per stage
 constexpr uint32_t kQTileBytes = 128 * kRowBytes;  // 8 KB per component
-constexpr int kTriMaxUnits = 29;                   // 464 rows per CTA round
-constexpr int kChunkTiles = 256;                   // k-tiles per accumulator drain
+constexpr int kTriMaxUnits = 15;                   // 240 rows x 256 columns per CTA round
+constexpr int kNumBoxes = 5;                       // P boxes of 256, 128, 64, 32, 16 rows
 
 struct Piece {
-  int q0, p0, np;     // first C column, first C row, rows (multiple of 16)
-  int qslot;          // which Q tile of the stage
-  int prow;           // first row inside the stage's P region
-  int tcol;           // first tensor-memory column inside the buffer
+  int q0;     // first C column (Q row)
+  int nh;     // 128-column halves: 1 or 2
+  int p0;     // first C row (P row)
+  int np;     // rows, multiple of 16, <= 256
+  int qslot;  // Q slot of the stage
+  int prow;   // first row inside the stage's P region
+  int tcol;   // first tensor-memory column (half h at tcol + h * np)
   int batch;
 };
 
@@ -62,7 +71,7 @@ struct KParams {
   int nq, npt, ntiles;
   int64_t bs_p_row, bs_p_k, bs_q_row, bs_q_k, bs_c_row, bs_c_col;
   // tri schedule
-  int n_in, nstrips, utot, T;
+  int n_in, nss, utot, T;
   int grid, rounds;
   // epilogue
   float* C;
@@ -74,53 +83,48 @@ struct KParams {
   int transpose;
   uint32_t* status;
   // shared-memory plan
-  int stages, stage_bytes, qslots, p_rows_max;
+  int stages, stage_bytes, qslots, slot_bytes, p_rows_max;
 };
 
-// 16-row units before strip b (every strip before the last is full).
-__host__ __device__ __forceinline__ int tri_prefix(int b) { return 4 * b * (b + 1); }
+struct TmaMaps {
+  CUtensorMap p[kNumBoxes];    // P (hi) with box heights 256, 128, 64, 32, 16
+  CUtensorMap plo[kNumBoxes];  // P remainder (3xTF32 only)
+  CUtensorMap q;               // Q (hi), 128-row boxes
+  CUtensorMap qlo;
+};
+
+// 16-row units before super-strip s (every super-strip before the last is full).
+__host__ __device__ __forceinline__ int tri_prefix(int s) { return 8 * s * (s + 1); }
 
 __host__ __device__ int round_pieces(const KParams& kp, int cta, int round, Piece* pc) {
-  int n = 0;
   if (kp.tri) {
-    const int s = round * kp.grid + cta;
-    int x = s * kp.T;
+    const int seg = round * kp.grid + cta;
+    int x = seg * kp.T;
     const int x1 = min(x + kp.T, kp.utot);
     if (x >= x1) return 0;
-    int qstrip[kMaxQSlots];
-    int nslots = 0;
-    int prow = 0;
+    int n = 0, prow = 0, tcol = 0;
     while (x < x1) {
-      int b = (int)((sqrtf(1.0f + (float)x) - 1.0f) * 0.5f);
-      if (b < 0) b = 0;
-      while (b + 1 < kp.nstrips && tri_prefix(b + 1) <= x) ++b;
-      while (b > 0 && tri_prefix(b) > x) --b;
-      const int send = (b == kp.nstrips - 1) ? kp.utot : tri_prefix(b + 1);
-      const int a = min(x1, send) - x;
-      const int nsplit = (a + 15) / 16;
-      const int base = a / nsplit, extra = a % nsplit;
-      int slot = -1;
-      for (int i = 0; i < nslots; ++i)
-        if (qstrip[i] == b) slot = i;
-      if (slot < 0) {
-        if (nslots == kMaxQSlots) return -1;
-        qstrip[nslots] = b;
-        slot = nslots++;
-      }
-      for (int k = 0; k < nsplit; ++k) {
-        const int u = base + (k < extra ? 1 : 0);
-        if (n == kMaxPieces) return -1;
-        pc[n].q0 = 128 * b;
-        pc[n].p0 = (x - tri_prefix(b)) * 16;
-        pc[n].np = u * 16;
-        pc[n].qslot = slot;
-        pc[n].prow = prow;
-        pc[n].tcol = prow;
-        pc[n].batch = 0;
-        prow += u * 16;
-        x += u;
-        ++n;
-      }
+      if (n == kMaxPieces) return -1;
+      int s = (int)((sqrtf(1.0f + 0.5f * (float)x) - 1.0f) * 0.5f);
+      if (s < 0) s = 0;
+      while (s + 1 < kp.nss && tri_prefix(s + 1) <= x) ++s;
+      while (s > 0 && tri_prefix(s) > x) --s;
+      const int send = (s == kp.nss - 1) ? kp.utot : tri_prefix(s + 1);
+      const int u = min(x1, send) - x;
+      if (u > 16) return -1;
+      Piece& p = pc[n];
+      p.q0 = 256 * s;
+      p.nh = (256 * s + 128 < kp.n_in) ? 2 : 1;
+      p.p0 = (x - tri_prefix(s)) * 16;
+      p.np = u * 16;
+      p.qslot = n;
+      p.prow = prow;
+      p.tcol = tcol;
+      p.batch = 0;
+      prow += p.np;
+      tcol += p.nh * p.np;
+      x += u;
+      ++n;
     }
     return n;
   }
@@ -131,14 +135,16 @@ __host__ __device__ int round_pieces(const KParams& kp, int cta, int round, Piec
   const int rem = t - batch * per;
   const int pt = rem / kp.nq;
   const int qt = rem - pt * kp.nq;
-  pc[0].q0 = qt * 128;
-  pc[0].p0 = pt * 256;
-  int rows = min(256, kp.R - pc[0].p0);
-  pc[0].np = (rows + 15) & ~15;
-  pc[0].qslot = 0;
-  pc[0].prow = 0;
-  pc[0].tcol = 0;
-  pc[0].batch = batch;
+  Piece& p = pc[0];
+  p.q0 = qt * 128;
+  p.nh = 1;
+  p.p0 = pt * 256;
+  const int rows = min(256, kp.R - p.p0);
+  p.np = (rows + 15) & ~15;
+  p.qslot = 0;
+  p.prow = 0;
+  p.tcol = 0;
+  p.batch = batch;
   return 1;
 }
 
@@ -157,11 +163,14 @@ struct OpTraits<OP_TF32X3> {
   static constexpr int kSplit = 2, kBK = 16, kFmt = 2;
 };
 
+__device__ __forceinline__ void abort_cta(const KParams& kp, volatile int* abort_flag) {
+  raise_status(kp.status, ST_TIMEOUT);
+  *abort_flag = 1;
+}
+
 template <int OP>
 __global__ void __launch_bounds__(kThreads, 1)
-    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmPlo,
-                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQlo,
-                   const __grid_constant__ KParams kp) {
+    tc_gemm_kernel(const __grid_constant__ TmaMaps maps, const __grid_constant__ KParams kp) {
   constexpr int SPLIT = OpTraits<OP>::kSplit;
   constexpr int BK = OpTraits<OP>::kBK;
   extern __shared__ uint8_t smem_raw[];
@@ -197,11 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmP);
-    tma_prefetch_desc(&tmQ);
+    for (int b = 0; b < kNumBoxes; ++b) tma_prefetch_desc(&maps.p[b]);
+    tma_prefetch_desc(&maps.q);
     if (SPLIT == 2) {
-      tma_prefetch_desc(&tmPlo);
-      tma_prefetch_desc(&tmQlo);
+      for (int b = 0; b < kNumBoxes; ++b) tma_prefetch_desc(&maps.plo[b]);
+      tma_prefetch_desc(&maps.qlo);
     }
   }
   tc_fence_before();
@@ -209,52 +218,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
 
-  const uint32_t q_region = (uint32_t)kp.qslots * kQTileBytes * SPLIT;
-  const uint32_t p_comp = (uint32_t)kp.p_rows_max * kRowBytes;  // one component of P region
+  const uint32_t q_region = (uint32_t)(kp.qslots * kp.slot_bytes);
+  const uint32_t p_comp = (uint32_t)kp.p_rows_max * kRowBytes;  // one component of the P region
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
       int stage = 0;
       uint32_t phase = 0;
-      Piece pc[kMaxPieces];
       for (int round = 0; round < kp.rounds && !*abort_flag; ++round) {
-        const int npc = round_pieces(kp, blockIdx.x, round, pc);
+        Piece pl[kMaxPieces];
+        const int npc = round_pieces(kp, blockIdx.x, round, pl);
         if (npc <= 0) break;
-        int nslot = 0;
-        int rows = 0;
-        for (int i = 0; i < npc; ++i) {
-          nslot = max(nslot, pc[i].qslot + 1);
-          rows += pc[i].np;
+        Piece pc[kMaxPieces];
+        uint32_t bytes = 0;
+#pragma unroll
+        for (int i = 0; i < kMaxPieces; ++i) {
+          pc[i] = pl[i];
+          if (i < npc) bytes += (uint32_t)(pc[i].nh * kQTileBytes + pc[i].np * kRowBytes) * SPLIT;
         }
-        const uint32_t bytes = (uint32_t)(nslot * kQTileBytes + rows * kRowBytes) * SPLIT;
         for (int kb = 0; kb < kp.kbc; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            raise_status(kp.status, ST_TIMEOUT);
-            *abort_flag = 1;
+            abort_cta(kp, abort_flag);
             break;
           }
           if (*abort_flag) break;
           uint8_t* sb = smem + (size_t)stage * kp.stage_bytes;
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          int done_slots = 0;
-          for (int i = 0; i < npc; ++i) {
+          uint64_t* bar = &full[stage];
+          mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+          for (int i = 0; i < kMaxPieces; ++i) {
+            if (i >= npc) break;
             const Piece& p = pc[i];
             const int bq = p.batch;
-            if (p.qslot >= done_slots) {  // first piece of a new Q tile
-              const int x = (int)(kp.q_k0 + bq * kp.bs_q_k) + kb * BK;
-              const int y = (int)(kp.q_row0 + bq * kp.bs_q_row) + p.q0;
-              uint8_t* dq = sb + p.qslot * kQTileBytes * SPLIT;
-              tma_load_2d(dq, &tmQ, &full[stage], x, y);
-              if (SPLIT == 2) tma_load_2d(dq + kQTileBytes, &tmQlo, &full[stage], x, y);
-              done_slots = p.qslot + 1;
+            const int xq = (int)(kp.q_k0 + bq * kp.bs_q_k) + kb * BK;
+            const int yq = (int)(kp.q_row0 + bq * kp.bs_q_row) + p.q0;
+            uint8_t* dq = sb + p.qslot * kp.slot_bytes;
+            for (int h = 0; h < p.nh; ++h) {
+              uint8_t* d = dq + h * kQTileBytes * SPLIT;
+              tma_load_2d(d, &maps.q, bar, xq, yq + 128 * h);
+              if (SPLIT == 2) tma_load_2d(d + kQTileBytes, &maps.qlo, bar, xq, yq + 128 * h);
             }
-            const int x = (int)(kp.p_k0 + bq * kp.bs_p_k) + kb * BK;
-            const int y0 = (int)(kp.p_row0 + bq * kp.bs_p_row) + p.p0;
-            for (int r = 0; r < p.np; r += 16) {
-              uint8_t* dp = sb + q_region + (uint32_t)(p.prow + r) * kRowBytes;
-              tma_load_2d(dp, &tmP, &full[stage], x, y0 + r);
-              if (SPLIT == 2) tma_load_2d(dp + p_comp, &tmPlo, &full[stage], x, y0 + r);
+            const int xp = (int)(kp.p_k0 + bq * kp.bs_p_k) + kb * BK;
+            const int yp = (int)(kp.p_row0 + bq * kp.bs_p_row) + p.p0;
+            int off = 0;
+#pragma unroll
+            for (int b = 0; b < kNumBoxes; ++b) {
+              const int rows = 256 >> b;
+              if (p.np & rows) {
+                uint8_t* d = sb + q_region + (uint32_t)(p.prow + off) * kRowBytes;
+                tma_load_2d(d, &maps.p[b], bar, xp, yp + off);
+                if (SPLIT == 2) tma_load_2d(d + p_comp, &maps.plo[b], bar, xp, yp + off);
+                off += rows;
+              }
             }
           }
           if (++stage == kp.stages) {
@@ -270,17 +286,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int step = 0;  // (round, chunk) counter: selects the accumulator buffer
-      Piece pc[kMaxPieces];
       bool ok = true;
       for (int round = 0; round < kp.rounds && ok && !*abort_flag; ++round) {
-        const int npc = round_pieces(kp, blockIdx.x, round, pc);
+        Piece pl[kMaxPieces];
+        const int npc = round_pieces(kp, blockIdx.x, round, pl);
         if (npc <= 0) break;
+        Piece pc[kMaxPieces];
+        uint32_t idesc[kMaxPieces];
+#pragma unroll
+        for (int i = 0; i < kMaxPieces; ++i) {
+          pc[i] = pl[i];
+          idesc[i] = make_idesc(OpTraits<OP>::kFmt, 128, (uint32_t)pc[i].np);
+        }
         for (int ch = 0; ch < kp.nchunks && ok; ++ch, ++step) {
           const int buf = step % nbuf;
           const int use = step / nbuf;
           if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) {
-            raise_status(kp.status, ST_TIMEOUT);
-            *abort_flag = 1;
+            abort_cta(kp, abort_flag);
             ok = false;
             break;
           }
@@ -290,32 +312,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kb1 = min(kp.kbc, kb0 + kp.kchunk);
           for (int kb = kb0; kb < kb1; ++kb) {
             if (!mbar_wait(&full[stage], phase)) {
-              raise_status(kp.status, ST_TIMEOUT);
-              *abort_flag = 1;
+              abort_cta(kp, abort_flag);
               ok = false;
               break;
             }
             tc_fence_after();
             const uint32_t sb = smem_u32(smem + (size_t)stage * kp.stage_bytes);
-            for (int i = 0; i < npc; ++i) {
-              const Piece& p = pc[i];
-              const uint32_t idesc = make_idesc(OpTraits<OP>::kFmt, 128, (uint32_t)p.np);
-              const uint32_t qa = sb + p.qslot * kQTileBytes * SPLIT;
-              const uint32_t pb = sb + q_region + (uint32_t)p.prow * kRowBytes;
-              const uint32_t d = tacc + (uint32_t)p.tcol;
 #pragma unroll
-              for (int kk = 0; kk < 2; ++kk) {
-                const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
-                const uint64_t ad = smem_desc_k_sw64(qa + kk * 32);
-                const uint64_t bd = smem_desc_k_sw64(pb + kk * 32);
-                if (SPLIT == 1) {
-                  umma_f16(d, ad, bd, idesc, acc);
-                } else {
-                  const uint64_t ad_lo = smem_desc_k_sw64(qa + kQTileBytes + kk * 32);
-                  const uint64_t bd_lo = smem_desc_k_sw64(pb + p_comp + kk * 32);
-                  umma_tf32(d, ad, bd, idesc, acc);
-                  umma_tf32(d, ad, bd_lo, idesc, 1u);
-                  umma_tf32(d, ad_lo, bd, idesc, 1u);
+            for (int i = 0; i < kMaxPieces; ++i) {
+              if (i >= npc) break;
+              const Piece& p = pc[i];
+              const uint32_t pb = sb + q_region + (uint32_t)p.prow * kRowBytes;
+              for (int h = 0; h < p.nh; ++h) {
+                const uint32_t qa = sb + p.qslot * kp.slot_bytes + h * kQTileBytes * SPLIT;
+                const uint32_t d = tacc + (uint32_t)(p.tcol + h * p.np);
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                  const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
+                  const uint64_t ad = smem_desc_k_sw64(qa + kk * 32);
+                  const uint64_t bd = smem_desc_k_sw64(pb + kk * 32);
+                  if (SPLIT == 1) {
+                    umma_f16(d, ad, bd, idesc[i], acc);
+                  } else {
+                    const uint64_t ad_lo = smem_desc_k_sw64(qa + kQTileBytes + kk * 32);
+                    const uint64_t bd_lo = smem_desc_k_sw64(pb + p_comp + kk * 32);
+                    umma_tf32(d, ad, bd, idesc[i], acc);
+                    umma_tf32(d, ad, bd_lo, idesc[i], 1u);
+                    umma_tf32(d, ad_lo, bd, idesc[i], 1u);
+                  }
                 }
               }
             }
@@ -333,18 +357,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------ epilogue (warps 2-5)
     const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
-    Piece pc[kMaxPieces];
     int step = 0;
     bool ok = true;
     for (int round = 0; round < kp.rounds && ok; ++round) {
+      Piece pc[kMaxPieces];
       const int npc = round_pieces(kp, blockIdx.x, round, pc);
       if (npc <= 0) break;
       for (int ch = 0; ch < kp.nchunks; ++ch, ++step) {
         const int buf = step % nbuf;
         const int use = step / nbuf;
-        if (!mbar_wait(&acc_full[buf], use & 1)) {
-          raise_status(kp.status, ST_TIMEOUT);
-          *abort_flag = 1;
+        if (!mbar_wait_sleep(&acc_full[buf], use & 1)) {
+          abort_cta(kp, abort_flag);
           ok = false;
           break;
         }
@@ -357,36 +380,71 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float beta = ch == 0 ? kp.beta : 1.f;
         for (int i = 0; i < npc; ++i) {
           const Piece& p = pc[i];
-          const int c = p.q0 + quarter * 32 + lane;
           const int64_t cr = kp.c_row0 + (int64_t)p.batch * kp.bs_c_row;
           const int64_t cc = kp.c_col0 + (int64_t)p.batch * kp.bs_c_col;
-          const uint32_t taddr =
-              tbase + buf * buf_cols + (uint32_t)p.tcol + ((uint32_t)(quarter * 32) << 16);
-          for (int n0 = 0; n0 < p.np; n0 += 16) {
-            float v[16];
-            tmem_ld16(taddr + (uint32_t)n0, v);
-            if (c >= kp.Cn) continue;
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int r = p.p0 + n0 + j;
-              if (r >= kp.R) break;
-              if (kp.mask == 1 && (int64_t)c - r < kp.mask_off) continue;
-              if (kp.mask == 2 && (int64_t)c - r > kp.mask_off) continue;
-              const int64_t idx =
-                  kp.transpose ? (cr + c) * kp.ldc + (cc + r) : (cr + r) * kp.ldc + (cc + c);
-              float val = kp.alpha * v[j];
-              if (beta != 0.f) {
-                float old = kp.C[idx];
-                if (kp.C_lo) old += kp.C_lo[idx];
-                val = fmaf(beta, old, val);
-              }
-              if (kp.C_lo) {
-                float hi, lo;
-                split_tf32(val, hi, lo);
-                kp.C[idx] = hi;
-                kp.C_lo[idx] = lo;
+          for (int h = 0; h < p.nh; ++h) {
+            const int c = p.q0 + 128 * h + quarter * 32 + lane;
+            const uint32_t taddr = tbase + buf * buf_cols + (uint32_t)(p.tcol + h * p.np) +
+                                   ((uint32_t)(quarter * 32) << 16);
+            for (int n0 = 0; n0 < p.np; n0 += 32) {
+              // 32 accumulator columns (C rows) per pass: every load of C is
+              // issued before any store so they overlap in flight.
+              float v[32];
+              if (p.np - n0 >= 32) {
+                tmem_ld32(taddr + (uint32_t)n0, v);
               } else {
-                kp.C[idx] = val;
+                float t16[16];
+                tmem_ld16(taddr + (uint32_t)n0, t16);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = t16[j];
+#pragma unroll
+                for (int j = 16; j < 32; ++j) v[j] = 0.f;
+              }
+              if (c >= kp.Cn) continue;
+              const int nn = min(32, p.np - n0);
+              const int r0 = p.p0 + n0;
+              const int64_t base =
+                  kp.transpose ? (cr + c) * kp.ldc + (cc + r0) : (cr + r0) * kp.ldc + (cc + c);
+              const int64_t stp = kp.transpose ? 1 : kp.ldc;
+              uint32_t keep = 0;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int r = r0 + j;
+                bool k = j < nn && r < kp.R;
+                if (kp.mask == 1) k = k && ((int64_t)c - r >= kp.mask_off);
+                if (kp.mask == 2) k = k && ((int64_t)c - r <= kp.mask_off);
+                keep |= (uint32_t)k << j;
+              }
+              float* __restrict__ Cp = kp.C + base;
+              float* __restrict__ Cl = kp.C_lo ? kp.C_lo + base : nullptr;
+              if (beta != 0.f) {
+                float old[32];
+#pragma unroll
+                for (int j = 0; j < 32; ++j) old[j] = ((keep >> j) & 1u) ? Cp[j * stp] : 0.f;
+                if (Cl) {
+#pragma unroll
+                  for (int j = 0; j < 32; ++j)
+                    if ((keep >> j) & 1u) old[j] += Cl[j * stp];
+                }
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = fmaf(beta, old[j], kp.alpha * v[j]);
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) v[j] = kp.alpha * v[j];
+              }
+              if (Cl) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  if (!((keep >> j) & 1u)) continue;
+                  float hi, lo;
+                  split_tf32(v[j], hi, lo);
+                  Cp[j * stp] = hi;
+                  Cl[j * stp] = lo;
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  if ((keep >> j) & 1u) Cp[j * stp] = v[j];
               }
             }
           }
@@ -459,15 +517,14 @@ int bk_of(int op) { return op == OP_TF32X3 ? 16 : 32; }
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 template <int OP>
-cudaError_t launch(const CUtensorMap& mp, const CUtensorMap& mpl, const CUtensorMap& mq, const CUtensorMap& mql,
-                   const KParams& kp, int grid, size_t smem, cudaStream_t st) {
+cudaError_t launch(const TmaMaps& maps, const KParams& kp, int grid, size_t smem, cudaStream_t st) {
   static int configured = 0;  // the attribute is per function, set it once per process
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
     if (e != cudaSuccess) return e;
     configured = 1;
   }
-  tc_gemm_kernel<OP><<<grid, kThreads, smem, st>>>(mp, mpl, mq, mql, kp);
+  tc_gemm_kernel<OP><<<grid, kThreads, smem, st>>>(maps, kp);
   note_launch();
   return cudaGetLastError();
 }
@@ -498,23 +555,26 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
   if (a.R <= 0 || a.Cn <= 0 || a.K <= 0 || a.batch <= 0) return cudaSuccess;
   const int es = esize_of(a.op);
   const int split = a.op == OP_TF32X3 ? 2 : 1;
-  CUtensorMap mp, mpl, mq, mql;
-  std::memset(&mpl, 0, sizeof(mpl));
-  std::memset(&mql, 0, sizeof(mql));
-  if (!make_map(&mp, a.P.hi, a.P.rows, a.P.cols, a.P.ld, es, a.op, 16)) return cudaErrorInvalidValue;
-  if (!make_map(&mq, a.Q.hi, a.Q.rows, a.Q.cols, a.Q.ld, es, a.op, 128)) return cudaErrorInvalidValue;
-  if (split == 2) {
-    if (!make_map(&mpl, a.P.lo, a.P.rows, a.P.cols, a.P.ld, es, a.op, 16)) return cudaErrorInvalidValue;
-    if (!make_map(&mql, a.Q.lo, a.Q.rows, a.Q.cols, a.Q.ld, es, a.op, 128)) return cudaErrorInvalidValue;
+  TmaMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  for (int b = 0; b < kNumBoxes; ++b) {
+    if (!make_map(&maps.p[b], a.P.hi, a.P.rows, a.P.cols, a.P.ld, es, a.op, 256 >> b)) return cudaErrorInvalidValue;
+    if (split == 2 && !make_map(&maps.plo[b], a.P.lo, a.P.rows, a.P.cols, a.P.ld, es, a.op, 256 >> b))
+      return cudaErrorInvalidValue;
   }
+  if (!make_map(&maps.q, a.Q.hi, a.Q.rows, a.Q.cols, a.Q.ld, es, a.op, 128)) return cudaErrorInvalidValue;
+  if (split == 2 && !make_map(&maps.qlo, a.Q.lo, a.Q.rows, a.Q.cols, a.Q.ld, es, a.op, 128))
+    return cudaErrorInvalidValue;
   KParams kp;
   std::memset(&kp, 0, sizeof(kp));
   kp.tri = a.tri;
   kp.kbc = (int)((a.K + bk_of(a.op) - 1) / bk_of(a.op));
-  // Drain the fp32 accumulators into C every kChunkTiles k-tiles: the tensor
-  // core's accumulation error grows with the number of MMAs summed in place,
-  // while C gets round-to-nearest adds.
-  kp.kchunk = std::min(kp.kbc, kChunkTiles);
+  // Drain the fp32 accumulators into C every chunk of k-tiles: the tensor
+  // core's in-place fp32 accumulation error grows with the number of MMAs
+  // summed in one accumulator, while C gets round-to-nearest adds.  32768
+  // elements of k per drain for 16-bit inputs, 4096 for 3xTF32.
+  const int chunk_tiles = split == 1 ? 1024 : 256;
+  kp.kchunk = std::min(kp.kbc, chunk_tiles);
   kp.nchunks = (kp.kbc + kp.kchunk - 1) / kp.kchunk;
   kp.p_row0 = (int)a.p_row0;
   kp.p_k0 = (int)a.p_k0;
@@ -537,30 +597,25 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
   if (a.tri) {
     const int n = (int)a.R;
     kp.n_in = n;
-    kp.nstrips = (n + 127) / 128;
-    kp.utot = tri_prefix(kp.nstrips - 1) + (n + 15) / 16;
+    kp.nss = (n + 255) / 256;
+    kp.utot = tri_prefix(kp.nss - 1) + (n + 15) / 16;
     grid = num_sms;
-    int rounds = (kp.utot + grid * kTriMaxUnits - 1) / (grid * kTriMaxUnits);
+    const int rounds = (kp.utot + grid * kTriMaxUnits - 1) / (grid * kTriMaxUnits);
     int T = (kp.utot + grid * rounds - 1) / (grid * rounds);
     // check the packing on the host with the same function the kernel uses
     while (true) {
       kp.grid = grid;
-      kp.rounds = (kp.utot + grid * T - 1) / (grid * T);
       kp.T = T;
+      kp.rounds = (kp.utot + grid * T - 1) / (grid * T);
       bool ok = true;
-      int slots = 1;
       Piece pc[kMaxPieces];
-      for (int s = 0; s < grid * kp.rounds && ok; ++s) {
-        const int np = round_pieces(kp, s % grid, s / grid, pc);
-        if (np < 0) ok = false;
-        for (int i = 0; i < np; ++i) slots = std::max(slots, pc[i].qslot + 1);
-      }
-      if (ok) {
-        kp.qslots = slots;
-        break;
-      }
+      for (int s = 0; s < grid * kp.rounds && ok; ++s)
+        if (round_pieces(kp, s % grid, s / grid, pc) < 0) ok = false;
+      if (ok) break;
       if (--T < 1) return cudaErrorInvalidValue;
     }
+    kp.qslots = kMaxPieces;
+    kp.slot_bytes = 2 * kQTileBytes * split;
     kp.p_rows_max = kp.T * 16;
   } else {
     kp.nq = (int)((a.Cn + 127) / 128);
@@ -576,9 +631,10 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
     kp.grid = grid;
     kp.rounds = (kp.ntiles + grid - 1) / grid;
     kp.qslots = 1;
+    kp.slot_bytes = kQTileBytes * split;
     kp.p_rows_max = 256;
   }
-  kp.stage_bytes = (int)((kp.qslots * kQTileBytes + kp.p_rows_max * kRowBytes) * split);
+  kp.stage_bytes = kp.qslots * kp.slot_bytes + kp.p_rows_max * (int)kRowBytes * split;
   kp.stage_bytes = (kp.stage_bytes + 1023) & ~1023;
   const int budget = 232448 - 1024 - 256;
   kp.stages = std::min(8, budget / kp.stage_bytes);
@@ -586,11 +642,11 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
   const size_t smem = 1024 + (size_t)kp.stages * kp.stage_bytes + 256;
   switch (a.op) {
     case OP_F16:
-      return launch<OP_F16>(mp, mpl, mq, mql, kp, grid, smem, st);
+      return launch<OP_F16>(maps, kp, grid, smem, st);
     case OP_BF16:
-      return launch<OP_BF16>(mp, mpl, mq, mql, kp, grid, smem, st);
+      return launch<OP_BF16>(maps, kp, grid, smem, st);
     default:
-      return launch<OP_TF32X3>(mp, mpl, mq, mql, kp, grid, smem, st);
+      return launch<OP_TF32X3>(maps, kp, grid, smem, st);
   }
 }
 
