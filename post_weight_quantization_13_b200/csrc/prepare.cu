@@ -117,87 +117,177 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
 }
 
 // ------------------------------------------------------------------ leaf
-// Factor the 128 x 128 diagonal block k of R (lower Cholesky, in place) and
-// invert it: M_kk = L_kk^-1 into M, and M_kk^T into Mt.  One CTA, 512
-// threads, both matrices in shared memory.
+// Factor the 128 x 128 diagonal block k of R (lower Cholesky) and invert the
+// factor: L_kk into R, M_kk = L_kk^-1 into M and M_kk^T into Mt (all split).
+// One CTA of 512 threads; thread (ty, tx) keeps the 8 x 4 block rows
+// [8ty, 8ty+8) x columns [4tx, 4tx+4) in registers.
+//   Cholesky, right-looking and unnormalised: at pivot j the owners of
+//   column j publish it to shared memory (double-buffered), the pivot's owner
+//   publishes 1/d_j, one barrier, then every thread applies
+//   A[r][c] -= A[r][j] A[c][j] / d_j to its elements with j < c <= r.
+//   Afterwards L[r][c] = A[r][c] / sqrt(d_c).
+//   Inverse, right-looking on B = I: at step j row j of B becomes row j of
+//   M (times 1/L_jj), is published, and rows r > j subtract L[r][j] M[j][:].
+// A pivot that is not positive raises ST_NOT_PD and is replaced by 1 so the
+// block stays finite.
 constexpr int LD = NB + 1;
 
 __global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* Mh, float* Ml, float* Mth,
                                                    float* Mtl, int64_t np_, int k, PrepHeader* hdr) {
-  extern __shared__ float sm[];
-  float* A = sm;             // [128][129]
-  float* Mi = sm + NB * LD;  // [128][129]
+  extern __shared__ float Ls[];            // [NB][LD]: L, then staging for M^T
+  __shared__ __align__(16) float colb[2][NB];  // published column (Cholesky) / row (inverse)
+  __shared__ float pinv[NB];               // 1 / d_j
+  __shared__ float rsq[NB];                // 1 / sqrt(d_j) = 1 / L_jj
+  __shared__ float dpiv[NB];               // d_j
+  const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
+  const int r0 = 8 * ty, c0 = 4 * tx;
   const int64_t o = (int64_t)k * NB;
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, c = e % NB;
-    const int64_t g = (o + i) * np_ + o + c;
-    A[i * LD + c] = Rh[g] + Rl[g];
-    Mi[i * LD + c] = 0.f;
+  float a[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t g = (o + r0 + i) * np_ + o + c0;
+    const float4 h = *reinterpret_cast<const float4*>(Rh + g);
+    const float4 l = *reinterpret_cast<const float4*>(Rl + g);
+    a[i][0] = h.x + l.x;
+    a[i][1] = h.y + l.y;
+    a[i][2] = h.z + l.z;
+    a[i][3] = h.w + l.w;
   }
-  __syncthreads();
-  // Un-normalised right-looking Cholesky: at step j every row i > j
-  // subtracts A[i][j] A[c][j] / d_j from A[i][c] (j < c <= i), d_j = A[j][j].
-  // Afterwards L[i][j] = A[i][j] / sqrt(d_j).  A pivot that is not positive
-  // raises ST_NOT_PD and is replaced by 1 so the block stays finite.
-  const int row = threadIdx.x >> 2;  // 4 threads per row
-  const int sub = threadIdx.x & 3;
-  __shared__ float piv[NB];
-  for (int j = 0; j < NB; ++j) {
-    float d = A[j * LD + j];
-    if (!(d > 0.f) || !isfinite(d)) {
-      if (threadIdx.x == 0) raise_status(&hdr->status, ST_NOT_PD);
-      d = 1.f;
+  // ---------------------------------------------------------- Cholesky
+  for (int jj = 0; jj < NB / 4; ++jj) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int j = 4 * jj + kk;
+      float* cb = colb[j & 1];
+      if (tx == jj) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (r0 + i >= j) cb[r0 + i] = a[i][kk];
+        if (ty == (j >> 3)) {
+          float d = (jj & 1) ? a[4 + kk][kk] : a[kk][kk];
+          if (!(d > 0.f) || !isfinite(d)) {
+            raise_status(&hdr->status, ST_NOT_PD);
+            d = 1.f;
+          }
+          dpiv[j] = d;
+          pinv[j] = 1.f / d;
+        }
+      }
+      __syncthreads();
+      if (r0 + 7 > j && c0 + 3 > j) {
+        const float dinv = pinv[j];
+        float cr[8], cc[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cr[i] = cb[r0 + i] * dinv;
+        const float4 c4 = *reinterpret_cast<const float4*>(cb + c0);
+        cc[0] = c4.x;
+        cc[1] = c4.y;
+        cc[2] = c4.z;
+        cc[3] = c4.w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int r = r0 + i, c = c0 + q;
+            if (r > j && c > j && c <= r) a[i][q] = fmaf(-cr[i], cc[q], a[i][q]);
+          }
+      }
     }
-    if (threadIdx.x == 0) piv[j] = d;
-    const float inv_d = 1.f / d;
-    if (row > j) {
-      const float aij = A[row * LD + j] * inv_d;
-      for (int c = j + 1 + sub; c <= row; c += 4) A[row * LD + c] -= aij * A[c * LD + j];
+  }
+  if (tid < NB) rsq[tid] = 1.f / sqrtf(dpiv[tid]);
+  __syncthreads();
+  // L[r][c] = A[r][c] / sqrt(d_c) below the diagonal, sqrt(d_r) on it
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = r0 + i, c = c0 + q;
+      float v = 0.f;
+      if (c < r) v = a[i][q] * rsq[c];
+      if (c == r) v = sqrtf(dpiv[r]);
+      a[i][q] = v;
+      Ls[r * LD + c] = v;
     }
-    __syncthreads();
-  }
-  // finalise L in place
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, c = e % NB;
-    if (c < i) A[i * LD + c] /= sqrtf(piv[c]);
-  }
   __syncthreads();
-  if (threadIdx.x < NB) A[threadIdx.x * LD + threadIdx.x] = sqrtf(piv[threadIdx.x]);
-  __syncthreads();
-  // M = L^-1, column by column, 4 threads per column.  The 8 columns of a
-  // warp run the same trip count so the shuffles stay convergent.
-  {
-    const int c = threadIdx.x >> 2;
-    const int cw = (threadIdx.x >> 5) * 8;  // first column of this warp
-    if (sub == 0) Mi[c * LD + c] = 1.f / A[c * LD + c];
-    __syncwarp();
-    for (int i = cw + 1; i < NB; ++i) {
-      float s = 0.f;
-      if (i > c)
-        for (int t = c + sub; t < i; t += 4) s = fmaf(A[i * LD + t], Mi[t * LD + c], s);
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      if (sub == 0 && i > c) Mi[i * LD + c] = -s / A[i * LD + i];
-      __syncwarp();
+  // ---------------------------------------------------------- inverse
+  float b[8][4];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) b[i][q] = (r0 + i == c0 + q) ? 1.f : 0.f;
+  for (int jj = 0; jj < NB / 4; ++jj) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int j = 4 * jj + kk;
+      float* rb = colb[j & 1];
+      if (ty == (j >> 3)) {
+        const float s = rsq[j];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float m;
+          if (jj & 1) {
+            m = b[4 + kk][q] * s;
+            b[4 + kk][q] = m;
+          } else {
+            m = b[kk][q] * s;
+            b[kk][q] = m;
+          }
+          rb[c0 + q] = m;
+        }
+      }
+      __syncthreads();
+      if (r0 + 7 > j) {
+        float lr[8], mr[4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lr[i] = Ls[(r0 + i) * LD + j];
+        const float4 m4 = *reinterpret_cast<const float4*>(rb + c0);
+        mr[0] = m4.x;
+        mr[1] = m4.y;
+        mr[2] = m4.z;
+        mr[3] = m4.w;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (r0 + i > j)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) b[i][q] = fmaf(-lr[i], mr[q], b[i][q]);
+      }
     }
   }
+  // ---------------------------------------------------------- write out
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t g = (o + r0 + i) * np_ + o + c0;
+    float4 h, l;
+    split_tf32(a[i][0], h.x, l.x);
+    split_tf32(a[i][1], h.y, l.y);
+    split_tf32(a[i][2], h.z, l.z);
+    split_tf32(a[i][3], h.w, l.w);
+    *reinterpret_cast<float4*>(Rh + g) = h;
+    *reinterpret_cast<float4*>(Rl + g) = l;
+    split_tf32(b[i][0], h.x, l.x);
+    split_tf32(b[i][1], h.y, l.y);
+    split_tf32(b[i][2], h.z, l.z);
+    split_tf32(b[i][3], h.w, l.w);
+    *reinterpret_cast<float4*>(Mh + g) = h;
+    *reinterpret_cast<float4*>(Ml + g) = l;
+  }
+  __syncthreads();  // Ls is reused for M
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) Ls[(r0 + i) * LD + c0 + q] = b[i][q];
   __syncthreads();
-  for (int e = threadIdx.x; e < NB * NB; e += blockDim.x) {
-    const int i = e / NB, c = e % NB;
-    const int64_t g = (o + i) * np_ + o + c;
-    const float l = c <= i ? A[i * LD + c] : 0.f;
-    float h, lo;
-    split_tf32(l, h, lo);
-    Rh[g] = h;
-    Rl[g] = lo;
-    const float m = c <= i ? Mi[i * LD + c] : 0.f;
-    split_tf32(m, h, lo);
-    Mh[g] = h;
-    Ml[g] = lo;
-    const float mt = i <= c ? Mi[c * LD + i] : 0.f;  // (M^T)[i][c] = M[c][i]
-    split_tf32(mt, h, lo);
-    Mth[g] = h;
-    Mtl[g] = lo;
+  // Mt[r][c] = M[c][r]
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int64_t g = (o + r0 + i) * np_ + o + c0;
+    float4 h, l;
+    split_tf32(Ls[(c0 + 0) * LD + r0 + i], h.x, l.x);
+    split_tf32(Ls[(c0 + 1) * LD + r0 + i], h.y, l.y);
+    split_tf32(Ls[(c0 + 2) * LD + r0 + i], h.z, l.z);
+    split_tf32(Ls[(c0 + 3) * LD + r0 + i], h.w, l.w);
+    *reinterpret_cast<float4*>(Mth + g) = h;
+    *reinterpret_cast<float4*>(Mtl + g) = l;
   }
 }
 
@@ -295,7 +385,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     CUDA_TRY(cudaGetLastError());
   }
   static bool leaf_cfg = false;
-  const size_t leaf_smem = 2 * NB * LD * sizeof(float);
+  const size_t leaf_smem = NB * LD * sizeof(float);
   if (!leaf_cfg) {
     CUDA_TRY(cudaFuncSetAttribute(leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)leaf_smem));
     leaf_cfg = true;

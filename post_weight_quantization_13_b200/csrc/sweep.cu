@@ -29,9 +29,13 @@ namespace gptq {
 namespace {
 
 constexpr int BW = 128;          // columns per sweep block
-constexpr int ROWS = 32;         // rows per sweep CTA
+constexpr int ROWS = 16;         // rows per sweep CTA (4 lanes per row)
+constexpr int NT = ROWS * 4;     // threads per sweep CTA
 constexpr int UPITCH = 36;       // floats per (j, lane) slice of U in smem
 constexpr int EPITCH = BW + 1;
+// interleaved diagonal block of U (BW x 4 x UPITCH floats) followed by 1/U_jj
+constexpr uint32_t kDiagBlockFloats = BW * 4 * UPITCH + BW;
+constexpr uint32_t kDiagBlockBytes = kDiagBlockFloats * 4;
 
 struct SweepParams {
   const float* Wp;
@@ -56,6 +60,8 @@ struct SweepParams {
   int64_t lde;
   int64_t e_col0;
   float* loss;
+  const float* Ud;   // this block's interleaved U tile and 1/U_jj (pack_diag_kernel)
+  uint32_t* status;
 };
 
 __device__ __forceinline__ void group_params(float lo, float hi, float amax, int sym, float fmaxq, float& s,
@@ -76,120 +82,34 @@ __device__ __forceinline__ void group_params(float lo, float hi, float amax, int
   }
 }
 
-template <int GSB, int J>
-struct Step {
-  template <typename Ctx>
-  static __device__ __forceinline__ void run(Ctx& c) {
-    c.template step<J>();
-    Step<GSB, J + 1>::run(c);
-  }
-};
+// One sweep block of BW = 128 processed columns.  Each row is handled by 4
+// lanes; lane q of a row holds the block's columns 4m + q (m = 0..31) in
+// registers w[].  The 128 columns are processed in 8 passes of 16; after a
+// pass the register window slides by 4 (w[k] <- w[k+4]), so the code of one
+// pass serves all passes (compact code, and the element being quantized is
+// always at a compile-time register index).
 template <int GSB>
-struct Step<GSB, BW> {
-  template <typename Ctx>
-  static __device__ __forceinline__ void run(Ctx&) {}
-};
-
-template <int GSB>
-struct SweepCtx {
-  const SweepParams& sp;
-  float (&w)[32];
-  const float* Us;  // [128][4][UPITCH]
-  const float* rd;  // [128]
-  float* Esh;       // [ROWS][EPITCH]
-  float* Esl;
-  uint8_t* Cs;      // [ROWS][BW]
-  int64_t row;
-  int rl, lane, q;
-  float s, z, fmaxq, lsum;
-
-  template <int J>
-  __device__ __forceinline__ void step() {
-    constexpr int I = J / 4, Q = J % 4;
-    if (J >= sp.ncols) return;
-    const bool gstart = (GSB < BW) ? (J % GSB == 0) : (J == 0 && sp.gstart0);
-    if (gstart) {
-      float lo = INFINITY, hi = -INFINITY, am = 0.f;
-#pragma unroll
-      for (int i = I; i < 32; ++i) {
-        const int col = 4 * i + q;
-        const bool in_group = (GSB < BW) ? (col < J + GSB) : (col < sp.ncols);
-        if (in_group) {
-          lo = fminf(lo, w[i]);
-          hi = fmaxf(hi, w[i]);
-          am = fmaxf(am, fabsf(w[i]));
-        }
-      }
-      if (GSB == BW && sp.gbeyond > 0 && row < sp.out) {
-        const float* src = sp.Wp + row * sp.ldw + sp.kB + BW;
-        for (int cidx = q; cidx < sp.gbeyond; cidx += 4) {
-          const float v = src[cidx];
-          lo = fminf(lo, v);
-          hi = fmaxf(hi, v);
-          am = fmaxf(am, fabsf(v));
-        }
-      }
-#pragma unroll
-      for (int m = 1; m <= 2; m <<= 1) {
-        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, m));
-        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, m));
-        am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
-      }
-      group_params(lo, hi, am, sp.sym, fmaxq, s, z);
-      if (q == 0 && row < sp.out) {
-        const int64_t g = sp.gs == -1 ? 0 : (sp.kB + J) / sp.gs;
-        sp.scales[row * sp.ngroups + g] = s;
-        sp.zeros[row * sp.ngroups + g] = (int32_t)z;
-      }
-    }
-    float e = 0.f;
-    if (q == Q) {
-      const float x = w[I];
-      float qf = rintf(__fdiv_rn(x, s)) + z;
-      qf = fminf(fmaxf(qf, 0.f), fmaxq);
-      const float deq = s * (qf - z);
-      e = (x - deq) * rd[J];
-      lsum = fmaf(e, e, lsum);
-      Cs[rl * BW + J] = (uint8_t)qf;
-      float eh, el;
-      split_tf32(e, eh, el);
-      Esh[rl * EPITCH + J] = eh;
-      Esl[rl * EPITCH + J] = el;
-    }
-    e = __shfl_sync(0xffffffffu, e, (lane & ~3) | Q);
-    const float* urow = Us + (J * 4 + q) * UPITCH;
-#pragma unroll
-    for (int m = I / 4; m < 8; ++m) {
-      const float4 u = *reinterpret_cast<const float4*>(urow + 4 * m);
-      if (4 * m + 0 >= I) w[4 * m + 0] = fmaf(-e, u.x, w[4 * m + 0]);
-      if (4 * m + 1 >= I) w[4 * m + 1] = fmaf(-e, u.y, w[4 * m + 1]);
-      if (4 * m + 2 >= I) w[4 * m + 2] = fmaf(-e, u.z, w[4 * m + 2]);
-      if (4 * m + 3 >= I) w[4 * m + 3] = fmaf(-e, u.w, w[4 * m + 3]);
-    }
-  }
-};
-
-template <int GSB>
-__global__ void __launch_bounds__(128) sweep_kernel(const SweepParams sp) {
+__global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
   extern __shared__ __align__(16) float smf[];
-  float* Us = smf;                                 // 128 * 4 * UPITCH
-  float* rd = Us + BW * 4 * UPITCH;                // 128
-  float* Esh = rd + BW;                            // ROWS * EPITCH
-  float* Esl = Esh + ROWS * EPITCH;                // ROWS * EPITCH
-  uint8_t* Cs = reinterpret_cast<uint8_t*>(Esl + ROWS * EPITCH);  // ROWS * BW
+  float* Us = smf;                                 // [128 j][4 q][UPITCH]: U[kB+j][kB+4m+q] at m
+  float* rd = Us + BW * 4 * UPITCH;                // [128] 1 / U_jj
+  float* Esh = rd + BW;                            // [ROWS][EPITCH]
+  float* Esl = Esh + ROWS * EPITCH;                // [ROWS][EPITCH]
+  uint8_t* Cs = reinterpret_cast<uint8_t*>(Esl + ROWS * EPITCH);  // [ROWS][BW]
   const int tid = threadIdx.x;
-  // U's diagonal block: Us[j][c % 4][c / 4] = U[kB+j][kB+c] = Ucm[kB+c][kB+j]
-  for (int e = tid; e < BW * BW; e += blockDim.x) {
-    const int c = e / BW, j = e % BW;
-    float v = 0.f;
-    if (c < sp.ncols && j < sp.ncols) {
-      const int64_t g = (sp.kB + c) * sp.ldu + sp.kB + j;
-      v = sp.Uh[g] + sp.Ul[g];
-    }
-    Us[(j * 4 + (c & 3)) * UPITCH + (c >> 2)] = v;
-    if (c == j) rd[j] = (j < sp.ncols) ? 1.f / v : 0.f;
+  __shared__ uint64_t ubar;
+  // U's diagonal block, already laid out for this kernel by pack_diag_kernel:
+  // one bulk copy of the interleaved block and the reciprocal diagonal.
+  if (tid == 0) {
+    mbar_init(&ubar, 1);
+    fence_mbar_init();
   }
-  for (int e = tid; e < ROWS * EPITCH; e += blockDim.x) {
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&ubar, kDiagBlockBytes);
+    bulk_load(Us, sp.Ud, kDiagBlockBytes, &ubar);
+  }
+  for (int e = tid; e < ROWS * EPITCH; e += NT) {
     Esh[e] = 0.f;
     Esl[e] = 0.f;
   }
@@ -197,27 +117,110 @@ __global__ void __launch_bounds__(128) sweep_kernel(const SweepParams sp) {
   const int rl = warp * 8 + (lane >> 2);
   const int q = lane & 3;
   const int64_t row = (int64_t)blockIdx.x * ROWS + rl;
+  const bool live = row < sp.out;
   float w[32];
   {
     const float* src = sp.Wp + row * sp.ldw + sp.kB;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) w[i] = (row < sp.out) ? src[4 * i + q] : 0.f;
+    for (int i = 0; i < 32; ++i) w[i] = live ? src[4 * i + q] : 0.f;
+  }
+  const float fmaxq = (float)sp.maxq;
+  float s = 1.f, z = 0.f, lsum = 0.f;
+  if (!mbar_wait(&ubar, 0)) raise_status(sp.status, ST_TIMEOUT);
+  // a group that started in an earlier block keeps that block's scale/zero
+  if (GSB == BW && !sp.gstart0 && live) {
+    const int64_t g = sp.gs == -1 ? 0 : sp.kB / sp.gs;
+    s = sp.scales[row * sp.ngroups + g];
+    z = (float)sp.zeros[row * sp.ngroups + g];
   }
   __syncthreads();
-  SweepCtx<GSB> ctx{sp, w, Us, rd, Esh, Esl, Cs, row, rl, lane, q, 1.f, 0.f, (float)sp.maxq, 0.f};
-  // a group that started in an earlier block keeps that block's scale/zero
-  if (GSB == BW && !sp.gstart0 && row < sp.out) {
-    const int64_t g = sp.gs == -1 ? 0 : sp.kB / sp.gs;
-    ctx.s = sp.scales[row * sp.ngroups + g];
-    ctx.z = (float)sp.zeros[row * sp.ngroups + g];
+  for (int mo = 0; mo < 32; mo += 4) {  // pass: columns 4*mo .. 4*mo + 15
+    if (4 * mo >= sp.ncols) break;
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi) {
+      const int cbase = 4 * (mo + mi);
+      if (cbase >= sp.ncols) break;
+      const bool gstart = (GSB < BW) ? (cbase % GSB == 0) : (cbase == 0 && sp.gstart0);
+      if (gstart) {
+        float lo = INFINITY, hi = -INFINITY, am = 0.f;
+#pragma unroll
+        for (int k = mi; k < 32; ++k) {
+          bool in_group;
+          if (GSB < BW)
+            in_group = k < mi + GSB / 4;
+          else
+            in_group = 4 * k + q < sp.ncols;  // pass 0: element k is column 4k + q
+          if (in_group) {
+            lo = fminf(lo, w[k]);
+            hi = fmaxf(hi, w[k]);
+            am = fmaxf(am, fabsf(w[k]));
+          }
+        }
+        if (GSB == BW && sp.gbeyond > 0 && live) {
+          const float* src = sp.Wp + row * sp.ldw + sp.kB + BW;
+          for (int ci = q; ci < sp.gbeyond; ci += 4) {
+            const float v = src[ci];
+            lo = fminf(lo, v);
+            hi = fmaxf(hi, v);
+            am = fmaxf(am, fabsf(v));
+          }
+        }
+#pragma unroll
+        for (int m = 1; m <= 2; m <<= 1) {
+          lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, m));
+          hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, m));
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
+        }
+        group_params(lo, hi, am, sp.sym, fmaxq, s, z);
+        if (q == 0 && live) {
+          const int64_t g = sp.gs == -1 ? 0 : (sp.kB + cbase) / sp.gs;
+          sp.scales[row * sp.ngroups + g] = s;
+          sp.zeros[row * sp.ngroups + g] = (int32_t)z;
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int j = cbase + t;
+        if (j >= sp.ncols) break;
+        float e = 0.f;
+        if (q == t) {
+          const float x = w[mi];
+          float qf = rintf(__fdiv_rn(x, s)) + z;
+          qf = fminf(fmaxf(qf, 0.f), fmaxq);
+          const float deq = s * (qf - z);
+          e = (x - deq) * rd[j];
+          lsum = fmaf(e, e, lsum);
+          Cs[rl * BW + j] = (uint8_t)qf;
+          float eh, el;
+          split_tf32(e, eh, el);
+          Esh[rl * EPITCH + j] = eh;
+          Esl[rl * EPITCH + j] = el;
+        }
+        e = __shfl_sync(0xffffffffu, e, (lane & ~3) | t);
+        // w[k] is column 4(mo + k) + q; its U entry is Us[j][q][mo + k]
+        const float* urow = Us + (j * 4 + q) * UPITCH + mo;
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+          const float4 u = *reinterpret_cast<const float4*>(urow + 4 * a);
+          if (4 * a + 0 >= mi) w[4 * a + 0] = fmaf(-e, u.x, w[4 * a + 0]);
+          if (4 * a + 1 >= mi) w[4 * a + 1] = fmaf(-e, u.y, w[4 * a + 1]);
+          if (4 * a + 2 >= mi) w[4 * a + 2] = fmaf(-e, u.z, w[4 * a + 2]);
+          if (4 * a + 3 >= mi) w[4 * a + 3] = fmaf(-e, u.w, w[4 * a + 3]);
+        }
+      }
+    }
+    // slide the register window by one pass
+#pragma unroll
+    for (int k = 0; k < 28; ++k) w[k] = w[k + 4];
+#pragma unroll
+    for (int k = 28; k < 32; ++k) w[k] = 0.f;
   }
-  Step<GSB, 0>::run(ctx);
-  float l = ctx.lsum;
+  float l = lsum;
   l += __shfl_xor_sync(0xffffffffu, l, 1);
   l += __shfl_xor_sync(0xffffffffu, l, 2);
-  if (q == 0 && row < sp.out && sp.loss) sp.loss[row] += l;
+  if (q == 0 && live && sp.loss) sp.loss[row] += l;
   __syncthreads();
-  for (int e = tid; e < ROWS * BW; e += blockDim.x) {
+  for (int e = tid; e < ROWS * BW; e += NT) {
     const int r = e / BW, c = e % BW;
     const int64_t gr = (int64_t)blockIdx.x * ROWS + r;
     if (gr >= sp.out) continue;
@@ -225,6 +228,27 @@ __global__ void __launch_bounds__(128) sweep_kernel(const SweepParams sp) {
     sp.El[gr * sp.lde + sp.e_col0 + c] = Esl[r * EPITCH + c];
     if (c < sp.ncols) sp.codes_p[gr * sp.ldw + sp.kB + c] = Cs[r * BW + c];
   }
+}
+
+// For every 128-column block k: Ud[k] = U's diagonal block in the sweep
+// kernel's layout, Us[j][c % 4][c / 4] = U[kB+j][kB+c] (= Ucm[kB+c][kB+j]),
+// then 1/U_jj.  One CTA per block.
+__global__ void __launch_bounds__(256) pack_diag_kernel(const float* __restrict__ U, int64_t in,
+                                                        float* __restrict__ Ud) {
+  const int64_t kB = (int64_t)blockIdx.x * BW;
+  const int ncols = (int)((in - kB) < BW ? (in - kB) : BW);
+  float* dst = Ud + (int64_t)blockIdx.x * kDiagBlockFloats;
+  for (int e = threadIdx.x; e < BW * 4 * UPITCH; e += blockDim.x) dst[e] = 0.f;
+  __syncthreads();
+  for (int e = threadIdx.x; e < BW * BW; e += blockDim.x) {
+    const int c = e / BW, j = e % BW;
+    if (c < ncols && j < ncols) {
+      const float v = U[(kB + c) * in + kB + j];
+      dst[(j * 4 + (c & 3)) * UPITCH + (c >> 2)] = v;
+      if (c == j) dst[BW * 4 * UPITCH + j] = 1.f / v;
+    }
+  }
+  if (threadIdx.x >= ncols && threadIdx.x < BW) dst[BW * 4 * UPITCH + threadIdx.x] = 0.f;
 }
 
 // Wp[r][p] = W[r][perm[p]] (0 for dead channels and the padding).
@@ -340,7 +364,7 @@ cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st) {
     configured = true;
   }
   const unsigned grid = (unsigned)((sp.out + ROWS - 1) / ROWS);
-  sweep_kernel<GSB><<<grid, 128, smem, st>>>(sp);
+  sweep_kernel<GSB><<<grid, NT, smem, st>>>(sp);
   note_launch();
   return cudaGetLastError();
 }
@@ -364,6 +388,7 @@ size_t quantize_ws_bytes(int64_t out, int64_t in, const gptq_config_t* cfg) {
   b += 2 * round_up(4 * np_ * np_, 256);   // Uh, Ul
   b += 2 * round_up(4 * out * bo, 256);    // Eh, El
   b += round_up(out * np_, 256);           // codes_p
+  b += round_up(4 * (int64_t)kDiagBlockFloats * (np_ / BW), 256);  // interleaved diagonal blocks
   b += round_up(4 * in, 256);              // inverse permutation
   return b;
 }
@@ -390,6 +415,8 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
   p += round_up(4 * out * bo, 256);
   uint8_t* codes_p = p;
   p += round_up(out * np_, 256);
+  float* Ud = (float*)p;
+  p += round_up(4 * (int64_t)kDiagBlockFloats * (np_ / BW), 256);
   int32_t* inv = (int32_t*)p;
   const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
 
@@ -417,6 +444,9 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
   {
     dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 32), (unsigned)np_);
     split_u_kernel<<<grid, 256, 0, st>>>(U, in, np_, Uh, Ul);
+    note_launch();
+    CUDA_TRY(cudaGetLastError());
+    pack_diag_kernel<<<(unsigned)(np_ / BW), 256, 0, st>>>(U, in, Ud);
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
@@ -456,6 +486,8 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
       sp.lde = bo;
       sp.e_col0 = k - o0;
       sp.loss = loss;
+      sp.Ud = Ud + (k / BW) * (int64_t)kDiagBlockFloats;
+      sp.status = &hdr->status;
       cudaError_t e;
       switch (gsb) {
         case 8:

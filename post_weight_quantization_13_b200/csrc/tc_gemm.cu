@@ -224,9 +224,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
+      // Parameters the loops use live in registers: the inline asm below
+      // clobbers memory, which would otherwise force reloads of the
+      // parameter block on every iteration.
+      const int rounds = kp.rounds, kbc = kp.kbc, stages = kp.stages, stage_bytes = kp.stage_bytes;
+      const int slot_bytes = kp.slot_bytes;
+      const int q_k0 = kp.q_k0, q_row0 = kp.q_row0, p_k0 = kp.p_k0, p_row0 = kp.p_row0;
+      const int64_t bs_q_k = kp.bs_q_k, bs_q_row = kp.bs_q_row, bs_p_k = kp.bs_p_k, bs_p_row = kp.bs_p_row;
       int stage = 0;
       uint32_t phase = 0;
-      for (int round = 0; round < kp.rounds && !*abort_flag; ++round) {
+      for (int round = 0; round < rounds && !*abort_flag; ++round) {
         Piece pl[kMaxPieces];
         const int npc = round_pieces(kp, blockIdx.x, round, pl);
         if (npc <= 0) break;
@@ -237,13 +244,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           pc[i] = pl[i];
           if (i < npc) bytes += (uint32_t)(pc[i].nh * kQTileBytes + pc[i].np * kRowBytes) * SPLIT;
         }
-        for (int kb = 0; kb < kp.kbc; ++kb) {
+        for (int kb = 0; kb < kbc; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) {
             abort_cta(kp, abort_flag);
             break;
           }
           if (*abort_flag) break;
-          uint8_t* sb = smem + (size_t)stage * kp.stage_bytes;
+          uint8_t* sb = smem + (size_t)stage * stage_bytes;
           uint64_t* bar = &full[stage];
           mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
@@ -251,16 +258,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i >= npc) break;
             const Piece& p = pc[i];
             const int bq = p.batch;
-            const int xq = (int)(kp.q_k0 + bq * kp.bs_q_k) + kb * BK;
-            const int yq = (int)(kp.q_row0 + bq * kp.bs_q_row) + p.q0;
-            uint8_t* dq = sb + p.qslot * kp.slot_bytes;
+            const int xq = (int)(q_k0 + bq * bs_q_k) + kb * BK;
+            const int yq = (int)(q_row0 + bq * bs_q_row) + p.q0;
+            uint8_t* dq = sb + p.qslot * slot_bytes;
             for (int h = 0; h < p.nh; ++h) {
               uint8_t* d = dq + h * kQTileBytes * SPLIT;
               tma_load_2d(d, &maps.q, bar, xq, yq + 128 * h);
               if (SPLIT == 2) tma_load_2d(d + kQTileBytes, &maps.qlo, bar, xq, yq + 128 * h);
             }
-            const int xp = (int)(kp.p_k0 + bq * kp.bs_p_k) + kb * BK;
-            const int yp = (int)(kp.p_row0 + bq * kp.bs_p_row) + p.p0;
+            const int xp = (int)(p_k0 + bq * bs_p_k) + kb * BK;
+            const int yp = (int)(p_row0 + bq * bs_p_row) + p.p0;
             int off = 0;
 #pragma unroll
             for (int b = 0; b < kNumBoxes; ++b) {
@@ -273,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
           }
-          if (++stage == kp.stages) {
+          if (++stage == stages) {
             stage = 0;
             phase ^= 1;
           }
@@ -283,11 +290,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
+      const int rounds = kp.rounds, nchunks = kp.nchunks, kchunk = kp.kchunk, kbc = kp.kbc;
+      const int stages = kp.stages, stage_bytes = kp.stage_bytes, slot_bytes = kp.slot_bytes;
       int stage = 0;
       uint32_t phase = 0;
       int step = 0;  // (round, chunk) counter: selects the accumulator buffer
       bool ok = true;
-      for (int round = 0; round < kp.rounds && ok && !*abort_flag; ++round) {
+      for (int round = 0; round < rounds && ok && !*abort_flag; ++round) {
         Piece pl[kMaxPieces];
         const int npc = round_pieces(kp, blockIdx.x, round, pl);
         if (npc <= 0) break;
@@ -298,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pc[i] = pl[i];
           idesc[i] = make_idesc(OpTraits<OP>::kFmt, 128, (uint32_t)pc[i].np);
         }
-        for (int ch = 0; ch < kp.nchunks && ok; ++ch, ++step) {
+        for (int ch = 0; ch < nchunks && ok; ++ch, ++step) {
           const int buf = step % nbuf;
           const int use = step / nbuf;
           if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) {
@@ -308,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t tacc = tbase + buf * buf_cols;
-          const int kb0 = ch * kp.kchunk;
-          const int kb1 = min(kp.kbc, kb0 + kp.kchunk);
+          const int kb0 = ch * kchunk;
+          const int kb1 = min(kbc, kb0 + kchunk);
           for (int kb = kb0; kb < kb1; ++kb) {
             if (!mbar_wait(&full[stage], phase)) {
               abort_cta(kp, abort_flag);
@@ -317,14 +326,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc_fence_after();
-            const uint32_t sb = smem_u32(smem + (size_t)stage * kp.stage_bytes);
+            const uint32_t sb = smem_u32(smem + (size_t)stage * stage_bytes);
 #pragma unroll
             for (int i = 0; i < kMaxPieces; ++i) {
               if (i >= npc) break;
               const Piece& p = pc[i];
               const uint32_t pb = sb + q_region + (uint32_t)p.prow * kRowBytes;
               for (int h = 0; h < p.nh; ++h) {
-                const uint32_t qa = sb + p.qslot * kp.slot_bytes + h * kQTileBytes * SPLIT;
+                const uint32_t qa = sb + p.qslot * slot_bytes + h * kQTileBytes * SPLIT;
                 const uint32_t d = tacc + (uint32_t)(p.tcol + h * p.np);
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
@@ -344,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
             }
             umma_commit(&empty[stage]);
-            if (++stage == kp.stages) {
+            if (++stage == stages) {
               stage = 0;
               phase ^= 1;
             }
@@ -357,13 +366,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------ epilogue (warps 2-5)
     const int quarter = warp & 3;  // tensor-memory lanes 32*quarter .. +31
+    const int rounds = kp.rounds, nchunks = kp.nchunks;
+    const int R = kp.R, Cn = kp.Cn, mask = kp.mask, transpose = kp.transpose;
+    const int64_t mask_off = kp.mask_off, ldc = kp.ldc, c_row0 = kp.c_row0, c_col0 = kp.c_col0;
+    const int64_t bs_c_row = kp.bs_c_row, bs_c_col = kp.bs_c_col;
+    const float alpha = kp.alpha, beta0 = kp.beta;
+    float* const Cbase = kp.C;
+    float* const Clbase = kp.C_lo;
     int step = 0;
     bool ok = true;
-    for (int round = 0; round < kp.rounds && ok; ++round) {
+    for (int round = 0; round < rounds && ok; ++round) {
       Piece pc[kMaxPieces];
       const int npc = round_pieces(kp, blockIdx.x, round, pc);
       if (npc <= 0) break;
-      for (int ch = 0; ch < kp.nchunks; ++ch, ++step) {
+      for (int ch = 0; ch < nchunks; ++ch, ++step) {
         const int buf = step % nbuf;
         const int use = step / nbuf;
         if (!mbar_wait_sleep(&acc_full[buf], use & 1)) {
@@ -377,11 +393,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         // the first chunk applies beta, later chunks accumulate onto C
-        const float beta = ch == 0 ? kp.beta : 1.f;
+        const float beta = ch == 0 ? beta0 : 1.f;
         for (int i = 0; i < npc; ++i) {
           const Piece& p = pc[i];
-          const int64_t cr = kp.c_row0 + (int64_t)p.batch * kp.bs_c_row;
-          const int64_t cc = kp.c_col0 + (int64_t)p.batch * kp.bs_c_col;
+          const int64_t cr = c_row0 + (int64_t)p.batch * bs_c_row;
+          const int64_t cc = c_col0 + (int64_t)p.batch * bs_c_col;
           for (int h = 0; h < p.nh; ++h) {
             const int c = p.q0 + 128 * h + quarter * 32 + lane;
             const uint32_t taddr = tbase + buf * buf_cols + (uint32_t)(p.tcol + h * p.np) +
@@ -400,23 +416,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 16; j < 32; ++j) v[j] = 0.f;
               }
-              if (c >= kp.Cn) continue;
+              if (c >= Cn) continue;
               const int nn = min(32, p.np - n0);
               const int r0 = p.p0 + n0;
               const int64_t base =
-                  kp.transpose ? (cr + c) * kp.ldc + (cc + r0) : (cr + r0) * kp.ldc + (cc + c);
-              const int64_t stp = kp.transpose ? 1 : kp.ldc;
+                  transpose ? (cr + c) * ldc + (cc + r0) : (cr + r0) * ldc + (cc + c);
+              const int64_t stp = transpose ? 1 : ldc;
               uint32_t keep = 0;
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
                 const int r = r0 + j;
-                bool k = j < nn && r < kp.R;
-                if (kp.mask == 1) k = k && ((int64_t)c - r >= kp.mask_off);
-                if (kp.mask == 2) k = k && ((int64_t)c - r <= kp.mask_off);
+                bool k = j < nn && r < R;
+                if (mask == 1) k = k && ((int64_t)c - r >= mask_off);
+                if (mask == 2) k = k && ((int64_t)c - r <= mask_off);
                 keep |= (uint32_t)k << j;
               }
-              float* __restrict__ Cp = kp.C + base;
-              float* __restrict__ Cl = kp.C_lo ? kp.C_lo + base : nullptr;
+              float* __restrict__ Cp = Cbase + base;
+              float* __restrict__ Cl = Clbase ? Clbase + base : nullptr;
               if (beta != 0.f) {
                 float old[32];
 #pragma unroll
@@ -427,10 +443,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if ((keep >> j) & 1u) old[j] += Cl[j * stp];
                 }
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = fmaf(beta, old[j], kp.alpha * v[j]);
+                for (int j = 0; j < 32; ++j) v[j] = fmaf(beta, old[j], alpha * v[j]);
               } else {
 #pragma unroll
-                for (int j = 0; j < 32; ++j) v[j] = kp.alpha * v[j];
+                for (int j = 0; j < 32; ++j) v[j] = alpha * v[j];
               }
               if (Cl) {
 #pragma unroll
