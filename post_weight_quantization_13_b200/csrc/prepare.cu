@@ -174,7 +174,8 @@ __global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* 
         }
       }
       __syncthreads();
-      if (r0 + 7 > j && c0 + 3 > j) {
+      // this block has elements with j < c <= r
+      if (r0 + 7 > j && c0 + 3 > j && c0 <= r0 + 7) {
         const float dinv = pinv[j];
         float cr[8], cc[4];
 #pragma unroll
@@ -184,13 +185,20 @@ __global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* 
         cc[1] = c4.y;
         cc[2] = c4.z;
         cc[3] = c4.w;
+        if (c0 > j && c0 + 3 <= r0) {  // whole block strictly inside the update
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+          for (int i = 0; i < 8; ++i)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int r = r0 + i, c = c0 + q;
-            if (r > j && c > j && c <= r) a[i][q] = fmaf(-cr[i], cc[q], a[i][q]);
-          }
+            for (int q = 0; q < 4; ++q) a[i][q] = fmaf(-cr[i], cc[q], a[i][q]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int r = r0 + i, c = c0 + q;
+              if (r > j && c > j && c <= r) a[i][q] = fmaf(-cr[i], cc[q], a[i][q]);
+            }
+        }
       }
     }
   }
@@ -236,7 +244,8 @@ __global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* 
         }
       }
       __syncthreads();
-      if (r0 + 7 > j) {
+      // rows r > j take row j of M, which is zero past column j
+      if (r0 + 7 > j && c0 <= j) {
         float lr[8], mr[4];
 #pragma unroll
         for (int i = 0; i < 8; ++i) lr[i] = Ls[(r0 + i) * LD + j];
@@ -245,11 +254,18 @@ __global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* 
         mr[1] = m4.y;
         mr[2] = m4.z;
         mr[3] = m4.w;
+        if (r0 > j) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (r0 + i > j)
+          for (int i = 0; i < 8; ++i)
 #pragma unroll
             for (int q = 0; q < 4; ++q) b[i][q] = fmaf(-lr[i], mr[q], b[i][q]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            if (r0 + i > j)
+#pragma unroll
+              for (int q = 0; q < 4; ++q) b[i][q] = fmaf(-lr[i], mr[q], b[i][q]);
+        }
       }
     }
   }

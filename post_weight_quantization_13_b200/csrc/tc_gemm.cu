@@ -19,11 +19,11 @@
 // against one or two 128-column Q tiles (two accumulators that share the P
 // tile: a 256 x N output from 256 + N operand rows per k).  Schedules:
 //   tri   the upper triangle of a symmetric S = X X^T, in 256-column
-//         super-strips; super-strip s needs rows [0, 256(s+1)).  All
-//         super-strips' rows, in 16-row units, are laid end to end and cut
-//         into equal segments, one per CTA and round: every CTA gets the
-//         same work (+-16 rows) and all CTAs stream the same k-window of X
-//         together, which keeps X L2-resident.
+//         super-strips; super-strip s needs rows [0, 256(s+1)), i.e. s + 1
+//         pieces of 256 rows.  One piece per CTA and round; all CTAs stream
+//         the same k-window of X together, which keeps X L2-resident.  With
+//         one 256 x 256 piece per round a stage is 32 KB, so seven stages
+//         fit in shared memory.
 //   grid  regular 128 x 256 tiles (optionally batched), one per round, with
 //         two tensor-memory buffers so a tile's epilogue overlaps the next
 //         tile's main loop.
@@ -47,7 +47,6 @@ constexpr int kThreads = 192;
 constexpr int kMaxPieces = 2;
 constexpr uint32_t kRowBytes = 64;                 // one K-major row per stage
 constexpr uint32_t kQTileBytes = 128 * kRowBytes;  // 8 KB per component
-constexpr int kTriMaxUnits = 15;                   // 240 rows x 256 columns per CTA round
 constexpr int kNumBoxes = 5;                       // P boxes of 256, 128, 64, 32, 16 rows
 
 struct Piece {
@@ -71,7 +70,7 @@ struct KParams {
   int nq, npt, ntiles;
   int64_t bs_p_row, bs_p_k, bs_q_row, bs_q_k, bs_c_row, bs_c_col;
   // tri schedule
-  int n_in, nss, utot, T;
+  int n_in, nss;
   int grid, rounds;
   // epilogue
   float* C;
@@ -93,40 +92,28 @@ struct TmaMaps {
   CUtensorMap qlo;
 };
 
-// 16-row units before super-strip s (every super-strip before the last is full).
-__host__ __device__ __forceinline__ int tri_prefix(int s) { return 8 * s * (s + 1); }
-
 __host__ __device__ int round_pieces(const KParams& kp, int cta, int round, Piece* pc) {
   if (kp.tri) {
-    const int seg = round * kp.grid + cta;
-    int x = seg * kp.T;
-    const int x1 = min(x + kp.T, kp.utot);
-    if (x >= x1) return 0;
-    int n = 0, prow = 0, tcol = 0;
-    while (x < x1) {
-      if (n == kMaxPieces) return -1;
-      int s = (int)((sqrtf(1.0f + 0.5f * (float)x) - 1.0f) * 0.5f);
-      if (s < 0) s = 0;
-      while (s + 1 < kp.nss && tri_prefix(s + 1) <= x) ++s;
-      while (s > 0 && tri_prefix(s) > x) --s;
-      const int send = (s == kp.nss - 1) ? kp.utot : tri_prefix(s + 1);
-      const int u = min(x1, send) - x;
-      if (u > 16) return -1;
-      Piece& p = pc[n];
-      p.q0 = 256 * s;
-      p.nh = (256 * s + 128 < kp.n_in) ? 2 : 1;
-      p.p0 = (x - tri_prefix(s)) * 16;
-      p.np = u * 16;
-      p.qslot = n;
-      p.prow = prow;
-      p.tcol = tcol;
-      p.batch = 0;
-      prow += p.np;
-      tcol += p.nh * p.np;
-      x += u;
-      ++n;
-    }
-    return n;
+    // piece index t -> (super-strip s, 256-row piece within it); super-strip
+    // s has s + 1 pieces (the last super-strip may have fewer rows)
+    const int t = round * kp.grid + cta;
+    if (t >= kp.ntiles) return 0;
+    int s = (int)((sqrtf(1.0f + 8.0f * (float)t) - 1.0f) * 0.5f);
+    if (s < 0) s = 0;
+    while (s + 1 < kp.nss && (s + 1) * (s + 2) / 2 <= t) ++s;
+    while (s > 0 && s * (s + 1) / 2 > t) --s;
+    const int piece = t - s * (s + 1) / 2;
+    Piece& p = pc[0];
+    p.q0 = 256 * s;
+    p.nh = (256 * s + 128 < kp.n_in) ? 2 : 1;
+    p.p0 = 256 * piece;
+    const int rows = min(256, kp.n_in - p.p0);
+    p.np = (rows + 15) & ~15;
+    p.qslot = 0;
+    p.prow = 0;
+    p.tcol = 0;
+    p.batch = 0;
+    return 1;
   }
   const int t = round * kp.grid + cta;
   if (t >= kp.ntiles) return 0;
@@ -611,28 +598,19 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
   kp.status = a.status;
   int grid;
   if (a.tri) {
+    // one CTA round = one 256-column super-strip x up to 256 rows; the
+    // upper triangle needs pieces 0..s of super-strip s
     const int n = (int)a.R;
     kp.n_in = n;
     kp.nss = (n + 255) / 256;
-    kp.utot = tri_prefix(kp.nss - 1) + (n + 15) / 16;
-    grid = num_sms;
-    const int rounds = (kp.utot + grid * kTriMaxUnits - 1) / (grid * kTriMaxUnits);
-    int T = (kp.utot + grid * rounds - 1) / (grid * rounds);
-    // check the packing on the host with the same function the kernel uses
-    while (true) {
-      kp.grid = grid;
-      kp.T = T;
-      kp.rounds = (kp.utot + grid * T - 1) / (grid * T);
-      bool ok = true;
-      Piece pc[kMaxPieces];
-      for (int s = 0; s < grid * kp.rounds && ok; ++s)
-        if (round_pieces(kp, s % grid, s / grid, pc) < 0) ok = false;
-      if (ok) break;
-      if (--T < 1) return cudaErrorInvalidValue;
-    }
-    kp.qslots = kMaxPieces;
+    kp.ntiles = 0;
+    for (int s = 0; s < kp.nss; ++s) kp.ntiles += (std::min(256 * (s + 1), n) + 255) / 256;
+    grid = std::min(num_sms, kp.ntiles);
+    kp.grid = grid;
+    kp.rounds = (kp.ntiles + grid - 1) / grid;
+    kp.qslots = 1;
     kp.slot_bytes = 2 * kQTileBytes * split;
-    kp.p_rows_max = kp.T * 16;
+    kp.p_rows_max = 256;
   } else {
     kp.nq = (int)((a.Cn + 127) / 128);
     kp.npt = (int)((a.R + 255) / 256);
