@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(256) rank_kernel(const float* __restrict__ hd,
 __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S, int64_t in, int64_t np_,
                                                      float scale, const int32_t* __restrict__ perm,
                                                      const uint8_t* __restrict__ dead, PrepHeader* hdr,
-                                                     float* __restrict__ Rh, float* __restrict__ Rl) {
+                                                     float* __restrict__ R) {
   const int64_t a = blockIdx.y;
   const float lam = hdr->lambda;
   for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < np_; b += (int64_t)gridDim.x * blockDim.x) {
@@ -109,10 +109,26 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
     } else {
       v = (a == b) ? 1.f : 0.f;
     }
-    float h, l;
-    split_tf32(v, h, l);
-    Rh[a * np_ + b] = h;
-    Rl[a * np_ + b] = l;
+    R[a * np_ + b] = v;
+  }
+}
+
+// Pk[r][c] = split(R[r0 + r][kB + c]): the panel below diagonal block k as a
+// 3xTF32 operand (rows x 128, row stride 128).
+__global__ void __launch_bounds__(256) split_panel_kernel(const float* __restrict__ R, int64_t np_, int64_t r0,
+                                                          int64_t kB, int64_t rows, float* __restrict__ Ph,
+                                                          float* __restrict__ Pl) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * 32;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e >> 5, c4 = (e & 31) << 2;
+    const float4 v = *reinterpret_cast<const float4*>(R + (r0 + r) * np_ + kB + c4);
+    float4 h, l;
+    split_tf32(v.x, h.x, l.x);
+    split_tf32(v.y, h.y, l.y);
+    split_tf32(v.z, h.z, l.z);
+    split_tf32(v.w, h.w, l.w);
+    *reinterpret_cast<float4*>(Ph + r * 128 + c4) = h;
+    *reinterpret_cast<float4*>(Pl + r * 128 + c4) = l;
   }
 }
 
@@ -132,8 +148,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
 // block stays finite.
 constexpr int LD = NB + 1;
 
-__global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* Mh, float* Ml, float* Mth,
-                                                   float* Mtl, int64_t np_, int k, PrepHeader* hdr) {
+__global__ void __launch_bounds__(512) leaf_kernel(const float* R, float* Mh, float* Ml, float* Mth, float* Mtl,
+                                                   int64_t np_, int k, PrepHeader* hdr) {
   extern __shared__ float Ls[];            // [NB][LD]: L, then staging for M^T
   __shared__ __align__(16) float colb[2][NB];  // published column (Cholesky) / row (inverse)
   __shared__ float pinv[NB];               // 1 / d_j
@@ -146,12 +162,11 @@ __global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* 
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int64_t g = (o + r0 + i) * np_ + o + c0;
-    const float4 h = *reinterpret_cast<const float4*>(Rh + g);
-    const float4 l = *reinterpret_cast<const float4*>(Rl + g);
-    a[i][0] = h.x + l.x;
-    a[i][1] = h.y + l.y;
-    a[i][2] = h.z + l.z;
-    a[i][3] = h.w + l.w;
+    const float4 h = *reinterpret_cast<const float4*>(R + g);
+    a[i][0] = h.x;
+    a[i][1] = h.y;
+    a[i][2] = h.z;
+    a[i][3] = h.w;
   }
   // ---------------------------------------------------------- Cholesky
   for (int jj = 0; jj < NB / 4; ++jj) {
@@ -274,12 +289,6 @@ __global__ void __launch_bounds__(512) leaf_kernel(float* Rh, float* Rl, float* 
   for (int i = 0; i < 8; ++i) {
     const int64_t g = (o + r0 + i) * np_ + o + c0;
     float4 h, l;
-    split_tf32(a[i][0], h.x, l.x);
-    split_tf32(a[i][1], h.y, l.y);
-    split_tf32(a[i][2], h.z, l.z);
-    split_tf32(a[i][3], h.w, l.w);
-    *reinterpret_cast<float4*>(Rh + g) = h;
-    *reinterpret_cast<float4*>(Rl + g) = l;
     split_tf32(b[i][0], h.x, l.x);
     split_tf32(b[i][1], h.y, l.y);
     split_tf32(b[i][2], h.z, l.z);
@@ -360,8 +369,9 @@ cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
 size_t prepare_ws_bytes(int64_t in) {
   const int64_t np_ = round_up(in, NB);
   size_t b = kHeaderBytes;
-  b += round_up((int64_t)sizeof(float) * in, 256);      // hd
-  b += 8 * round_up((int64_t)sizeof(float) * np_ * np_, 256);  // R, M, Mt, XT (hi, lo)
+  b += round_up((int64_t)sizeof(float) * in, 256);               // hd
+  b += 9 * round_up((int64_t)sizeof(float) * np_ * np_, 256);    // R; L, M, Mt, X^T (hi, lo)
+  b += 2 * round_up((int64_t)sizeof(float) * np_ * NB, 256);     // split panel
   return b;
 }
 
@@ -375,14 +385,17 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   float* hd = (float*)p;
   p += round_up((int64_t)sizeof(float) * in, 256);
   const size_t mat = round_up((int64_t)sizeof(float) * np_ * np_, 256);
-  float* Rh = (float*)p; p += mat;
-  float* Rl = (float*)p; p += mat;
+  float* R = (float*)p; p += mat;      // reversed, damped Hessian; Schur complements in place
+  float* Lh = (float*)p; p += mat;     // L's panels (split), for the inverse
+  float* Ll = (float*)p; p += mat;
   float* Mh = (float*)p; p += mat;
   float* Ml = (float*)p; p += mat;
   float* Mth = (float*)p; p += mat;
   float* Mtl = (float*)p; p += mat;
   float* Xh = (float*)p; p += mat;
   float* Xl = (float*)p; p += mat;
+  float* Pkh = (float*)p; p += round_up((int64_t)sizeof(float) * np_ * NB, 256);
+  float* Pkl = (float*)p;
   const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
 
   CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
@@ -396,7 +409,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   CUDA_TRY(cudaGetLastError());
   {
     dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 16), (unsigned)np_);
-    gather_kernel<<<grid, 256, 0, st>>>(S, in, np_, scale, perm, dead, hdr, Rh, Rl);
+    gather_kernel<<<grid, 256, 0, st>>>(S, in, np_, scale, perm, dead, hdr, R);
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
@@ -408,45 +421,58 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   }
   const int KB = (int)(np_ / NB);
   for (int k = 0; k < KB; ++k) {
-    leaf_kernel<<<1, 512, leaf_smem, st>>>(Rh, Rl, Mh, Ml, Mth, Mtl, np_, k, hdr);
+    leaf_kernel<<<1, 512, leaf_smem, st>>>(R, Mh, Ml, Mth, Mtl, np_, k, hdr);
     note_launch();
     CUDA_TRY(cudaGetLastError());
-    const int64_t r0 = (int64_t)(k + 1) * NB;
+    const int64_t kB = (int64_t)k * NB;
+    const int64_t r0 = kB + NB;
     const int64_t m = np_ - r0;
     if (m <= 0) break;
-    // panel: L[r0:, k] = R[r0:, k] M_kk^T   (in place, split)
+    split_panel_kernel<<<(unsigned)std::min<int64_t>((m * 32 + 255) / 256, 1024), 256, 0, st>>>(R, np_, r0, kB, m,
+                                                                                                 Pkh, Pkl);
+    note_launch();
+    CUDA_TRY(cudaGetLastError());
+    // panel: L[r0:, k] = R[r0:, k] M_kk^T   -> L's panel (split)
     GemmArgs pg;
     pg.op = OP_TF32X3;
-    pg.P = {Rh, Rl, np_, np_, np_};
+    pg.P = {Pkh, Pkl, m, NB, NB};
     pg.Q = {Mh, Ml, np_, np_, np_};
     pg.R = m;
     pg.Cn = NB;
     pg.K = NB;
-    pg.p_row0 = r0;
-    pg.p_k0 = (int64_t)k * NB;
-    pg.q_row0 = (int64_t)k * NB;
-    pg.q_k0 = (int64_t)k * NB;
-    pg.C = Rh;
-    pg.C_lo = Rl;
+    pg.p_row0 = 0;
+    pg.p_k0 = 0;
+    pg.q_row0 = kB;
+    pg.q_k0 = kB;
+    pg.C = Lh;
+    pg.C_lo = Ll;
     pg.ldc = np_;
     pg.c_row0 = r0;
-    pg.c_col0 = (int64_t)k * NB;
+    pg.c_col0 = kB;
     pg.alpha = 1.f;
     pg.beta = 0.f;
     pg.status = &hdr->status;
     CUDA_TRY(run_gemm(pg, st, dev.sms, force_simt));
     // trailing: R[r0:, r0:] -= L[r0:, k] L[r0:, k]^T   (lower triangle)
-    GemmArgs tg = pg;
-    tg.Q = pg.P;
+    GemmArgs tg;
+    tg.op = OP_TF32X3;
+    tg.P = {Lh, Ll, np_, np_, np_};
+    tg.Q = tg.P;
     tg.R = m;
     tg.Cn = m;
+    tg.K = NB;
+    tg.p_row0 = r0;
+    tg.p_k0 = kB;
     tg.q_row0 = r0;
-    tg.q_k0 = (int64_t)k * NB;
+    tg.q_k0 = kB;
+    tg.C = R;
+    tg.ldc = np_;
     tg.c_row0 = r0;
     tg.c_col0 = r0;
     tg.alpha = -1.f;
     tg.beta = 1.f;
     tg.mask = 2;
+    tg.status = &hdr->status;
     CUDA_TRY(run_gemm(tg, st, dev.sms, force_simt));
   }
   // triangular inverse: merge groups pairwise, M21 = -M22 (L21 M11)
@@ -470,7 +496,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
       // X^T[o1+c][o2+r] = (L21 M11)[r][c] = sum_t L[o2+r][o1+t] Mt[o1+c][o1+t]
       GemmArgs a;
       a.op = OP_TF32X3;
-      a.P = {Rh, Rl, np_, np_, np_};
+      a.P = {Lh, Ll, np_, np_, np_};
       a.Q = {Mth, Mtl, np_, np_, np_};
       a.R = s2;
       a.Cn = s1;

@@ -81,6 +81,11 @@ struct KParams {
   int64_t mask_off;
   int transpose;
   uint32_t* status;
+  // TMA epilogue: accumulators staged in shared memory, written by a bulk
+  // tensor store (beta == 0) or reduce-add (beta == 1)
+  int epi_tma;
+  int epi_split;  // also store the tf32 remainder (through map clo)
+  int lower;      // grid schedule over tiles that hold elements with c - r <= mask_off only
   // shared-memory plan
   int stages, stage_bytes, qslots, slot_bytes, p_rows_max;
 };
@@ -90,7 +95,16 @@ struct TmaMaps {
   CUtensorMap plo[kNumBoxes];  // P remainder (3xTF32 only)
   CUtensorMap q;               // Q (hi), 128-row boxes
   CUtensorMap qlo;
+  CUtensorMap c;               // output (TMA epilogue): 32 x 128 tiles, 3-D (batch)
+  CUtensorMap clo;             // output remainder (split outputs)
 };
+constexpr uint32_t kStageTileBytes = 32 * 128 * 4;  // one epilogue pass: 32 rows x 128 columns fp32
+
+// Column tiles of row tile pt that hold an element with c - r <= mask_off.
+__host__ __device__ __forceinline__ int lower_tiles(const KParams& kp, int pt) {
+  const int64_t last = ((int64_t)pt * 256 + 255 + kp.mask_off) / 128 + 1;
+  return (int)(last < 0 ? 0 : (last > kp.nq ? kp.nq : last));
+}
 
 __host__ __device__ int round_pieces(const KParams& kp, int cta, int round, Piece* pc) {
   if (kp.tri) {
@@ -114,6 +128,28 @@ __host__ __device__ int round_pieces(const KParams& kp, int cta, int round, Piec
     p.tcol = 0;
     p.batch = 0;
     return 1;
+  }
+  if (kp.lower) {
+    int t = round * kp.grid + cta;
+    if (t >= kp.ntiles) return 0;
+    for (int pt = 0; pt < kp.npt; ++pt) {
+      const int cnt = lower_tiles(kp, pt);
+      if (t < cnt) {
+        Piece& p = pc[0];
+        p.q0 = t * 128;
+        p.nh = 1;
+        p.p0 = pt * 256;
+        const int rows = min(256, kp.R - p.p0);
+        p.np = (rows + 15) & ~15;
+        p.qslot = 0;
+        p.prow = 0;
+        p.tcol = 0;
+        p.batch = 0;
+        return 1;
+      }
+      t -= cnt;
+    }
+    return 0;
   }
   const int t = round * kp.grid + cta;
   if (t >= kp.ntiles) return 0;
@@ -162,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int BK = OpTraits<OP>::kBK;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint64_t* full = (uint64_t*)(smem + (size_t)kp.stages * kp.stage_bytes);
+  uint64_t* full = (uint64_t*)(smem + (size_t)kp.stages * kp.stage_bytes + (kp.epi_tma ? 2 * kStageTileBytes : 0));
   uint64_t* empty = full + kp.stages;
   uint64_t* acc_full = empty + kp.stages;  // [2]
   uint64_t* acc_empty = acc_full + 2;      // [2]
@@ -360,6 +396,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float alpha = kp.alpha, beta0 = kp.beta;
     float* const Cbase = kp.C;
     float* const Clbase = kp.C_lo;
+    const int epi_tma = kp.epi_tma, epi_split = kp.epi_split;
+    uint8_t* const stage_out = smem + (size_t)kp.stages * kp.stage_bytes;  // 2 x 16 KB
+    int epi_pass = 0;
     int step = 0;
     bool ok = true;
     for (int round = 0; round < rounds && ok; ++round) {
@@ -389,6 +428,88 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = p.q0 + 128 * h + quarter * 32 + lane;
             const uint32_t taddr = tbase + buf * buf_cols + (uint32_t)(p.tcol + h * p.np) +
                                    ((uint32_t)(quarter * 32) << 16);
+            if (epi_tma) {
+              const int cl = quarter * 32 + lane;  // column inside the 128-column tile
+              const bool reduce = beta != 0.f;     // beta is 0 (store) or 1 (reduce-add)
+              for (int n0 = 0; n0 < p.np; n0 += 32) {
+                float v[32];
+                if (p.np - n0 >= 32) {
+                  tmem_ld32(taddr + (uint32_t)n0, v);
+                } else {
+                  float t16[16];
+                  tmem_ld16(taddr + (uint32_t)n0, t16);
+#pragma unroll
+                  for (int j = 0; j < 16; ++j) v[j] = t16[j];
+#pragma unroll
+                  for (int j = 16; j < 32; ++j) v[j] = 0.f;
+                }
+                const int r0 = p.p0 + n0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                  float x = alpha * v[j];
+                  if (mask == 1 && (int64_t)c - (r0 + j) < mask_off) x = 0.f;
+                  if (mask == 2 && (int64_t)c - (r0 + j) > mask_off) x = 0.f;
+                  v[j] = x;
+                }
+                // the staging buffer is free once the bulk copy that last read it is done
+                uint8_t* sb0 = stage_out + (epi_split ? 0 : (epi_pass & 1) * kStageTileBytes);
+                if (threadIdx.x == 64) {
+                  if (epi_split)
+                    bulk_wait_read<0>();
+                  else
+                    bulk_wait_read<1>();
+                }
+                named_bar_sync(1, 128);
+                float* sh = reinterpret_cast<float*>(sb0);
+                float* sl = reinterpret_cast<float*>(sb0 + kStageTileBytes);
+                if (!transpose) {
+                  // tile [32 rows][128 columns]
+#pragma unroll
+                  for (int j = 0; j < 32; ++j) {
+                    if (epi_split) {
+                      float hi, lo;
+                      split_tf32(v[j], hi, lo);
+                      sh[j * 128 + cl] = hi;
+                      sl[j * 128 + cl] = lo;
+                    } else {
+                      sh[j * 128 + cl] = v[j];
+                    }
+                  }
+                } else {
+                  // tile [128 columns of C = rows of the output][32], 128-byte swizzle
+#pragma unroll
+                  for (int m = 0; m < 8; ++m) {
+                    const int off = cl * 32 + ((m ^ (cl & 7)) * 4);
+                    if (epi_split) {
+                      float4 h4, l4;
+                      split_tf32(v[4 * m + 0], h4.x, l4.x);
+                      split_tf32(v[4 * m + 1], h4.y, l4.y);
+                      split_tf32(v[4 * m + 2], h4.z, l4.z);
+                      split_tf32(v[4 * m + 3], h4.w, l4.w);
+                      *reinterpret_cast<float4*>(sh + off) = h4;
+                      *reinterpret_cast<float4*>(sl + off) = l4;
+                    } else {
+                      *reinterpret_cast<float4*>(sh + off) =
+                          make_float4(v[4 * m + 0], v[4 * m + 1], v[4 * m + 2], v[4 * m + 3]);
+                    }
+                  }
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (threadIdx.x == 64) {
+                  const int tc = p.q0 + 128 * h, tr = r0;
+                  const int x = transpose ? tr : tc, y = transpose ? tc : tr;
+                  if (reduce)
+                    tma_reduce_add_3d(&maps.c, sh, x, y, p.batch);
+                  else
+                    tma_store_3d(&maps.c, sh, x, y, p.batch);
+                  if (epi_split) tma_store_3d(&maps.clo, sl, x, y, p.batch);
+                  bulk_commit();
+                }
+                ++epi_pass;
+              }
+              continue;
+            }
             for (int n0 = 0; n0 < p.np; n0 += 32) {
               // 32 accumulator columns (C rows) per pass: every load of C is
               // issued before any store so they overlap in flight.
@@ -456,6 +577,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&acc_empty[buf]);
       }
     }
+    if (epi_tma && threadIdx.x == 64) bulk_wait_all();
   }
 
   __syncthreads();
@@ -511,6 +633,23 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int6
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D output map (columns, rows, batch) for the TMA epilogue.  box_x x box_y
+// fp32 tiles, no swizzle (box_x = 128) or 128-byte swizzle (box_x = 32).
+bool make_out_map(CUtensorMap* m, const float* base, int64_t xdim, int64_t ydim, int64_t ld, int64_t batch,
+                  int64_t bstride, int box_x, int box_y) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)xdim, (cuuint64_t)ydim, (cuuint64_t)batch};
+  cuuint64_t gstride[2] = {(cuuint64_t)(ld * 4), (cuuint64_t)(bstride * 4)};
+  cuuint32_t box[3] = {(cuuint32_t)box_x, (cuuint32_t)box_y, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), gdim, gstride, box, estride,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   box_x == 32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -615,6 +754,13 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
     kp.nq = (int)((a.Cn + 127) / 128);
     kp.npt = (int)((a.R + 255) / 256);
     kp.ntiles = kp.nq * kp.npt * a.batch;
+    if (a.mask == 2 && a.batch == 1) {  // skip tiles entirely above the kept band
+      kp.lower = 1;
+      kp.mask_off = a.mask_off;
+      kp.ntiles = 0;
+      for (int pt = 0; pt < kp.npt; ++pt) kp.ntiles += lower_tiles(kp, pt);
+      if (kp.ntiles == 0) return cudaSuccess;
+    }
     kp.bs_p_row = a.bs_p_row;
     kp.bs_p_k = a.bs_p_k;
     kp.bs_q_row = a.bs_q_row;
@@ -628,12 +774,34 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
     kp.slot_bytes = kQTileBytes * split;
     kp.p_rows_max = 256;
   }
+  // TMA epilogue when the output allows it: beta 0 (store) or 1 (reduce-add),
+  // 16-byte aligned rows, and masks only where masked elements can add 0.
+  {
+    const int64_t bstride = a.batch > 1 ? a.bs_c_row * a.ldc + a.bs_c_col : a.ldc * (a.transpose ? a.Cn : a.R);
+    const float* cbase = a.C + a.c_row0 * a.ldc + a.c_col0;
+    bool ok = (a.beta == 0.f || a.beta == 1.f) && ((uintptr_t)cbase & 15u) == 0 && (a.ldc % 4) == 0 &&
+              (bstride % 4) == 0 && !(a.mask != 0 && a.beta == 0.f);
+    if (a.C_lo) {
+      const float* lbase = a.C_lo + a.c_row0 * a.ldc + a.c_col0;
+      ok = ok && a.beta == 0.f && kp.nchunks == 1 && ((uintptr_t)lbase & 15u) == 0;
+    }
+    if (ok) {
+      const int bx = a.transpose ? 32 : 128, by = a.transpose ? 128 : 32;
+      const int64_t xd = a.transpose ? a.R : a.Cn, yd = a.transpose ? a.Cn : a.R;
+      ok = make_out_map(&maps.c, cbase, xd, yd, a.ldc, a.batch, bstride, bx, by);
+      if (ok && a.C_lo)
+        ok = make_out_map(&maps.clo, a.C_lo + a.c_row0 * a.ldc + a.c_col0, xd, yd, a.ldc, a.batch, bstride, bx,
+                          by);
+    }
+    kp.epi_tma = ok ? 1 : 0;
+    kp.epi_split = (ok && a.C_lo) ? 1 : 0;
+  }
   kp.stage_bytes = kp.qslots * kp.slot_bytes + kp.p_rows_max * (int)kRowBytes * split;
   kp.stage_bytes = (kp.stage_bytes + 1023) & ~1023;
-  const int budget = 232448 - 1024 - 256;
+  const int budget = 232448 - 1024 - 256 - (kp.epi_tma ? 2 * (int)kStageTileBytes : 0);
   kp.stages = std::min(8, budget / kp.stage_bytes);
   if (kp.stages < 2) return cudaErrorInvalidValue;
-  const size_t smem = 1024 + (size_t)kp.stages * kp.stage_bytes + 256;
+  const size_t smem = 1024 + (size_t)kp.stages * kp.stage_bytes + (kp.epi_tma ? 2 * kStageTileBytes : 0) + 256;
   switch (a.op) {
     case OP_F16:
       return launch<OP_F16>(maps, kp, grid, smem, st);
