@@ -134,183 +134,206 @@ __global__ void __launch_bounds__(256) split_panel_kernel(const float* __restric
 
 // ------------------------------------------------------------------ leaf
 // Factor the 128 x 128 diagonal block k of R (lower Cholesky) and invert the
-// factor: L_kk into R, M_kk = L_kk^-1 into M and M_kk^T into Mt (all split).
-// One CTA of 512 threads; thread (ty, tx) keeps the 8 x 4 block rows
-// [8ty, 8ty+8) x columns [4tx, 4tx+4) in registers.
-//   Cholesky, right-looking and unnormalised: at pivot j the owners of
-//   column j publish it to shared memory (double-buffered), the pivot's owner
-//   publishes 1/d_j, one barrier, then every thread applies
-//   A[r][c] -= A[r][j] A[c][j] / d_j to its elements with j < c <= r.
-//   Afterwards L[r][c] = A[r][c] / sqrt(d_c).
-//   Inverse, right-looking on B = I: at step j row j of B becomes row j of
-//   M (times 1/L_jj), is published, and rows r > j subtract L[r][j] M[j][:].
+// factor: M_kk = L_kk^-1 into M and M_kk^T into Mt (both split).  One CTA of
+// 512 threads with A (the block, then L) and M in shared memory, recursively:
+//   f(o, h): f(o, h/2); L21 = A21 M11^T; A22 -= L21 L21^T; f(o + h/2, h/2);
+//            M21 = -M22 (L21 M11)
+// down to 32 x 32 blocks, which one warp factors and inverts in registers
+// with shuffles (no block-wide barrier per pivot).  The products between
+// levels are small shared-memory GEMMs over all 512 threads.
 // A pivot that is not positive raises ST_NOT_PD and is replaced by 1 so the
 // block stays finite.
 constexpr int LD = NB + 1;
 
+// Warp 0: A[o:o+32, o:o+32] -> L (lower, in place) and M[o:, o:] = L^-1.
+// Lane i keeps row i (Cholesky) or column i of M (inverse) in registers; the
+// window w[] slides by 4 columns every 4 steps so the loops stay rolled and
+// the code small.  Column j of L is broadcast through the shared scratch Lt
+// (Lt[j][k] = L[k][j]), read with vector loads.  Elements above the diagonal
+// of w are updated too: they are never read back.
+__device__ __forceinline__ void leaf32(float* A, float* M, float* Lt, float* rdiag, int o, PrepHeader* hdr) {
+  const int i = threadIdx.x & 31;
+  float w[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) w[c] = A[(o + i) * LD + o + c];
+#pragma unroll 1
+  for (int j4 = 0; j4 < 32; j4 += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j4 + u;                       // w[t] = column j4 + t of row i
+      float d = __shfl_sync(0xffffffffu, w[u], j);
+      if (!(d > 0.f) || !isfinite(d)) {
+        if (i == 0) raise_status(&hdr->status, ST_NOT_PD);
+        d = 1.f;
+      }
+      const float rs = rsqrtf(d);
+      const float lj = (i == j) ? d * rs : w[u] * rs;  // L[i][j] for i >= j
+      const float lstore = (i >= j) ? lj : 0.f;
+      A[(o + i) * LD + o + j] = lstore;
+      Lt[j * 32 + i] = lstore;
+      if (i == j) rdiag[j] = rs;                  // 1 / L[j][j]
+      __syncwarp();
+      const float* cj = Lt + j * 32 + j4;         // cj[t] = L[j4 + t][j]
+#pragma unroll
+      for (int t = u + 1; t < 4; ++t) w[t] = fmaf(-lj, cj[t], w[t]);
+#pragma unroll
+      for (int q = 1; q < 8; ++q) {
+        if (j4 + 4 * q >= 32) break;
+        const float4 c4 = *reinterpret_cast<const float4*>(cj + 4 * q);
+        w[4 * q + 0] = fmaf(-lj, c4.x, w[4 * q + 0]);
+        w[4 * q + 1] = fmaf(-lj, c4.y, w[4 * q + 1]);
+        w[4 * q + 2] = fmaf(-lj, c4.z, w[4 * q + 2]);
+        w[4 * q + 3] = fmaf(-lj, c4.w, w[4 * q + 3]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 28; ++t) w[t] = w[t + 4];
+#pragma unroll
+    for (int t = 28; t < 32; ++t) w[t] = 0.f;
+  }
+  __syncwarp();
+  // lane c: column c of M = L^-1, right-looking on the identity column:
+  // M[r][c] = b_r / L[r][r], then b_k -= L[k][r] M[r][c] for k > r
+#pragma unroll
+  for (int t = 0; t < 32; ++t) w[t] = (t == i) ? 1.f : 0.f;
+#pragma unroll 1
+  for (int r4 = 0; r4 < 32; r4 += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = r4 + u;
+      const float m = w[u] * rdiag[r];
+      M[(o + r) * LD + o + i] = m;
+      const float* cr = Lt + r * 32 + r4;         // cr[t] = L[r4 + t][r]
+#pragma unroll
+      for (int t = u + 1; t < 4; ++t) w[t] = fmaf(-cr[t], m, w[t]);
+#pragma unroll
+      for (int q = 1; q < 8; ++q) {
+        if (r4 + 4 * q >= 32) break;
+        const float4 c4 = *reinterpret_cast<const float4*>(cr + 4 * q);
+        w[4 * q + 0] = fmaf(-c4.x, m, w[4 * q + 0]);
+        w[4 * q + 1] = fmaf(-c4.y, m, w[4 * q + 1]);
+        w[4 * q + 2] = fmaf(-c4.z, m, w[4 * q + 2]);
+        w[4 * q + 3] = fmaf(-c4.w, m, w[4 * q + 3]);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 28; ++t) w[t] = w[t + 4];
+#pragma unroll
+    for (int t = 28; t < 32; ++t) w[t] = 0.f;
+  }
+  __syncwarp();
+}
+
+// C = sign * X op(Y) over H x H outputs in shared memory, all 512 threads,
+// each computing a 2 x 4 (H = 64) or 1 x 2 (H = 32) block; results are
+// written after every thread has read its operands.
+//   NT: C[r][c] = sum_t X[r][t] Y[c][t]      NN: C[r][c] = sum_t X[r][t] Y[t][c]
+// lower: keep only c <= r; accumulate: C += instead of C =.
+template <int H, bool NT>
+__device__ __forceinline__ void smem_gemm(const float* X, const float* Y, float* C, float sign, bool lower,
+                                          bool accumulate) {
+  constexpr int RB = H == 64 ? 2 : 1;           // rows per thread
+  constexpr int CB = H == 64 ? 4 : 2;           // columns per thread
+  constexpr int TPR = H / CB;                   // threads per row group
+  const int t = threadIdx.x;
+  const int r0 = (t / TPR) * RB, c0 = (t % TPR) * CB;
+  float acc[RB][CB] = {};
+#pragma unroll 4
+  for (int k = 0; k < H; ++k) {
+    float xv[RB], yv[CB];
+#pragma unroll
+    for (int u = 0; u < RB; ++u) xv[u] = X[(r0 + u) * LD + k];
+#pragma unroll
+    for (int v = 0; v < CB; ++v) yv[v] = NT ? Y[(c0 + v) * LD + k] : Y[k * LD + c0 + v];
+#pragma unroll
+    for (int u = 0; u < RB; ++u)
+#pragma unroll
+      for (int v = 0; v < CB; ++v) acc[u][v] = fmaf(xv[u], yv[v], acc[u][v]);
+  }
+  __syncthreads();
+#pragma unroll
+  for (int u = 0; u < RB; ++u)
+#pragma unroll
+    for (int v = 0; v < CB; ++v) {
+      const int r = r0 + u, c = c0 + v;
+      if (lower && c > r) continue;
+      const float x = sign * acc[u][v];
+      C[r * LD + c] = accumulate ? C[r * LD + c] + x : x;
+    }
+  __syncthreads();
+}
+
+// One level of the recursion for a block of size 2H at offset o.
+template <int H>
+__device__ __forceinline__ void leaf_merge_first(float* A, float* M, int o) {
+  float* A21 = A + (o + H) * LD + o;
+  float* A22 = A + (o + H) * LD + o + H;
+  const float* M11 = M + o * LD + o;
+  smem_gemm<H, true>(A21, M11, A21, 1.f, false, false);  // L21 = A21 M11^T
+  smem_gemm<H, true>(A21, A21, A22, -1.f, true, true);   // A22 -= L21 L21^T (lower)
+}
+template <int H>
+__device__ __forceinline__ void leaf_merge_second(float* A, float* M, int o) {
+  const float* L21 = A + (o + H) * LD + o;
+  const float* M11 = M + o * LD + o;
+  const float* M22 = M + (o + H) * LD + o + H;
+  float* X = A + o * LD + o + H;  // upper block of A: free space
+  smem_gemm<H, false>(L21, M11, X, 1.f, false, false);                  // X = L21 M11
+  smem_gemm<H, false>(M22, X, M + (o + H) * LD + o, -1.f, false, false);  // M21 = -M22 X
+}
+
 __global__ void __launch_bounds__(512) leaf_kernel(const float* R, float* Mh, float* Ml, float* Mth, float* Mtl,
                                                    int64_t np_, int k, PrepHeader* hdr) {
-  extern __shared__ float Ls[];            // [NB][LD]: L, then staging for M^T
-  __shared__ __align__(16) float colb[2][NB];  // published column (Cholesky) / row (inverse)
-  __shared__ float pinv[NB];               // 1 / d_j
-  __shared__ float rsq[NB];                // 1 / sqrt(d_j) = 1 / L_jj
-  __shared__ float dpiv[NB];               // d_j
-  const int tid = threadIdx.x, ty = tid >> 5, tx = tid & 31;
-  const int r0 = 8 * ty, c0 = 4 * tx;
+  extern __shared__ float sm[];
+  float* A = sm;             // [NB][LD]
+  float* M = sm + NB * LD;   // [NB][LD]
+  __shared__ __align__(16) float Lt[32 * 32];   // leaf32 scratch
+  __shared__ float rdiag[32];
   const int64_t o = (int64_t)k * NB;
-  float a[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t g = (o + r0 + i) * np_ + o + c0;
-    const float4 h = *reinterpret_cast<const float4*>(R + g);
-    a[i][0] = h.x;
-    a[i][1] = h.y;
-    a[i][2] = h.z;
-    a[i][3] = h.w;
+  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+    const int r = e / (NB / 4), c4 = (e % (NB / 4)) * 4;
+    const float4 v = *reinterpret_cast<const float4*>(R + (o + r) * np_ + o + c4);
+    A[r * LD + c4 + 0] = v.x;
+    A[r * LD + c4 + 1] = v.y;
+    A[r * LD + c4 + 2] = v.z;
+    A[r * LD + c4 + 3] = v.w;
   }
-  // ---------------------------------------------------------- Cholesky
-  for (int jj = 0; jj < NB / 4; ++jj) {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int j = 4 * jj + kk;
-      float* cb = colb[j & 1];
-      if (tx == jj) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (r0 + i >= j) cb[r0 + i] = a[i][kk];
-        if (ty == (j >> 3)) {
-          float d = (jj & 1) ? a[4 + kk][kk] : a[kk][kk];
-          if (!(d > 0.f) || !isfinite(d)) {
-            raise_status(&hdr->status, ST_NOT_PD);
-            d = 1.f;
-          }
-          dpiv[j] = d;
-          pinv[j] = 1.f / d;
-        }
-      }
-      __syncthreads();
-      // this block has elements with j < c <= r
-      if (r0 + 7 > j && c0 + 3 > j && c0 <= r0 + 7) {
-        const float dinv = pinv[j];
-        float cr[8], cc[4];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) cr[i] = cb[r0 + i] * dinv;
-        const float4 c4 = *reinterpret_cast<const float4*>(cb + c0);
-        cc[0] = c4.x;
-        cc[1] = c4.y;
-        cc[2] = c4.z;
-        cc[3] = c4.w;
-        if (c0 > j && c0 + 3 <= r0) {  // whole block strictly inside the update
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) a[i][q] = fmaf(-cr[i], cc[q], a[i][q]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int r = r0 + i, c = c0 + q;
-              if (r > j && c > j && c <= r) a[i][q] = fmaf(-cr[i], cc[q], a[i][q]);
-            }
-        }
-      }
-    }
-  }
-  if (tid < NB) rsq[tid] = 1.f / sqrtf(dpiv[tid]);
+  for (int e = threadIdx.x; e < NB * LD; e += blockDim.x) M[e] = 0.f;
   __syncthreads();
-  // L[r][c] = A[r][c] / sqrt(d_c) below the diagonal, sqrt(d_r) on it
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int r = r0 + i, c = c0 + q;
-      float v = 0.f;
-      if (c < r) v = a[i][q] * rsq[c];
-      if (c == r) v = sqrtf(dpiv[r]);
-      a[i][q] = v;
-      Ls[r * LD + c] = v;
-    }
+  const bool w0 = threadIdx.x < 32;
+  // first half (64)
+  if (w0) leaf32(A, M, Lt, rdiag, 0, hdr);
   __syncthreads();
-  // ---------------------------------------------------------- inverse
-  float b[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) b[i][q] = (r0 + i == c0 + q) ? 1.f : 0.f;
-  for (int jj = 0; jj < NB / 4; ++jj) {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const int j = 4 * jj + kk;
-      float* rb = colb[j & 1];
-      if (ty == (j >> 3)) {
-        const float s = rsq[j];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          float m;
-          if (jj & 1) {
-            m = b[4 + kk][q] * s;
-            b[4 + kk][q] = m;
-          } else {
-            m = b[kk][q] * s;
-            b[kk][q] = m;
-          }
-          rb[c0 + q] = m;
-        }
-      }
-      __syncthreads();
-      // rows r > j take row j of M, which is zero past column j
-      if (r0 + 7 > j && c0 <= j) {
-        float lr[8], mr[4];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) lr[i] = Ls[(r0 + i) * LD + j];
-        const float4 m4 = *reinterpret_cast<const float4*>(rb + c0);
-        mr[0] = m4.x;
-        mr[1] = m4.y;
-        mr[2] = m4.z;
-        mr[3] = m4.w;
-        if (r0 > j) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) b[i][q] = fmaf(-lr[i], mr[q], b[i][q]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            if (r0 + i > j)
-#pragma unroll
-              for (int q = 0; q < 4; ++q) b[i][q] = fmaf(-lr[i], mr[q], b[i][q]);
-        }
-      }
-    }
-  }
-  // ---------------------------------------------------------- write out
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t g = (o + r0 + i) * np_ + o + c0;
+  leaf_merge_first<32>(A, M, 0);
+  if (w0) leaf32(A, M, Lt, rdiag, 32, hdr);
+  __syncthreads();
+  leaf_merge_second<32>(A, M, 0);
+  // 128 level, first part
+  leaf_merge_first<64>(A, M, 0);
+  // second half (64)
+  if (w0) leaf32(A, M, Lt, rdiag, 64, hdr);
+  __syncthreads();
+  leaf_merge_first<32>(A, M, 64);
+  if (w0) leaf32(A, M, Lt, rdiag, 96, hdr);
+  __syncthreads();
+  leaf_merge_second<32>(A, M, 64);
+  // 128 level, second part
+  leaf_merge_second<64>(A, M, 0);
+  // write M and M^T (split)
+  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
+    const int r = e / (NB / 4), c4 = (e % (NB / 4)) * 4;
+    const int64_t g = (o + r) * np_ + o + c4;
     float4 h, l;
-    split_tf32(b[i][0], h.x, l.x);
-    split_tf32(b[i][1], h.y, l.y);
-    split_tf32(b[i][2], h.z, l.z);
-    split_tf32(b[i][3], h.w, l.w);
+    split_tf32(M[r * LD + c4 + 0], h.x, l.x);
+    split_tf32(M[r * LD + c4 + 1], h.y, l.y);
+    split_tf32(M[r * LD + c4 + 2], h.z, l.z);
+    split_tf32(M[r * LD + c4 + 3], h.w, l.w);
     *reinterpret_cast<float4*>(Mh + g) = h;
     *reinterpret_cast<float4*>(Ml + g) = l;
-  }
-  __syncthreads();  // Ls is reused for M
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) Ls[(r0 + i) * LD + c0 + q] = b[i][q];
-  __syncthreads();
-  // Mt[r][c] = M[c][r]
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int64_t g = (o + r0 + i) * np_ + o + c0;
-    float4 h, l;
-    split_tf32(Ls[(c0 + 0) * LD + r0 + i], h.x, l.x);
-    split_tf32(Ls[(c0 + 1) * LD + r0 + i], h.y, l.y);
-    split_tf32(Ls[(c0 + 2) * LD + r0 + i], h.z, l.z);
-    split_tf32(Ls[(c0 + 3) * LD + r0 + i], h.w, l.w);
+    split_tf32(M[(c4 + 0) * LD + r], h.x, l.x);
+    split_tf32(M[(c4 + 1) * LD + r], h.y, l.y);
+    split_tf32(M[(c4 + 2) * LD + r], h.z, l.z);
+    split_tf32(M[(c4 + 3) * LD + r], h.w, l.w);
     *reinterpret_cast<float4*>(Mth + g) = h;
     *reinterpret_cast<float4*>(Mtl + g) = l;
   }
@@ -414,7 +437,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     CUDA_TRY(cudaGetLastError());
   }
   static bool leaf_cfg = false;
-  const size_t leaf_smem = NB * LD * sizeof(float);
+  const size_t leaf_smem = 2 * NB * LD * sizeof(float);
   if (!leaf_cfg) {
     CUDA_TRY(cudaFuncSetAttribute(leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)leaf_smem));
     leaf_cfg = true;
