@@ -210,6 +210,61 @@ gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out,
                                   int32_t* zeros, int32_t* g_idx, float* loss,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/* Size of the fixed device scratch used by gptq_quantize_layer_noalloc:
+ * 16 MiB, enough for layers up to 1024 x 1024 at block_size 128. */
+#define GPTQ_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/*
+ * gptq_quantize_layer without a caller workspace and without allocating.
+ * The GPTQ paper has no counterpart to this call: it is a convenience of
+ * this library.  It is meant for callers that cannot allocate device memory
+ * at the moment they quantize: code running inside an allocator callback or
+ * an out-of-memory handler (allocating there would re-enter the allocator),
+ * code that must not add the device-wide synchronisation that cudaFree
+ * implies, and processes whose device memory is already fully claimed by a
+ * caching allocator.  Nothing inside this call runs cudaMalloc, cudaFree or
+ * any other routine that allocates device memory.
+ *
+ * Arguments, outputs and results are those of gptq_quantize_layer, without
+ * ws / ws_bytes.  Instead the call uses one static device array of
+ * GPTQ_STATIC_SCRATCH_BYTES bytes (256-byte aligned) that the library's
+ * device code carries; it exists once per device, from when that code is
+ * loaded on the device.
+ *
+ * Limit: a layer whose quantize workspace needs more than
+ * GPTQ_STATIC_SCRATCH_BYTES is rejected with GPTQ_ERR_WORKSPACE before any
+ * work is queued; gptq_last_error() gives the bytes needed.  Such layers
+ * need gptq_quantize_layer with a caller workspace.
+ *
+ * Device and setup: the call works on the calling thread's current device;
+ * stream must belong to it.  The first call on each device looks up the
+ * scratch's address with cudaGetSymbolAddress (which may also load the
+ * library's device code on that device) and caches it; make that first call
+ * before any stream capture begins.  Later calls only read the cached
+ * address.
+ *
+ * Zero state: no byte of the scratch has to start at zero.  Each call clears
+ * the scratch's 256-byte status header itself, on stream, before its first
+ * kernel, and writes every other scratch byte before reading it.
+ *
+ * Overlapping calls race: all calls on one device share the one scratch.
+ * Two calls whose device work overlaps in time (from two host threads, or on
+ * two streams with no ordering between them) corrupt each other's scratch and
+ * both results are undefined.  Order them: issue them on one stream, or make
+ * the later stream wait on an event recorded after the earlier call.  The
+ * call is asynchronous, so the scratch stays in use until stream has
+ * finished the call's work.
+ */
+gptq_status_t gptq_quantize_layer_noalloc(const void* W, gptq_dtype_t wt,
+                                          int64_t out, int64_t in, int64_t ldw,
+                                          const float* U, const int32_t* perm,
+                                          const uint8_t* dead,
+                                          const gptq_config_t* cfg,
+                                          int32_t* codes, uint32_t* qweight,
+                                          float* scales, int32_t* zeros,
+                                          int32_t* g_idx, float* loss,
+                                          void* stream);
+
 #ifdef __cplusplus
 }
 #endif

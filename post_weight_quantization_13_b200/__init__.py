@@ -7,6 +7,7 @@ carry the C ABI's names (``include/gptq.h``):
     gptq_hessian_accumulate(S, X, n_accum=None, stream=None)
     gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, stream=None)
     gptq_quantize_layer(W, U, perm, dead, cfg, scales, zeros, g_idx, ws, ...)
+    gptq_quantize_layer_noalloc(W, U, perm, dead, cfg, scales, zeros, g_idx, ...)
 
 plus ``solve_layer`` which allocates the outputs and workspace and makes the
 three calls in order.  If the shared library is missing the import fails: there
@@ -22,7 +23,8 @@ __all__ = [
     "GptqConfig", "GptqError", "LIB_PATH", "lib", "GPTQ_OK",
     "gptq_abi_version", "gptq_last_error", "gptq_kernel_launches", "gptq_validate_config",
     "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
-    "gptq_quantize_layer", "solve_layer", "STATUS_NAMES",
+    "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "GPTQ_STATIC_SCRATCH_BYTES",
+    "solve_layer", "STATUS_NAMES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
@@ -68,6 +70,12 @@ lib.gptq_quantize_layer.argtypes = [_p, ctypes.c_int, _i64, _i64, _i64, _p, _p, 
                                     ctypes.POINTER(_Config), _p, _p, _p, _p, _p, _p,
                                     _p, ctypes.c_size_t, _p]
 lib.gptq_quantize_layer.restype = ctypes.c_int
+lib.gptq_quantize_layer_noalloc.argtypes = [_p, ctypes.c_int, _i64, _i64, _i64, _p, _p, _p,
+                                            ctypes.POINTER(_Config), _p, _p, _p, _p, _p, _p, _p]
+lib.gptq_quantize_layer_noalloc.restype = ctypes.c_int
+
+# bytes of the library's static scratch (GPTQ_STATIC_SCRATCH_BYTES in gptq.h)
+GPTQ_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class GptqError(RuntimeError):
@@ -176,6 +184,19 @@ def gptq_quantize_layer(W, U, perm, dead, cfg, scales, zeros, g_idx, ws, codes=N
                                    _ptr(codes), _ptr(qweight), _ptr(scales), _ptr(zeros),
                                    _ptr(g_idx), _ptr(loss), _ptr(ws),
                                    ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def gptq_quantize_layer_noalloc(W, U, perm, dead, cfg, scales, zeros, g_idx, codes=None,
+                                qweight=None, loss=None, stream=None) -> None:
+    """gptq_quantize_layer on the library's static device scratch: allocates
+    nothing, for layers whose workspace fits GPTQ_STATIC_SCRATCH_BYTES.  Calls
+    on one device share that scratch and must not overlap in time."""
+    _rowmajor(W, "W")
+    c = GptqConfig.of(cfg).c()
+    _check(lib.gptq_quantize_layer_noalloc(_ptr(W), _dt(W), W.shape[0], W.shape[1], W.stride(0),
+                                           _ptr(U), _ptr(perm), _ptr(dead), ctypes.byref(c),
+                                           _ptr(codes), _ptr(qweight), _ptr(scales), _ptr(zeros),
+                                           _ptr(g_idx), _ptr(loss), _stream(stream)))
 
 
 def solve_layer(W, X=None, cfg=None, S=None, n=None, with_codes=True, stream=None):
