@@ -35,6 +35,16 @@ UNIT = "weights/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def kernel_sources_sha256():
+    """Hash of the sources the SYRK kernel is built from."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("tc_gemm.cu", "gemm.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "post_weight_quantization_13_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -200,6 +210,24 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x: float, pg, device) -> float:
+    """The maximum of x over all ranks (x itself without a process group).
+    Every rank must call it at the same point."""
+    if pg is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, weights_per_layer: int, layers: int, elapsed_ms: float) -> float:
+    """Weights/s of the whole job: every rank solves ``layers`` layers of
+    ``weights_per_layer`` weights in ``elapsed_ms`` (the slowest rank's time)."""
+    return world * weights_per_layer * layers / (elapsed_ms / 1e3)
+
+
 # ------------------------------------------------------------------ GPU
 def run_ours(args):
     import numpy as np
@@ -251,12 +279,13 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    phase_ms = {"hessian": [], "prepare": [], "quantize": []}
+    phase_ms = {"hessian": [], "prepare": [], "quantize": [], "syrk": []}
 
     def step(record=False):
-        e0, e1, e2, e3 = ev(), ev(), ev(), ev()
+        e0, es, e1, e2, e3 = ev(), ev(), ev(), ev(), ev()
         e0.record(stream)
         S.zero_()
+        es.record(stream)
         n = g.gptq_hessian_accumulate(S, X, 0, stream)
         e1.record(stream)
         g.gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, stream)
@@ -264,7 +293,7 @@ def run_ours(args):
         g.gptq_quantize_layer(W, U, perm, dead, cfg, scales, zeros, g_idx, ws, qweight=qweight,
                               stream=stream)
         e3.record(stream)
-        return (e0, e1, e2, e3) if record else None
+        return (e0, es, e1, e2, e3) if record else None
 
     for _ in range(args.warmup):
         step()
@@ -288,29 +317,41 @@ def run_ours(args):
     launches = g.gptq_kernel_launches() - launches0
     clocks = sampler.stop()
     elapsed = start.elapsed_time(end)  # ms
-    for e0, e1, e2, e3 in marks:
+    for e0, es, e1, e2, e3 in marks:
         phase_ms["hessian"].append(e0.elapsed_time(e1))
+        phase_ms["syrk"].append(es.elapsed_time(e1))
         phase_ms["prepare"].append(e1.elapsed_time(e2))
         phase_ms["quantize"].append(e2.elapsed_time(e3))
-    if pg:
-        t = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, pg, dev)
     ms_step = elapsed / args.steps
-    value = world * out * in_ * args.steps / (elapsed / 1e3)
+    value = job_throughput(world, out * in_, args.steps, elapsed)
 
-    # the dominant kernel: one tcgen05 SYRK launch per step (plus S.zero_)
-    hess_ms = statistics.mean(phase_ms["hessian"])
+    # the dominant kernel: one tcgen05 SYRK launch per step, timed alone
+    hess_ms = statistics.mean(phase_ms["syrk"])
     flops = in_ * (in_ + 1) * n_tok
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
     achieved = flops / (hess_ms / 1e3) / 1e12
+    # whole-step roofline: each step at the slower of its tensor-core and HBM
+    # floors (a1 Hessian and a4 factorisation on tensor cores, a6 lazy
+    # update and the gathers/packing on HBM), against the measured peaks
+    bw = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]) * 1e9
+    pf = peak * 1e12
+    nblk = -(-in_ // q.block_size)
+    terms = {"a1_hessian": flops / pf, "a4_factor": (2.0 / 3.0) * in_ ** 3 / pf,
+             "a6_lazy_update": 4.0 * out * in_ * max(nblk - 1, 0) / bw,
+             "a2_a3_a7_bytes": (8.0 * in_ * in_ + out * in_ * (2 + 4 + q.bits / 8)) / bw}
+    t_roof = sum(terms.values()) * 1e3
+    step_roof = {"t_roof_ms": t_roof, "frac": t_roof / ms_step,
+                 "terms_ms": {k: v * 1e3 for k, v in terms.items()}}
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         with open(tpath) as f:
             t = json.load(f).get(f"hessian_syrk:{wl.name}")
-        traffic = t.get("bytes_per_launch") if t else None
+        # counters taken on an older build of the kernel no longer apply
+        if t and t.get("kernel_sources_sha256") == kernel_sources_sha256():
+            traffic = t.get("bytes_per_launch")
 
     # e2e: host buffers in, results out, every step, through the same ABI calls
     e2e = None
@@ -332,14 +373,10 @@ def run_ours(args):
                 h.copy_(d, non_blocking=True)
         s1.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = s0.elapsed_time(s1)
-        if pg:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(s0.elapsed_time(s1), pg, dev)
         h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
         d2h = sum(t.numel() * t.element_size() for t in outs_d)
-        e2e = {"value": world * out * in_ * args.e2e_steps / (e_ms / 1e3), "unit": UNIT,
+        e2e = {"value": job_throughput(world, out * in_, args.e2e_steps, e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps}
 
@@ -368,6 +405,7 @@ def run_ours(args):
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16)",
                          "flops_per_launch": flops},
+            "step_roofline": step_roof,
             "gpu_launches": launches,
             "clocks": clocks,
             "e2e": e2e,
