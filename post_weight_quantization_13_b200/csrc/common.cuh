@@ -257,6 +257,20 @@ __device__ __forceinline__ uint64_t smem_desc_k_sw64(uint32_t smem_addr) {
   return d;
 }
 
+// The same for 128-byte swizzling: rows of 128 bytes, 8-row core groups
+// 1024 bytes apart, layout type SWIZZLE_128B = 2.  The start address may
+// step by 32 bytes inside the 128-byte row to select a K = 16 (16-bit) or
+// K = 8 (32-bit) slice; stage bases are 1024-byte aligned (base offset 0).
+__device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
 // Instruction descriptor: dense, fp32 accumulator (bits 4-5 = 1), A/B format
 // (bits 7-9 / 10-12: f16 = 0, bf16 = 1, tf32 = 2), both operands K-major
 // (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.

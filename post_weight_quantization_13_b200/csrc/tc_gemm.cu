@@ -45,8 +45,8 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kMaxPieces = 2;
-constexpr uint32_t kRowBytes = 64;                 // one K-major row per stage
-constexpr uint32_t kQTileBytes = 128 * kRowBytes;  // 8 KB per component
+constexpr uint32_t kRowBytes = 128;                // one K-major row per stage (128-byte swizzle)
+constexpr uint32_t kQTileBytes = 128 * kRowBytes;  // 16 KB per component
 constexpr int kNumBoxes = 5;                       // P boxes of 256, 128, 64, 32, 16 rows
 
 struct Piece {
@@ -175,15 +175,15 @@ template <int OP>
 struct OpTraits;
 template <>
 struct OpTraits<OP_F16> {
-  static constexpr int kSplit = 1, kBK = 32, kFmt = 0;
+  static constexpr int kSplit = 1, kBK = 64, kFmt = 0;
 };
 template <>
 struct OpTraits<OP_BF16> {
-  static constexpr int kSplit = 1, kBK = 32, kFmt = 1;
+  static constexpr int kSplit = 1, kBK = 64, kFmt = 1;
 };
 template <>
 struct OpTraits<OP_TF32X3> {
-  static constexpr int kSplit = 2, kBK = 16, kFmt = 2;
+  static constexpr int kSplit = 2, kBK = 32, kFmt = 2;
 };
 
 __device__ __forceinline__ void abort_cta(const KParams& kp, volatile int* abort_flag) {
@@ -359,15 +359,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t qa = sb + p.qslot * slot_bytes + h * kQTileBytes * SPLIT;
                 const uint32_t d = tacc + (uint32_t)(p.tcol + h * p.np);
 #pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
+                for (int kk = 0; kk < (int)(kRowBytes / 32); ++kk) {
                   const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
-                  const uint64_t ad = smem_desc_k_sw64(qa + kk * 32);
-                  const uint64_t bd = smem_desc_k_sw64(pb + kk * 32);
+                  const uint64_t ad = smem_desc_k_sw128(qa + kk * 32);
+                  const uint64_t bd = smem_desc_k_sw128(pb + kk * 32);
                   if (SPLIT == 1) {
                     umma_f16(d, ad, bd, idesc[i], acc);
                   } else {
-                    const uint64_t ad_lo = smem_desc_k_sw64(qa + kQTileBytes + kk * 32);
-                    const uint64_t bd_lo = smem_desc_k_sw64(pb + p_comp + kk * 32);
+                    const uint64_t ad_lo = smem_desc_k_sw128(qa + kQTileBytes + kk * 32);
+                    const uint64_t bd_lo = smem_desc_k_sw128(pb + p_comp + kk * 32);
                     umma_tf32(d, ad, bd, idesc[i], acc);
                     umma_tf32(d, ad, bd_lo, idesc[i], 1u);
                     umma_tf32(d, ad_lo, bd, idesc[i], 1u);
@@ -631,7 +631,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int6
   cuuint32_t box[2] = {(cuuint32_t)(kRowBytes / esize), (cuuint32_t)box_rows};
   cuuint32_t estride[2] = {1, 1};
   CUresult r = enc(m, dt, 2, const_cast<void*>(base), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -654,7 +654,7 @@ bool make_out_map(CUtensorMap* m, const float* base, int64_t xdim, int64_t ydim,
 }
 
 int esize_of(int op) { return op == OP_TF32X3 ? 4 : 2; }
-int bk_of(int op) { return op == OP_TF32X3 ? 16 : 32; }
+int bk_of(int op) { return op == OP_TF32X3 ? 32 : 64; }  // elements per 128-byte row
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
@@ -715,7 +715,7 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
   // core's in-place fp32 accumulation error grows with the number of MMAs
   // summed in one accumulator, while C gets round-to-nearest adds.  32768
   // elements of k per drain for 16-bit inputs, 4096 for 3xTF32.
-  const int chunk_tiles = split == 1 ? 1024 : 256;
+  const int chunk_tiles = (split == 1 ? 32768 : 4096) / bk_of(a.op);
   kp.kchunk = std::min(kp.kbc, chunk_tiles);
   kp.nchunks = (kp.kbc + kp.kchunk - 1) / kp.kchunk;
   kp.p_row0 = (int)a.p_row0;
