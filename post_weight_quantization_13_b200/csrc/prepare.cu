@@ -90,26 +90,39 @@ __global__ void __launch_bounds__(256) rank_kernel(const float* __restrict__ hd,
 }
 
 // ------------------------------------------------------------------ gather
-// R[a][b] = H_perm_damped[in-1-a][in-1-b] (split), identity in the padding.
+// Lower triangle (b <= a) of R[a][b] = H_perm_damped[in-1-a][in-1-b], with
+// the identity in the padding.  Only the lower triangle is ever read: the
+// factorisation's leaf ignores what lies above the diagonal and the trailing
+// updates add into lower tiles only.  With the natural order (i <= j for
+// b <= a) the S reads run along rows of the stored upper triangle, so they
+// coalesce; each block takes whole rows, four columns per thread.
 __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S, int64_t in, int64_t np_,
                                                      float scale, const int32_t* __restrict__ perm,
                                                      const uint8_t* __restrict__ dead, PrepHeader* hdr,
                                                      float* __restrict__ R) {
-  const int64_t a = blockIdx.y;
   const float lam = hdr->lambda;
-  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < np_; b += (int64_t)gridDim.x * blockDim.x) {
-    float v;
-    if (a < in && b < in) {
-      const int64_t i = perm[in - 1 - a], j = perm[in - 1 - b];
-      const int64_t lo = min(i, j), hi = max(i, j);
-      const float s = S[lo * in + hi];
-      if (!isfinite(s)) raise_status(&hdr->status, ST_NONFINITE);
-      v = s * scale;
-      if (i == j) v = (dead[i] ? 1.f : v) + lam;
-    } else {
-      v = (a == b) ? 1.f : 0.f;
+  for (int64_t a = blockIdx.x; a < np_; a += gridDim.x) {
+    const int64_t i = a < in ? perm[in - 1 - a] : -1;
+    for (int64_t b0 = (int64_t)threadIdx.x * 4; b0 <= a; b0 += (int64_t)blockDim.x * 4) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t b = b0 + u;
+        float x = 0.f;
+        if (a < in && b < in) {
+          const int64_t j = perm[in - 1 - b];
+          const int64_t lo = min(i, j), hi = max(i, j);
+          const float sv = S[lo * in + hi];
+          if (!isfinite(sv)) raise_status(&hdr->status, ST_NONFINITE);
+          x = sv * scale;
+          if (i == j) x = (dead[i] ? 1.f : x) + lam;
+        } else if (a == b) {
+          x = 1.f;
+        }
+        v[u] = x;
+      }
+      *reinterpret_cast<float4*>(R + a * np_ + b0) = make_float4(v[0], v[1], v[2], v[3]);
     }
-    R[a * np_ + b] = v;
   }
 }
 
@@ -146,80 +159,65 @@ __global__ void __launch_bounds__(256) split_panel_kernel(const float* __restric
 constexpr int LD = NB + 1;
 
 // Warp 0: A[o:o+32, o:o+32] -> L (lower, in place) and M[o:, o:] = L^-1.
-// Lane i keeps row i (Cholesky) or column i of M (inverse) in registers; the
-// window w[] slides by 4 columns every 4 steps so the loops stay rolled and
-// the code small.  Column j of L is broadcast through the shared scratch Lt
-// (Lt[j][k] = L[k][j]), read with vector loads.  Elements above the diagonal
-// of w are updated too: they are never read back.
-__device__ __forceinline__ void leaf32(float* A, float* M, float* Lt, float* rdiag, int o, PrepHeader* hdr) {
+// Lane i keeps row i (Cholesky) or column i of M (inverse) in registers as a
+// window w[t] = element j + t that slides by one column per pivot, so each
+// loop is rolled and small: code size, not arithmetic, sets the cost of a
+// routine that runs once per launch.  Column j of L goes through the shared
+// scratch Lt from the diagonal down (Lt[j][t] = L[j + t][j]) and is read back
+// with vector loads; window entries past the block's edge read stale scratch
+// and are never used.
+__device__ __noinline__ void leaf32(float* A, float* M, float* Lt, float* rdiag, int o, PrepHeader* hdr) {
   const int i = threadIdx.x & 31;
   float w[32];
 #pragma unroll
   for (int c = 0; c < 32; ++c) w[c] = A[(o + i) * LD + o + c];
 #pragma unroll 1
-  for (int j4 = 0; j4 < 32; j4 += 4) {
+  for (int j = 0; j < 32; ++j) {
+    float d = __shfl_sync(0xffffffffu, w[0], j);
+    if (!(d > 0.f) || !isfinite(d)) {
+      if (i == 0) raise_status(&hdr->status, ST_NOT_PD);
+      d = 1.f;
+    }
+    const float rs = rsqrtf(d);
+    const float lj = (i == j) ? d * rs : w[0] * rs;  // L[i][j] for i >= j
+    A[(o + i) * LD + o + j] = (i >= j) ? lj : 0.f;
+    if (i >= j) Lt[j * 32 + (i - j)] = lj;
+    if (i == j) rdiag[j] = rs;  // 1 / L[j][j]
+    __syncwarp();
+    const float* cj = Lt + j * 32;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = j4 + u;                       // w[t] = column j4 + t of row i
-      float d = __shfl_sync(0xffffffffu, w[u], j);
-      if (!(d > 0.f) || !isfinite(d)) {
-        if (i == 0) raise_status(&hdr->status, ST_NOT_PD);
-        d = 1.f;
-      }
-      const float rs = rsqrtf(d);
-      const float lj = (i == j) ? d * rs : w[u] * rs;  // L[i][j] for i >= j
-      const float lstore = (i >= j) ? lj : 0.f;
-      A[(o + i) * LD + o + j] = lstore;
-      Lt[j * 32 + i] = lstore;
-      if (i == j) rdiag[j] = rs;                  // 1 / L[j][j]
-      __syncwarp();
-      const float* cj = Lt + j * 32 + j4;         // cj[t] = L[j4 + t][j]
-#pragma unroll
-      for (int t = u + 1; t < 4; ++t) w[t] = fmaf(-lj, cj[t], w[t]);
-#pragma unroll
-      for (int q = 1; q < 8; ++q) {
-        if (j4 + 4 * q >= 32) break;
-        const float4 c4 = *reinterpret_cast<const float4*>(cj + 4 * q);
-        w[4 * q + 0] = fmaf(-lj, c4.x, w[4 * q + 0]);
-        w[4 * q + 1] = fmaf(-lj, c4.y, w[4 * q + 1]);
-        w[4 * q + 2] = fmaf(-lj, c4.z, w[4 * q + 2]);
-        w[4 * q + 3] = fmaf(-lj, c4.w, w[4 * q + 3]);
-      }
+    for (int q = 0; q < 8; ++q) {
+      const float4 c4 = *reinterpret_cast<const float4*>(cj + 4 * q);
+      if (q > 0) w[4 * q + 0] = fmaf(-lj, c4.x, w[4 * q + 0]);
+      w[4 * q + 1] = fmaf(-lj, c4.y, w[4 * q + 1]);
+      w[4 * q + 2] = fmaf(-lj, c4.z, w[4 * q + 2]);
+      w[4 * q + 3] = fmaf(-lj, c4.w, w[4 * q + 3]);
     }
 #pragma unroll
-    for (int t = 0; t < 28; ++t) w[t] = w[t + 4];
-#pragma unroll
-    for (int t = 28; t < 32; ++t) w[t] = 0.f;
+    for (int t = 0; t < 31; ++t) w[t] = w[t + 1];
+    w[31] = 0.f;
   }
   __syncwarp();
-  // lane c: column c of M = L^-1, right-looking on the identity column:
-  // M[r][c] = b_r / L[r][r], then b_k -= L[k][r] M[r][c] for k > r
+  // lane i: column i of M = L^-1 by forward substitution on the identity
+  // column, w[t] = b_{r+t}: M[r][i] = b_r / L[r][r]; b_k -= L[k][r] M[r][i]
 #pragma unroll
   for (int t = 0; t < 32; ++t) w[t] = (t == i) ? 1.f : 0.f;
 #pragma unroll 1
-  for (int r4 = 0; r4 < 32; r4 += 4) {
+  for (int r = 0; r < 32; ++r) {
+    const float m = w[0] * rdiag[r];
+    M[(o + r) * LD + o + i] = m;
+    const float* cr = Lt + r * 32;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int r = r4 + u;
-      const float m = w[u] * rdiag[r];
-      M[(o + r) * LD + o + i] = m;
-      const float* cr = Lt + r * 32 + r4;         // cr[t] = L[r4 + t][r]
-#pragma unroll
-      for (int t = u + 1; t < 4; ++t) w[t] = fmaf(-cr[t], m, w[t]);
-#pragma unroll
-      for (int q = 1; q < 8; ++q) {
-        if (r4 + 4 * q >= 32) break;
-        const float4 c4 = *reinterpret_cast<const float4*>(cr + 4 * q);
-        w[4 * q + 0] = fmaf(-c4.x, m, w[4 * q + 0]);
-        w[4 * q + 1] = fmaf(-c4.y, m, w[4 * q + 1]);
-        w[4 * q + 2] = fmaf(-c4.z, m, w[4 * q + 2]);
-        w[4 * q + 3] = fmaf(-c4.w, m, w[4 * q + 3]);
-      }
+    for (int q = 0; q < 8; ++q) {
+      const float4 c4 = *reinterpret_cast<const float4*>(cr + 4 * q);
+      if (q > 0) w[4 * q + 0] = fmaf(-c4.x, m, w[4 * q + 0]);
+      w[4 * q + 1] = fmaf(-c4.y, m, w[4 * q + 1]);
+      w[4 * q + 2] = fmaf(-c4.z, m, w[4 * q + 2]);
+      w[4 * q + 3] = fmaf(-c4.w, m, w[4 * q + 3]);
     }
 #pragma unroll
-    for (int t = 0; t < 28; ++t) w[t] = w[t + 4];
-#pragma unroll
-    for (int t = 28; t < 32; ++t) w[t] = 0.f;
+    for (int t = 0; t < 31; ++t) w[t] = w[t + 1];
+    w[31] = 0.f;
   }
   __syncwarp();
 }
@@ -287,7 +285,7 @@ __global__ void __launch_bounds__(512) leaf_kernel(const float* R, float* Mh, fl
   extern __shared__ float sm[];
   float* A = sm;             // [NB][LD]
   float* M = sm + NB * LD;   // [NB][LD]
-  __shared__ __align__(16) float Lt[32 * 32];   // leaf32 scratch
+  __shared__ __align__(16) float Lt[32 * 32 + 32];   // leaf32 scratch (+ window overrun)
   __shared__ float rdiag[32];
   const int64_t o = (int64_t)k * NB;
   for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
@@ -368,17 +366,38 @@ __global__ void __launch_bounds__(256) transpose_blocks_kernel(const float* __re
 }
 
 // U (column-major, in x in): U_cm[x][y] = Mt[in-1-x][in-1-y] for y <= x, 0 above.
+// U[x][y] = M[in-1-y][in-1-x] = Mt[in-1-x][in-1-y] for y <= x (U = J M J with
+// J the reversal), 0 above.  Rows of Mt are read backwards; with in % 4 == 0
+// four consecutive y map to one aligned float4 of Mt.
 __global__ void __launch_bounds__(256) write_u_kernel(const float* __restrict__ Mth, const float* __restrict__ Mtl,
                                                       int64_t np_, int64_t in, float* __restrict__ U) {
-  const int64_t x = blockIdx.y;
-  const int64_t src = (in - 1 - x) * np_;
-  for (int64_t y = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; y < in; y += (int64_t)gridDim.x * blockDim.x) {
-    float v = 0.f;
-    if (y <= x) {
-      const int64_t q = in - 1 - y;
-      v = Mth[src + q] + Mtl[src + q];
+  const bool vec = (in & 3) == 0;
+  for (int64_t x = blockIdx.x; x < in; x += gridDim.x) {
+    const int64_t src = (in - 1 - x) * np_;
+    if (vec) {
+      for (int64_t y = (int64_t)threadIdx.x * 4; y < in; y += (int64_t)blockDim.x * 4) {
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (y <= x) {
+          const int64_t q = in - 4 - y;  // Mt[.., q .. q+3] holds y+3 .. y
+          const float4 h = *reinterpret_cast<const float4*>(Mth + src + q);
+          const float4 l = *reinterpret_cast<const float4*>(Mtl + src + q);
+          o.x = h.w + l.w;
+          o.y = (y + 1 <= x) ? h.z + l.z : 0.f;
+          o.z = (y + 2 <= x) ? h.y + l.y : 0.f;
+          o.w = (y + 3 <= x) ? h.x + l.x : 0.f;
+        }
+        *reinterpret_cast<float4*>(U + x * in + y) = o;
+      }
+    } else {
+      for (int64_t y = threadIdx.x; y < in; y += blockDim.x) {
+        float v = 0.f;
+        if (y <= x) {
+          const int64_t q = in - 1 - y;
+          v = Mth[src + q] + Mtl[src + q];
+        }
+        U[x * in + y] = v;
+      }
     }
-    U[x * in + y] = v;
   }
 }
 
@@ -431,7 +450,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   note_launch();
   CUDA_TRY(cudaGetLastError());
   {
-    dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 16), (unsigned)np_);
+    const unsigned grid = (unsigned)std::min<int64_t>(np_, (int64_t)dev.sms * 8);
     gather_kernel<<<grid, 256, 0, st>>>(S, in, np_, scale, perm, dead, hdr, R);
     note_launch();
     CUDA_TRY(cudaGetLastError());
@@ -573,7 +592,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     groups.swap(next);
   }
   {
-    dim3 grid((unsigned)std::min<int64_t>((in + 255) / 256, 16), (unsigned)in);
+    const unsigned grid = (unsigned)std::min<int64_t>(in, (int64_t)dev.sms * 8);
     write_u_kernel<<<grid, 256, 0, st>>>(Mth, Mtl, np_, in, U);
     note_launch();
     CUDA_TRY(cudaGetLastError());

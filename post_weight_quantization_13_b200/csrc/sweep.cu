@@ -235,80 +235,72 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
 // then 1/U_jj.  One CTA per block.
 __global__ void __launch_bounds__(256) pack_diag_kernel(const float* __restrict__ U, int64_t in,
                                                         float* __restrict__ Ud) {
+  // blockIdx.x = diagonal block, blockIdx.y = which 16 of its 128 rows (c)
   const int64_t kB = (int64_t)blockIdx.x * BW;
   const int ncols = (int)((in - kB) < BW ? (in - kB) : BW);
   float* dst = Ud + (int64_t)blockIdx.x * kDiagBlockFloats;
-  for (int e = threadIdx.x; e < BW * 4 * UPITCH; e += blockDim.x) dst[e] = 0.f;
-  __syncthreads();
-  for (int e = threadIdx.x; e < BW * BW; e += blockDim.x) {
-    const int c = e / BW, j = e % BW;
-    if (c < ncols && j < ncols) {
-      const float v = U[(kB + c) * in + kB + j];
-      dst[(j * 4 + (c & 3)) * UPITCH + (c >> 2)] = v;
-      if (c == j) dst[BW * 4 * UPITCH + j] = 1.f / v;
-    }
+  const int c0 = blockIdx.y * 16;
+  if (blockIdx.y == 0)  // the pitch padding of every (j, q) slice
+    for (int e = threadIdx.x; e < BW * 4 * (UPITCH - BW / 4); e += blockDim.x)
+      dst[(e / (UPITCH - BW / 4)) * UPITCH + BW / 4 + e % (UPITCH - BW / 4)] = 0.f;
+  for (int e = threadIdx.x; e < 16 * BW; e += blockDim.x) {
+    const int c = c0 + e / BW, j = e % BW;
+    float v = 0.f;
+    if (c < ncols && j < ncols) v = U[(kB + c) * in + kB + j];
+    dst[(j * 4 + (c & 3)) * UPITCH + (c >> 2)] = v;
+    if (c == j) dst[BW * 4 * UPITCH + j] = (c < ncols) ? 1.f / v : 0.f;
   }
-  if (threadIdx.x >= ncols && threadIdx.x < BW) dst[BW * 4 * UPITCH + threadIdx.x] = 0.f;
 }
 
-// Wp[r][p] = W[r][perm[p]] (0 for dead channels and the padding).
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Wp[r][p] = W[r][perm[p]] in fp32 (0 for dead columns and the padding):
+// whole rows per block, four processed columns per thread.
 template <typename T>
 __global__ void __launch_bounds__(256) gather_w_kernel(const T* __restrict__ W, int64_t ldw_in, int64_t out,
                                                        int64_t in, int64_t np_, const int32_t* __restrict__ perm,
                                                        const uint8_t* __restrict__ dead, float* __restrict__ Wp) {
-  const int64_t r = blockIdx.y;
-  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < np_; p += (int64_t)gridDim.x * blockDim.x) {
-    float v = 0.f;
-    if (p < in) {
-      const int32_t c = perm[p];
-      if (!dead[c]) v = static_cast<float>(W[r * ldw_in + c]);
+  for (int64_t r = blockIdx.x; r < out; r += gridDim.x) {
+    for (int64_t p = (int64_t)threadIdx.x * 4; p < np_; p += (int64_t)blockDim.x * 4) {
+      float v[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        v[t] = 0.f;
+        if (p + t < in) {
+          const int32_t c = perm[p + t];
+          if (!dead[c]) v[t] = to_f32(W[r * ldw_in + c]);
+        }
+      }
+      *reinterpret_cast<float4*>(Wp + r * np_ + p) = make_float4(v[0], v[1], v[2], v[3]);
     }
-    Wp[r * np_ + p] = v;
-  }
-}
-template <>
-__global__ void __launch_bounds__(256) gather_w_kernel<__half>(const __half* __restrict__ W, int64_t ldw_in,
-                                                               int64_t out, int64_t in, int64_t np_,
-                                                               const int32_t* __restrict__ perm,
-                                                               const uint8_t* __restrict__ dead,
-                                                               float* __restrict__ Wp) {
-  const int64_t r = blockIdx.y;
-  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < np_; p += (int64_t)gridDim.x * blockDim.x) {
-    float v = 0.f;
-    if (p < in) {
-      const int32_t c = perm[p];
-      if (!dead[c]) v = __half2float(W[r * ldw_in + c]);
-    }
-    Wp[r * np_ + p] = v;
-  }
-}
-template <>
-__global__ void __launch_bounds__(256) gather_w_kernel<__nv_bfloat16>(const __nv_bfloat16* __restrict__ W,
-                                                                      int64_t ldw_in, int64_t out, int64_t in,
-                                                                      int64_t np_, const int32_t* __restrict__ perm,
-                                                                      const uint8_t* __restrict__ dead,
-                                                                      float* __restrict__ Wp) {
-  const int64_t r = blockIdx.y;
-  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < np_; p += (int64_t)gridDim.x * blockDim.x) {
-    float v = 0.f;
-    if (p < in) {
-      const int32_t c = perm[p];
-      if (!dead[c]) v = __bfloat162float(W[r * ldw_in + c]);
-    }
-    Wp[r * np_ + p] = v;
   }
 }
 
 // Uh/Ul[c][j] = split(Ucm[c][j]) with the padding zero.
 __global__ void __launch_bounds__(256) split_u_kernel(const float* __restrict__ U, int64_t in, int64_t np_,
                                                       float* __restrict__ Uh, float* __restrict__ Ul) {
-  const int64_t c = blockIdx.y;
-  for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < np_; j += (int64_t)gridDim.x * blockDim.x) {
-    const float v = (c < in && j < in) ? U[c * in + j] : 0.f;
-    float h, l;
-    split_tf32(v, h, l);
-    Uh[c * np_ + j] = h;
-    Ul[c * np_ + j] = l;
+  // four columns per thread; U rows are float4-aligned when in % 4 == 0
+  const bool vec = (in & 3) == 0;
+  for (int64_t c = blockIdx.x; c < np_; c += gridDim.x) {
+    for (int64_t j = (int64_t)threadIdx.x * 4; j < np_; j += (int64_t)blockDim.x * 4) {
+      float v[4];
+      if (vec && c < in && j + 3 < in) {
+        const float4 u = *reinterpret_cast<const float4*>(U + c * in + j);
+        v[0] = u.x, v[1] = u.y, v[2] = u.z, v[3] = u.w;
+      } else {
+#pragma unroll
+        for (int t = 0; t < 4; ++t) v[t] = (c < in && j + t < in) ? U[c * in + j + t] : 0.f;
+      }
+      float4 h, l;
+      split_tf32(v[0], h.x, l.x);
+      split_tf32(v[1], h.y, l.y);
+      split_tf32(v[2], h.z, l.z);
+      split_tf32(v[3], h.w, l.w);
+      *reinterpret_cast<float4*>(Uh + c * np_ + j) = h;
+      *reinterpret_cast<float4*>(Ul + c * np_ + j) = l;
+    }
   }
 }
 
@@ -423,7 +415,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
   CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
   if (loss) CUDA_TRY(cudaMemsetAsync(loss, 0, sizeof(float) * out, st));
   {
-    dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 32), (unsigned)out);
+    const unsigned grid = (unsigned)std::min<int64_t>(out, (int64_t)dev.sms * 8);
     switch (wt) {
       case GPTQ_F16:
         gather_w_kernel<__half><<<grid, 256, 0, st>>>((const __half*)W, ldw, out, in, np_, perm, dead, Wp);
@@ -442,11 +434,11 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
     CUDA_TRY(cudaGetLastError());
   }
   {
-    dim3 grid((unsigned)std::min<int64_t>((np_ + 255) / 256, 32), (unsigned)np_);
+    const unsigned grid = (unsigned)std::min<int64_t>(np_, (int64_t)dev.sms * 8);
     split_u_kernel<<<grid, 256, 0, st>>>(U, in, np_, Uh, Ul);
     note_launch();
     CUDA_TRY(cudaGetLastError());
-    pack_diag_kernel<<<(unsigned)(np_ / BW), 256, 0, st>>>(U, in, Ud);
+    pack_diag_kernel<<<dim3((unsigned)(np_ / BW), BW / 16), 256, 0, st>>>(U, in, Ud);
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
