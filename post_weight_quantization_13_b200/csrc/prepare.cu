@@ -11,16 +11,17 @@
 // Cholesky and one triangular inverse (2/3 n^3 flops) instead of
 // factor -> invert -> factor again.
 //
-// Working matrices are kept "split" (hi rounded to tf32 plus exact fp32
-// remainder) so every block product runs on the tensor cores with 3xTF32
-// accuracy.  The matrix is padded to a multiple of 128 with identity
-// (block-diagonal, so the padding never mixes with the real channels).
-//   Cholesky:  right-looking, 128-wide panels; the diagonal block is
-//              factored and inverted in one CTA (leaf_kernel), the panel is
-//              R_ik M_kk^T and the trailing update R -= L_ik L_jk^T.
+// The matrix is padded to a multiple of 128 with identity (block-diagonal,
+// so the padding never mixes with the real channels).
+//   Cholesky:  right-looking with 64-wide blocks in one cooperative launch
+//              (factor_kernel): one CTA factors and inverts each diagonal
+//              block while the others form the panel L_ik = R_ik M_kk^T and
+//              the trailing update R -= L_ik L_jk^T, in fp32.
 //   Inverse:   pairs of already inverted diagonal groups are merged,
 //              M21 = -M22 (L21 M11), doubling the group size each level; all
-//              merges of one level are one batched launch.
+//              merges of one level are one batched tensor-core launch on
+//              "split" operands (hi rounded to tf32 plus the exact fp32
+//              remainder, 3xTF32 accuracy).
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -126,51 +127,40 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
   }
 }
 
-// Pk[r][c] = split(R[r0 + r][kB + c]): the panel below diagonal block k as a
-// 3xTF32 operand (rows x 128, row stride 128).
-__global__ void __launch_bounds__(256) split_panel_kernel(const float* __restrict__ R, int64_t np_, int64_t r0,
-                                                          int64_t kB, int64_t rows, float* __restrict__ Ph,
-                                                          float* __restrict__ Pl) {
-  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * 32;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t r = e >> 5, c4 = (e & 31) << 2;
-    const float4 v = *reinterpret_cast<const float4*>(R + (r0 + r) * np_ + kB + c4);
-    float4 h, l;
-    split_tf32(v.x, h.x, l.x);
-    split_tf32(v.y, h.y, l.y);
-    split_tf32(v.z, h.z, l.z);
-    split_tf32(v.w, h.w, l.w);
-    *reinterpret_cast<float4*>(Ph + r * 128 + c4) = h;
-    *reinterpret_cast<float4*>(Pl + r * 128 + c4) = l;
-  }
-}
+// ------------------------------------------------------------------ factor
+// Blocked right-looking Cholesky of R = L L^T in one cooperative launch (all
+// CTAs resident), with FB x FB blocks.  Step k (after a grid barrier):
+//   CTA 0      panel tile (k+1, k): L = A M_kk^T; then A_{k+1,k+1} -= L L^T
+//              and the leaf: L_{k+1,k+1} and its inverse M_{k+1,k+1};
+//   CTAs 1..   the other panel tiles L_ik = A_ik M_kk^T (i > k + 1), then
+//              the trailing tiles A_ij -= L_ik L_jk^T (i >= j > k, except
+//              (k+1, k+1)) once every panel tile of the step is done (a
+//              per-step counter).
+// So the factorisation of the next diagonal block overlaps the trailing
+// update of this step.  Tile products are fp32 FMA on register blocks.
+// Tiles that other CTAs write during the launch are read with L2-only loads
+// (the L1 caches are not coherent), after a flag or barrier with fences.
+// Outputs: L's tiles below the diagonal (fp32 in R, split hi/lo in Lh/Ll)
+// and the diagonal blocks of M = L^-1 (fp32 in MD; split in Mh/Ml and
+// transposed in Mth/Mtl), which the blocked inverse then merges.
+constexpr int FB = 64;          // block size
+constexpr int FNT = 256;        // threads per CTA
+constexpr int FP = FB + 1;      // pitch of the leaf's A and M tiles
+constexpr int TP = FB + 4;      // pitch of transposed operand tiles (float4 rows)
 
-// ------------------------------------------------------------------ leaf
-// Factor the 128 x 128 diagonal block k of R (lower Cholesky) and invert the
-// factor: M_kk = L_kk^-1 into M and M_kk^T into Mt (both split).  One CTA of
-// 512 threads with A (the block, then L) and M in shared memory, recursively:
-//   f(o, h): f(o, h/2); L21 = A21 M11^T; A22 -= L21 L21^T; f(o + h/2, h/2);
-//            M21 = -M22 (L21 M11)
-// down to 32 x 32 blocks, which one warp factors and inverts in registers
-// with shuffles (no block-wide barrier per pivot).  The products between
-// levels are small shared-memory GEMMs over all 512 threads.
-// A pivot that is not positive raises ST_NOT_PD and is replaced by 1 so the
-// block stays finite.
-constexpr int LD = NB + 1;
-
-// Warp 0: A[o:o+32, o:o+32] -> L (lower, in place) and M[o:, o:] = L^-1.
-// Lane i keeps row i (Cholesky) or column i of M (inverse) in registers as a
-// window w[t] = element j + t that slides by one column per pivot, so each
-// loop is rolled and small: code size, not arithmetic, sets the cost of a
-// routine that runs once per launch.  Column j of L goes through the shared
-// scratch Lt from the diagonal down (Lt[j][t] = L[j + t][j]) and is read back
-// with vector loads; window entries past the block's edge read stale scratch
-// and are never used.
+// Warp 0: A[o:o+32, o:o+32] -> L (lower, in place) and M[o:, o:] = L^-1
+// (pitch P).  Lane i keeps row i (Cholesky) or column i of M (inverse) in
+// registers as a window w[t] = element j + t that slides by one column per
+// pivot, so each loop is rolled and small.  Column j of L goes through the
+// shared scratch Lt from the diagonal down (Lt[j][t] = L[j + t][j]) and is
+// read back with vector loads; window entries past the block's edge read
+// stale scratch and are never used.
+template <int P>
 __device__ __noinline__ void leaf32(float* A, float* M, float* Lt, float* rdiag, int o, PrepHeader* hdr) {
   const int i = threadIdx.x & 31;
   float w[32];
 #pragma unroll
-  for (int c = 0; c < 32; ++c) w[c] = A[(o + i) * LD + o + c];
+  for (int c = 0; c < 32; ++c) w[c] = A[(o + i) * P + o + c];
 #pragma unroll 1
   for (int j = 0; j < 32; ++j) {
     float d = __shfl_sync(0xffffffffu, w[0], j);
@@ -180,7 +170,7 @@ __device__ __noinline__ void leaf32(float* A, float* M, float* Lt, float* rdiag,
     }
     const float rs = rsqrtf(d);
     const float lj = (i == j) ? d * rs : w[0] * rs;  // L[i][j] for i >= j
-    A[(o + i) * LD + o + j] = (i >= j) ? lj : 0.f;
+    A[(o + i) * P + o + j] = (i >= j) ? lj : 0.f;
     if (i >= j) Lt[j * 32 + (i - j)] = lj;
     if (i == j) rdiag[j] = rs;  // 1 / L[j][j]
     __syncwarp();
@@ -205,7 +195,7 @@ __device__ __noinline__ void leaf32(float* A, float* M, float* Lt, float* rdiag,
 #pragma unroll 1
   for (int r = 0; r < 32; ++r) {
     const float m = w[0] * rdiag[r];
-    M[(o + r) * LD + o + i] = m;
+    M[(o + r) * P + o + i] = m;
     const float* cr = Lt + r * 32;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -222,120 +212,314 @@ __device__ __noinline__ void leaf32(float* A, float* M, float* Lt, float* rdiag,
   __syncwarp();
 }
 
-// C = sign * X op(Y) over H x H outputs in shared memory, all 512 threads,
-// each computing a 2 x 4 (H = 64) or 1 x 2 (H = 32) block; results are
+// 32 x 32 products inside the leaf (FNT threads, 2 x 2 outputs each), pitch FP:
+//   NT: C[r][c] = sign * sum_t X[r][t] Y[c][t]     NN: ... X[r][t] Y[t][c]
+// lower: keep only c <= r; accumulate: C += instead of C =.  Results are
 // written after every thread has read its operands.
-//   NT: C[r][c] = sum_t X[r][t] Y[c][t]      NN: C[r][c] = sum_t X[r][t] Y[t][c]
-// lower: keep only c <= r; accumulate: C += instead of C =.
-template <int H, bool NT>
-__device__ __forceinline__ void smem_gemm(const float* X, const float* Y, float* C, float sign, bool lower,
-                                          bool accumulate) {
-  constexpr int RB = H == 64 ? 2 : 1;           // rows per thread
-  constexpr int CB = H == 64 ? 4 : 2;           // columns per thread
-  constexpr int TPR = H / CB;                   // threads per row group
+template <bool NT>
+__device__ __forceinline__ void gemm32(const float* X, const float* Y, float* C, float sign, bool lower,
+                                       bool accumulate) {
   const int t = threadIdx.x;
-  const int r0 = (t / TPR) * RB, c0 = (t % TPR) * CB;
-  float acc[RB][CB] = {};
+  const int r0 = (t / 16) * 2, c0 = (t % 16) * 2;
+  float acc[2][2] = {};
 #pragma unroll 4
-  for (int k = 0; k < H; ++k) {
-    float xv[RB], yv[CB];
-#pragma unroll
-    for (int u = 0; u < RB; ++u) xv[u] = X[(r0 + u) * LD + k];
-#pragma unroll
-    for (int v = 0; v < CB; ++v) yv[v] = NT ? Y[(c0 + v) * LD + k] : Y[k * LD + c0 + v];
-#pragma unroll
-    for (int u = 0; u < RB; ++u)
-#pragma unroll
-      for (int v = 0; v < CB; ++v) acc[u][v] = fmaf(xv[u], yv[v], acc[u][v]);
+  for (int k = 0; k < 32; ++k) {
+    const float x0 = X[r0 * FP + k], x1 = X[(r0 + 1) * FP + k];
+    const float y0 = NT ? Y[c0 * FP + k] : Y[k * FP + c0];
+    const float y1 = NT ? Y[(c0 + 1) * FP + k] : Y[k * FP + c0 + 1];
+    acc[0][0] = fmaf(x0, y0, acc[0][0]);
+    acc[0][1] = fmaf(x0, y1, acc[0][1]);
+    acc[1][0] = fmaf(x1, y0, acc[1][0]);
+    acc[1][1] = fmaf(x1, y1, acc[1][1]);
   }
   __syncthreads();
 #pragma unroll
-  for (int u = 0; u < RB; ++u)
+  for (int u = 0; u < 2; ++u)
 #pragma unroll
-    for (int v = 0; v < CB; ++v) {
+    for (int v = 0; v < 2; ++v) {
       const int r = r0 + u, c = c0 + v;
       if (lower && c > r) continue;
       const float x = sign * acc[u][v];
-      C[r * LD + c] = accumulate ? C[r * LD + c] + x : x;
+      C[r * FP + c] = accumulate ? C[r * FP + c] + x : x;
     }
   __syncthreads();
 }
 
-// One level of the recursion for a block of size 2H at offset o.
-template <int H>
-__device__ __forceinline__ void leaf_merge_first(float* A, float* M, int o) {
-  float* A21 = A + (o + H) * LD + o;
-  float* A22 = A + (o + H) * LD + o + H;
-  const float* M11 = M + o * LD + o;
-  smem_gemm<H, true>(A21, M11, A21, 1.f, false, false);  // L21 = A21 M11^T
-  smem_gemm<H, true>(A21, A21, A22, -1.f, true, true);   // A22 -= L21 L21^T (lower)
-}
-template <int H>
-__device__ __forceinline__ void leaf_merge_second(float* A, float* M, int o) {
-  const float* L21 = A + (o + H) * LD + o;
-  const float* M11 = M + o * LD + o;
-  const float* M22 = M + (o + H) * LD + o + H;
-  float* X = A + o * LD + o + H;  // upper block of A: free space
-  smem_gemm<H, false>(L21, M11, X, 1.f, false, false);                  // X = L21 M11
-  smem_gemm<H, false>(M22, X, M + (o + H) * LD + o, -1.f, false, false);  // M21 = -M22 X
+// The FB x FB leaf on A (lower triangle read) and M (zeroed by the caller):
+// two 32-blocks and their merge.  Leaves L in A's lower triangle, M = L^-1.
+__device__ void leaf64(float* A, float* M, float* Lt, float* rdiag, PrepHeader* hdr) {
+  const bool w0 = threadIdx.x < 32;
+  if (w0) leaf32<FP>(A, M, Lt, rdiag, 0, hdr);
+  __syncthreads();
+  float* A21 = A + 32 * FP;
+  float* A22 = A + 32 * FP + 32;
+  gemm32<true>(A21, M, A21, 1.f, false, false);   // L21 = A21 M11^T
+  gemm32<true>(A21, A21, A22, -1.f, true, true);  // A22 -= L21 L21^T (lower)
+  if (w0) leaf32<FP>(A, M, Lt, rdiag, 32, hdr);
+  __syncthreads();
+  float* X = A + 32;                                            // A's upper block: free space
+  gemm32<false>(A21, M, X, 1.f, false, false);                  // X = L21 M11
+  gemm32<false>(M + 32 * FP + 32, X, M + 32 * FP, -1.f, false, false);  // M21 = -M22 X
 }
 
-__global__ void __launch_bounds__(512) leaf_kernel(const float* R, float* Mh, float* Ml, float* Mth, float* Mtl,
-                                                   int64_t np_, int k, PrepHeader* hdr) {
-  extern __shared__ float sm[];
-  float* A = sm;             // [NB][LD]
-  float* M = sm + NB * LD;   // [NB][LD]
-  __shared__ __align__(16) float Lt[32 * 32 + 32];   // leaf32 scratch (+ window overrun)
-  __shared__ float rdiag[32];
-  const int64_t o = (int64_t)k * NB;
-  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
-    const int r = e / (NB / 4), c4 = (e % (NB / 4)) * 4;
-    const float4 v = *reinterpret_cast<const float4*>(R + (o + r) * np_ + o + c4);
-    A[r * LD + c4 + 0] = v.x;
-    A[r * LD + c4 + 1] = v.y;
-    A[r * LD + c4 + 2] = v.z;
-    A[r * LD + c4 + 3] = v.w;
-  }
-  for (int e = threadIdx.x; e < NB * LD; e += blockDim.x) M[e] = 0.f;
-  __syncthreads();
-  const bool w0 = threadIdx.x < 32;
-  // first half (64)
-  if (w0) leaf32(A, M, Lt, rdiag, 0, hdr);
-  __syncthreads();
-  leaf_merge_first<32>(A, M, 0);
-  if (w0) leaf32(A, M, Lt, rdiag, 32, hdr);
-  __syncthreads();
-  leaf_merge_second<32>(A, M, 0);
-  // 128 level, first part
-  leaf_merge_first<64>(A, M, 0);
-  // second half (64)
-  if (w0) leaf32(A, M, Lt, rdiag, 64, hdr);
-  __syncthreads();
-  leaf_merge_first<32>(A, M, 64);
-  if (w0) leaf32(A, M, Lt, rdiag, 96, hdr);
-  __syncthreads();
-  leaf_merge_second<32>(A, M, 64);
-  // 128 level, second part
-  leaf_merge_second<64>(A, M, 0);
-  // write M and M^T (split)
-  for (int e = threadIdx.x; e < NB * NB / 4; e += blockDim.x) {
-    const int r = e / (NB / 4), c4 = (e % (NB / 4)) * 4;
-    const int64_t g = (o + r) * np_ + o + c4;
-    float4 h, l;
-    split_tf32(M[r * LD + c4 + 0], h.x, l.x);
-    split_tf32(M[r * LD + c4 + 1], h.y, l.y);
-    split_tf32(M[r * LD + c4 + 2], h.z, l.z);
-    split_tf32(M[r * LD + c4 + 3], h.w, l.w);
-    *reinterpret_cast<float4*>(Mh + g) = h;
-    *reinterpret_cast<float4*>(Ml + g) = l;
-    split_tf32(M[(c4 + 0) * LD + r], h.x, l.x);
-    split_tf32(M[(c4 + 1) * LD + r], h.y, l.y);
-    split_tf32(M[(c4 + 2) * LD + r], h.z, l.z);
-    split_tf32(M[(c4 + 3) * LD + r], h.w, l.w);
-    *reinterpret_cast<float4*>(Mth + g) = h;
-    *reinterpret_cast<float4*>(Mtl + g) = l;
+// T[t][r] = G[r][t] for an FB x FB tile of a row-major matrix (row stride ld).
+__device__ __forceinline__ void load_tile_t(float* T, const float* G, int64_t ld) {
+  for (int e = threadIdx.x; e < FB * FB / 4; e += FNT) {
+    const int r = e % FB, t4 = (e / FB) * 4;
+    const float4 v = __ldcg(reinterpret_cast<const float4*>(G + (int64_t)r * ld + t4));
+    T[(t4 + 0) * TP + r] = v.x;
+    T[(t4 + 1) * TP + r] = v.y;
+    T[(t4 + 2) * TP + r] = v.z;
+    T[(t4 + 3) * TP + r] = v.w;
   }
 }
+
+// acc[u][v] = sum_t X[t][r0 + u] Y[t][c0 + v] over an FB-long inner dimension
+// (X, Y transposed tiles); thread t owns rows 4 (t / 16) and columns 4 (t % 16).
+__device__ __forceinline__ void tile_product(const float* X, const float* Y, float acc[4][4]) {
+  const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+#pragma unroll 4
+  for (int t = 0; t < FB; ++t) {
+    const float4 x = *reinterpret_cast<const float4*>(X + t * TP + r0);
+    const float4 y = *reinterpret_cast<const float4*>(Y + t * TP + c0);
+    const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(xs[u], ys[v], acc[u][v]);
+  }
+}
+
+struct FactorParams {
+  float* R;
+  int64_t np_;
+  int T;          // blocks per side
+  float* MD;      // [T][FB][FB] diagonal blocks of M (fp32)
+  float *Lh, *Ll, *Mh, *Ml, *Mth, *Mtl;
+  unsigned* sync;  // [0] arrivals, [1] generation, [2] abort
+  int* pdone;      // [T]: panel tiles finished in step k
+  PrepHeader* hdr;
+};
+
+// Grid-wide barrier for a cooperative launch, bounded by kWaitLimitNs.
+// Returns false once any CTA has given up (all CTAs then leave the loop).
+__device__ bool grid_barrier(const FactorParams& fp) {
+  __shared__ int ok_s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile unsigned* vs = fp.sync;
+    const unsigned gen = vs[1];
+    __threadfence();
+    bool ok = true;
+    if (atomicAdd(&fp.sync[0], 1u) == gridDim.x - 1) {
+      atomicExch(&fp.sync[0], 0u);
+      __threadfence();
+      atomicAdd(&fp.sync[1], 1u);
+    } else {
+      const uint64_t t0 = globaltimer();
+      while (vs[1] == gen) {
+        if (vs[2]) break;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          raise_status(&fp.hdr->status, ST_TIMEOUT);
+          atomicExch(&fp.sync[2], 1u);
+          break;
+        }
+      }
+    }
+    __threadfence();
+    ok_s = ok && vs[2] == 0;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// Wait until pdone[k] (panel tiles finished in step k) reaches target
+// (bounded); false on timeout or abort.
+__device__ bool wait_panels(const FactorParams& fp, int k, int target) {
+  __shared__ int ok_s;
+  if (threadIdx.x == 0) {
+    volatile int* vf = fp.pdone;
+    volatile unsigned* vs = fp.sync;
+    bool ok = true;
+    const uint64_t t0 = globaltimer();
+    while (vf[k] < target) {
+      if (vs[2]) {
+        ok = false;
+        break;
+      }
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        raise_status(&fp.hdr->status, ST_TIMEOUT);
+        atomicExch(&fp.sync[2], 1u);
+        ok = false;
+        break;
+      }
+    }
+    __threadfence();
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// Write the leaf's M (pitch FP) as diagonal block b: fp32 to MD, split to
+// Mh/Ml and, transposed, to Mth/Mtl.
+__device__ void store_diag_m(const FactorParams& fp, const float* M, int b) {
+  const int64_t o = (int64_t)b * FB;
+  float* md = fp.MD + (int64_t)b * FB * FB;
+  for (int e = threadIdx.x; e < FB * FB; e += FNT) {
+    const int r = e / FB, c = e % FB;
+    const float v = M[r * FP + c], vt = M[c * FP + r];
+    md[e] = v;
+    float h, l;
+    split_tf32(v, h, l);
+    fp.Mh[(o + r) * fp.np_ + o + c] = h;
+    fp.Ml[(o + r) * fp.np_ + o + c] = l;
+    split_tf32(vt, h, l);
+    fp.Mth[(o + r) * fp.np_ + o + c] = h;
+    fp.Mtl[(o + r) * fp.np_ + o + c] = l;
+  }
+}
+
+// Panel tile (i, k): L_ik = A_ik M_kk^T.  X, Y: transposed operand tiles.
+// Writes R (fp32) and Lh/Ll (split); leaves acc in registers.
+__device__ void panel_tile(const FactorParams& fp, int i, int k, float* X, float* Y, float acc[4][4]) {
+  const int64_t np_ = fp.np_;
+  float* Rt = fp.R + (int64_t)i * FB * np_ + (int64_t)k * FB;
+  load_tile_t(X, Rt, np_);
+  load_tile_t(Y, fp.MD + (int64_t)k * FB * FB, FB);
+  __syncthreads();
+  tile_product(X, Y, acc);
+  const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int64_t g = (int64_t)(r0 + u) * np_ + c0;
+    *reinterpret_cast<float4*>(Rt + g) = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+    float4 h, l;
+    split_tf32(acc[u][0], h.x, l.x);
+    split_tf32(acc[u][1], h.y, l.y);
+    split_tf32(acc[u][2], h.z, l.z);
+    split_tf32(acc[u][3], h.w, l.w);
+    const int64_t go = (int64_t)i * FB * np_ + (int64_t)k * FB + g;
+    *reinterpret_cast<float4*>(fp.Lh + go) = h;
+    *reinterpret_cast<float4*>(fp.Ll + go) = l;
+  }
+  __syncthreads();  // X, Y free again
+}
+
+__global__ void __launch_bounds__(FNT, 1) factor_kernel(const FactorParams fp) {
+  extern __shared__ __align__(16) float fsm[];
+  float* X = fsm;               // [FB][TP]
+  float* Y = X + FB * TP;       // [FB][TP]
+  float* LT = Y + FB * TP;      // [FB][TP]: L_{k+1,k} transposed (CTA 0)
+  float* A = LT + FB * TP;      // [FB][FP]
+  float* M = A + FB * FP;       // [FB][FP]
+  float* Lt = M + FB * FP;      // [32 * 32 + 32]
+  float* rdiag = Lt + 32 * 32 + 32;  // [32]
+  const int64_t np_ = fp.np_;
+  const int T = fp.T;
+  const int G = gridDim.x;
+  const int cta = blockIdx.x;
+
+  if (cta == 0) {  // the first diagonal block
+    const float* R0 = fp.R;
+    for (int e = threadIdx.x; e < FB * FB; e += FNT) {
+      const int r = e / FB, c = e % FB;
+      A[r * FP + c] = __ldcg(R0 + (int64_t)r * np_ + c);
+      M[r * FP + c] = 0.f;
+    }
+    __syncthreads();
+    leaf64(A, M, Lt, rdiag, fp.hdr);
+    store_diag_m(fp, M, 0);
+  }
+  if (!grid_barrier(fp)) return;
+
+  for (int k = 0; k + 1 < T; ++k) {
+    float acc[4][4];
+    if (cta == 0) {
+      // panel tile (k+1, k), then the next diagonal block
+      panel_tile(fp, k + 1, k, X, Y, acc);
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(&fp.pdone[k], 1);
+      }
+      const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) LT[(c0 + v) * TP + r0 + u] = acc[u][v];
+      __syncthreads();
+      tile_product(LT, LT, acc);  // L L^T
+      const float* Rd = fp.R + (int64_t)(k + 1) * FB * np_ + (int64_t)(k + 1) * FB;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float4 rv = __ldcg(reinterpret_cast<const float4*>(Rd + (int64_t)(r0 + u) * np_ + c0));
+        A[(r0 + u) * FP + c0 + 0] = rv.x - acc[u][0];
+        A[(r0 + u) * FP + c0 + 1] = rv.y - acc[u][1];
+        A[(r0 + u) * FP + c0 + 2] = rv.z - acc[u][2];
+        A[(r0 + u) * FP + c0 + 3] = rv.w - acc[u][3];
+      }
+      for (int e = threadIdx.x; e < FB * FP; e += FNT) M[e] = 0.f;
+      __syncthreads();
+      leaf64(A, M, Lt, rdiag, fp.hdr);
+      store_diag_m(fp, M, k + 1);
+    } else {
+      // tasks of this step, dealt round-robin to CTAs 1..G-1: first the
+      // panel tiles i = k + 2 .. T - 1, then the trailing tiles column by
+      // column (j = k + 1 .. T - 1, i = j .. T - 1, without (k+1, k+1))
+      const int W = G - 1, slot = cta - 1;
+      const int npanel = T - k - 2;
+      const int m = T - k - 1;  // trailing tiles span m x m blocks
+      const int ntrail = m * (m + 1) / 2 - 1;
+      int q = slot;
+      for (; q < npanel; q += W) {
+        const int i = k + 2 + q;
+        panel_tile(fp, i, k, X, Y, acc);
+        if (threadIdx.x == 0) {
+          __threadfence();
+          atomicAdd(&fp.pdone[k], 1);
+        }
+      }
+      // every panel tile of the step (CTA 0 adds the first one)
+      if (q < npanel + ntrail && !wait_panels(fp, k, npanel + 1)) return;
+      int jj = 0, base = 0;  // column walk: tiles before column jj
+      for (; q < npanel + ntrail; q += W) {
+        const int t = q - npanel;
+        while (t >= base + (m - jj - (jj == 0 ? 1 : 0))) {
+          base += m - jj - (jj == 0 ? 1 : 0);
+          ++jj;
+        }
+        const int j = k + 1 + jj;
+        const int i = k + 1 + (jj == 0 ? 1 : jj) + (t - base);
+        const float* Li = fp.R + (int64_t)i * FB * np_ + (int64_t)k * FB;
+        const float* Lj = fp.R + (int64_t)j * FB * np_ + (int64_t)k * FB;
+        load_tile_t(X, Li, np_);
+        if (i != j) load_tile_t(Y, Lj, np_);
+        __syncthreads();
+        tile_product(X, i != j ? Y : X, acc);
+        float* Ct = fp.R + (int64_t)i * FB * np_ + (int64_t)j * FB;
+        const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float4* cp = reinterpret_cast<float4*>(Ct + (int64_t)(r0 + u) * np_ + c0);
+          float4 cv = __ldcg(cp);
+          cv.x -= acc[u][0];
+          cv.y -= acc[u][1];
+          cv.z -= acc[u][2];
+          cv.w -= acc[u][3];
+          *cp = cv;
+        }
+        __syncthreads();
+      }
+    }
+    if (!grid_barrier(fp)) return;
+  }
+}
+
+size_t factor_smem_bytes() { return sizeof(float) * (3 * FB * TP + 2 * FB * FP + 32 * 32 + 32 + 32); }
 
 // Mt[o1 + c][o2 + r] = M[o2 + r][o1 + c] for the merged blocks of one level.
 __global__ void __launch_bounds__(256) transpose_blocks_kernel(const float* __restrict__ Mh,
@@ -413,7 +597,8 @@ size_t prepare_ws_bytes(int64_t in) {
   size_t b = kHeaderBytes;
   b += round_up((int64_t)sizeof(float) * in, 256);               // hd
   b += 9 * round_up((int64_t)sizeof(float) * np_ * np_, 256);    // R; L, M, Mt, X^T (hi, lo)
-  b += 2 * round_up((int64_t)sizeof(float) * np_ * NB, 256);     // split panel
+  b += round_up((int64_t)sizeof(float) * np_ * FB, 256);         // diagonal blocks of M
+  b += round_up((int64_t)sizeof(int) * (np_ / FB + 4), 256);      // barrier and panel flags
   return b;
 }
 
@@ -436,8 +621,9 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   float* Mtl = (float*)p; p += mat;
   float* Xh = (float*)p; p += mat;
   float* Xl = (float*)p; p += mat;
-  float* Pkh = (float*)p; p += round_up((int64_t)sizeof(float) * np_ * NB, 256);
-  float* Pkl = (float*)p;
+  float* MD = (float*)p; p += round_up((int64_t)sizeof(float) * np_ * FB, 256);
+  unsigned* sync = (unsigned*)p;  // [0..2] barrier, then panel flags
+  const int T = (int)(np_ / FB);
   const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
 
   CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
@@ -455,71 +641,40 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
-  static bool leaf_cfg = false;
-  const size_t leaf_smem = 2 * NB * LD * sizeof(float);
-  if (!leaf_cfg) {
-    CUDA_TRY(cudaFuncSetAttribute(leaf_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)leaf_smem));
-    leaf_cfg = true;
-  }
-  const int KB = (int)(np_ / NB);
-  for (int k = 0; k < KB; ++k) {
-    leaf_kernel<<<1, 512, leaf_smem, st>>>(R, Mh, Ml, Mth, Mtl, np_, k, hdr);
+  // blocked Cholesky of R and the inverses of its diagonal blocks
+  {
+    static bool factor_cfg = false;
+    const size_t fsmem = factor_smem_bytes();
+    if (!factor_cfg) {
+      CUDA_TRY(cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem));
+      factor_cfg = true;
+    }
+    CUDA_TRY(cudaMemsetAsync(sync, 0, sizeof(int) * (T + 4), st));
+    FactorParams fp;
+    fp.R = R;
+    fp.np_ = np_;
+    fp.T = T;
+    fp.MD = MD;
+    fp.Lh = Lh;
+    fp.Ll = Ll;
+    fp.Mh = Mh;
+    fp.Ml = Ml;
+    fp.Mth = Mth;
+    fp.Mtl = Mtl;
+    fp.sync = sync;
+    fp.pdone = (int*)(sync + 4);
+    fp.hdr = hdr;
+    int per_sm = 0;
+    CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, factor_kernel, FNT, fsmem));
+    if (per_sm < 1) return fail(GPTQ_ERR_CUDA, "factor_kernel does not fit on an SM");
+    const int grid = std::max(2, std::min(dev.sms, T * T));
+    void* args[] = {&fp};
+    CUDA_TRY(cudaLaunchCooperativeKernel((const void*)factor_kernel, dim3(grid), dim3(FNT), args, fsmem, st));
     note_launch();
-    CUDA_TRY(cudaGetLastError());
-    const int64_t kB = (int64_t)k * NB;
-    const int64_t r0 = kB + NB;
-    const int64_t m = np_ - r0;
-    if (m <= 0) break;
-    split_panel_kernel<<<(unsigned)std::min<int64_t>((m * 32 + 255) / 256, 1024), 256, 0, st>>>(R, np_, r0, kB, m,
-                                                                                                 Pkh, Pkl);
-    note_launch();
-    CUDA_TRY(cudaGetLastError());
-    // panel: L[r0:, k] = R[r0:, k] M_kk^T   -> L's panel (split)
-    GemmArgs pg;
-    pg.op = OP_TF32X3;
-    pg.P = {Pkh, Pkl, m, NB, NB};
-    pg.Q = {Mh, Ml, np_, np_, np_};
-    pg.R = m;
-    pg.Cn = NB;
-    pg.K = NB;
-    pg.p_row0 = 0;
-    pg.p_k0 = 0;
-    pg.q_row0 = kB;
-    pg.q_k0 = kB;
-    pg.C = Lh;
-    pg.C_lo = Ll;
-    pg.ldc = np_;
-    pg.c_row0 = r0;
-    pg.c_col0 = kB;
-    pg.alpha = 1.f;
-    pg.beta = 0.f;
-    pg.status = &hdr->status;
-    CUDA_TRY(run_gemm(pg, st, dev.sms, force_simt));
-    // trailing: R[r0:, r0:] -= L[r0:, k] L[r0:, k]^T   (lower triangle)
-    GemmArgs tg;
-    tg.op = OP_TF32X3;
-    tg.P = {Lh, Ll, np_, np_, np_};
-    tg.Q = tg.P;
-    tg.R = m;
-    tg.Cn = m;
-    tg.K = NB;
-    tg.p_row0 = r0;
-    tg.p_k0 = kB;
-    tg.q_row0 = r0;
-    tg.q_k0 = kB;
-    tg.C = R;
-    tg.ldc = np_;
-    tg.c_row0 = r0;
-    tg.c_col0 = r0;
-    tg.alpha = -1.f;
-    tg.beta = 1.f;
-    tg.mask = 2;
-    tg.status = &hdr->status;
-    CUDA_TRY(run_gemm(tg, st, dev.sms, force_simt));
   }
   // triangular inverse: merge groups pairwise, M21 = -M22 (L21 M11)
   std::vector<std::pair<int64_t, int64_t>> groups;  // (offset, size)
-  for (int k = 0; k < KB; ++k) groups.push_back({(int64_t)k * NB, NB});
+  for (int k = 0; k < T; ++k) groups.push_back({(int64_t)k * FB, FB});
   while (groups.size() > 1) {
     std::vector<std::pair<int64_t, int64_t>> next;
     size_t i = 0;
