@@ -262,35 +262,51 @@ __device__ void leaf64(float* A, float* M, float* Lt, float* rdiag, PrepHeader* 
   gemm32<false>(M + 32 * FP + 32, X, M + 32 * FP, -1.f, false, false);  // M21 = -M22 X
 }
 
-// T[t][r] = G[r][t] for an FB x FB tile of a row-major matrix (row stride ld).
-__device__ __forceinline__ void load_tile_t(float* T, const float* G, int64_t ld) {
+// 16-byte global -> shared copy through L2 only (cp.async.cg): tiles that
+// other CTAs write during the launch must not come from a stale L1 line.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// S[r][t] (pitch TP) <- G[r][t] for an FB x FB tile (row stride ld), async.
+__device__ __forceinline__ void prefetch_tile(float* S, const float* G, int64_t ld) {
   for (int e = threadIdx.x; e < FB * FB / 4; e += FNT) {
-    const int r = e % FB, t4 = (e / FB) * 4;
-    const float4 v = __ldcg(reinterpret_cast<const float4*>(G + (int64_t)r * ld + t4));
-    T[(t4 + 0) * TP + r] = v.x;
-    T[(t4 + 1) * TP + r] = v.y;
-    T[(t4 + 2) * TP + r] = v.z;
-    T[(t4 + 3) * TP + r] = v.w;
+    const int r = e / (FB / 4), t4 = (e % (FB / 4)) * 4;
+    cp_async16(S + r * TP + t4, G + (int64_t)r * ld + t4);
   }
 }
 
-// acc[u][v] = sum_t X[t][r0 + u] Y[t][c0 + v] over an FB-long inner dimension
-// (X, Y transposed tiles); thread t owns rows 4 (t / 16) and columns 4 (t % 16).
+// acc[u][v] = sum_t X[tr + 16u][t] Y[tc + 16v][t]   (tr = tid / 16, tc = tid % 16)
+// X, Y row-major tiles of pitch TP.  Output rows and columns are strided by
+// 16 so that the 16 column groups of a warp read 16 consecutive rows of Y
+// (two conflict-free wavefronts per vector load).
 __device__ __forceinline__ void tile_product(const float* X, const float* Y, float acc[4][4]) {
-  const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
 #pragma unroll
   for (int u = 0; u < 4; ++u)
 #pragma unroll
     for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
-#pragma unroll 4
-  for (int t = 0; t < FB; ++t) {
-    const float4 x = *reinterpret_cast<const float4*>(X + t * TP + r0);
-    const float4 y = *reinterpret_cast<const float4*>(Y + t * TP + c0);
-    const float xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll 2
+  for (int t = 0; t < FB; t += 4) {
+    float4 x[4], y[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = *reinterpret_cast<const float4*>(X + (tr + 16 * u) * TP + t);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) y[v] = *reinterpret_cast<const float4*>(Y + (tc + 16 * v) * TP + t);
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(xs[u], ys[v], acc[u][v]);
+      for (int v = 0; v < 4; ++v) {
+        acc[u][v] = fmaf(x[u].x, y[v].x, acc[u][v]);
+        acc[u][v] = fmaf(x[u].y, y[v].y, acc[u][v]);
+        acc[u][v] = fmaf(x[u].z, y[v].z, acc[u][v]);
+        acc[u][v] = fmaf(x[u].w, y[v].w, acc[u][v]);
+      }
   }
 }
 
@@ -384,53 +400,49 @@ __device__ void store_diag_m(const FactorParams& fp, const float* M, int b) {
   }
 }
 
-// Panel tile (i, k): L_ik = A_ik M_kk^T.  X, Y: transposed operand tiles.
-// Writes R (fp32) and Lh/Ll (split); leaves acc in registers.
-__device__ void panel_tile(const FactorParams& fp, int i, int k, float* X, float* Y, float acc[4][4]) {
-  const int64_t np_ = fp.np_;
-  float* Rt = fp.R + (int64_t)i * FB * np_ + (int64_t)k * FB;
-  load_tile_t(X, Rt, np_);
-  load_tile_t(Y, fp.MD + (int64_t)k * FB * FB, FB);
-  __syncthreads();
-  tile_product(X, Y, acc);
-  const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
+// Store the panel tile L (acc, strided layout) at block (i, k): fp32 to R,
+// split to Lh/Ll.
+__device__ __forceinline__ void store_panel(const FactorParams& fp, int i, int k, const float acc[4][4]) {
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  const int64_t base = (int64_t)i * FB * fp.np_ + (int64_t)k * FB;
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int64_t g = (int64_t)(r0 + u) * np_ + c0;
-    *reinterpret_cast<float4*>(Rt + g) = make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
-    float4 h, l;
-    split_tf32(acc[u][0], h.x, l.x);
-    split_tf32(acc[u][1], h.y, l.y);
-    split_tf32(acc[u][2], h.z, l.z);
-    split_tf32(acc[u][3], h.w, l.w);
-    const int64_t go = (int64_t)i * FB * np_ + (int64_t)k * FB + g;
-    *reinterpret_cast<float4*>(fp.Lh + go) = h;
-    *reinterpret_cast<float4*>(fp.Ll + go) = l;
-  }
-  __syncthreads();  // X, Y free again
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const int64_t g = base + (int64_t)(tr + 16 * u) * fp.np_ + tc + 16 * v;
+      float h, l;
+      split_tf32(acc[u][v], h, l);
+      fp.R[g] = acc[u][v];
+      fp.Lh[g] = h;
+      fp.Ll[g] = l;
+    }
 }
 
 __global__ void __launch_bounds__(FNT, 1) factor_kernel(const FactorParams fp) {
   extern __shared__ __align__(16) float fsm[];
-  float* X = fsm;               // [FB][TP]
-  float* Y = X + FB * TP;       // [FB][TP]
-  float* LT = Y + FB * TP;      // [FB][TP]: L_{k+1,k} transposed (CTA 0)
-  float* A = LT + FB * TP;      // [FB][FP]
-  float* M = A + FB * FP;       // [FB][FP]
-  float* Lt = M + FB * FP;      // [32 * 32 + 32]
+  // double-buffered operand tiles [FB][TP]: X at buffers 0-1, Y at 2-3,
+  // the target C at 4-5
+  auto Xb = [&](int b) { return fsm + (0 + b) * FB * TP; };
+  auto Yb = [&](int b) { return fsm + (2 + b) * FB * TP; };
+  auto Cb = [&](int b) { return fsm + (4 + b) * FB * TP; };
+  float* LT = fsm + 6 * FB * TP;     // [FB][TP]: L_{k+1,k} (CTA 0)
+  float* A = LT + FB * TP;           // [FB][FP]
+  float* M = A + FB * FP;            // [FB][FP]
+  float* Lt = M + FB * FP;           // [32 * 32 + 32]
   float* rdiag = Lt + 32 * 32 + 32;  // [32]
   const int64_t np_ = fp.np_;
   const int T = fp.T;
   const int G = gridDim.x;
   const int cta = blockIdx.x;
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+  auto tile = [&](int i, int j) { return fp.R + (int64_t)i * FB * np_ + (int64_t)j * FB; };
 
   if (cta == 0) {  // the first diagonal block
-    const float* R0 = fp.R;
     for (int e = threadIdx.x; e < FB * FB; e += FNT) {
       const int r = e / FB, c = e % FB;
-      A[r * FP + c] = __ldcg(R0 + (int64_t)r * np_ + c);
-      M[r * FP + c] = 0.f;
+      A[r * FP + c] = __ldcg(fp.R + (int64_t)r * np_ + c);
     }
+    for (int e = threadIdx.x; e < FB * FP; e += FNT) M[e] = 0.f;
     __syncthreads();
     leaf64(A, M, Lt, rdiag, fp.hdr);
     store_diag_m(fp, M, 0);
@@ -440,28 +452,36 @@ __global__ void __launch_bounds__(FNT, 1) factor_kernel(const FactorParams fp) {
   for (int k = 0; k + 1 < T; ++k) {
     float acc[4][4];
     if (cta == 0) {
-      // panel tile (k+1, k), then the next diagonal block
-      panel_tile(fp, k + 1, k, X, Y, acc);
+      // panel tile (k+1, k) = A M_kk^T with M_kk still in shared memory,
+      // then A_{k+1,k+1} -= L L^T and the leaf on it
+      prefetch_tile(Xb(0), tile(k + 1, k), np_);
+      prefetch_tile(Cb(0), tile(k + 1, k + 1), np_);
+      cp_async_commit();
+      for (int e = threadIdx.x; e < FB * FB; e += FNT) {
+        const int r = e / FB, c = e % FB;
+        Yb(0)[r * TP + c] = M[r * FP + c];
+      }
+      cp_async_wait<0>();
+      __syncthreads();
+      tile_product(Xb(0), Yb(0), acc);
+      store_panel(fp, k + 1, k, acc);
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) LT[(tr + 16 * u) * TP + tc + 16 * v] = acc[u][v];
+      __syncthreads();
       if (threadIdx.x == 0) {
         __threadfence();
         atomicAdd(&fp.pdone[k], 1);
       }
-      const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
+      tile_product(LT, LT, acc);  // L L^T
 #pragma unroll
       for (int u = 0; u < 4; ++u)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) LT[(c0 + v) * TP + r0 + u] = acc[u][v];
-      __syncthreads();
-      tile_product(LT, LT, acc);  // L L^T
-      const float* Rd = fp.R + (int64_t)(k + 1) * FB * np_ + (int64_t)(k + 1) * FB;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float4 rv = __ldcg(reinterpret_cast<const float4*>(Rd + (int64_t)(r0 + u) * np_ + c0));
-        A[(r0 + u) * FP + c0 + 0] = rv.x - acc[u][0];
-        A[(r0 + u) * FP + c0 + 1] = rv.y - acc[u][1];
-        A[(r0 + u) * FP + c0 + 2] = rv.z - acc[u][2];
-        A[(r0 + u) * FP + c0 + 3] = rv.w - acc[u][3];
-      }
+        for (int v = 0; v < 4; ++v) {
+          const int r = tr + 16 * u, c = tc + 16 * v;
+          A[r * FP + c] = Cb(0)[r * TP + c] - acc[u][v];
+        }
       for (int e = threadIdx.x; e < FB * FP; e += FNT) M[e] = 0.f;
       __syncthreads();
       leaf64(A, M, Lt, rdiag, fp.hdr);
@@ -473,53 +493,78 @@ __global__ void __launch_bounds__(FNT, 1) factor_kernel(const FactorParams fp) {
       const int W = G - 1, slot = cta - 1;
       const int npanel = T - k - 2;
       const int m = T - k - 1;  // trailing tiles span m x m blocks
-      const int ntrail = m * (m + 1) / 2 - 1;
+      const int total = npanel + m * (m + 1) / 2 - 1;
       int q = slot;
       for (; q < npanel; q += W) {
         const int i = k + 2 + q;
-        panel_tile(fp, i, k, X, Y, acc);
+        prefetch_tile(Xb(0), tile(i, k), np_);
+        prefetch_tile(Yb(0), fp.MD + (int64_t)k * FB * FB, FB);
+        cp_async_commit();
+        cp_async_wait<0>();
+        __syncthreads();
+        tile_product(Xb(0), Yb(0), acc);
+        store_panel(fp, i, k, acc);
+        __syncthreads();
         if (threadIdx.x == 0) {
           __threadfence();
           atomicAdd(&fp.pdone[k], 1);
         }
       }
       // every panel tile of the step (CTA 0 adds the first one)
-      if (q < npanel + ntrail && !wait_panels(fp, k, npanel + 1)) return;
+      if (q < total && !wait_panels(fp, k, npanel + 1)) return;
       int jj = 0, base = 0;  // column walk: tiles before column jj
-      for (; q < npanel + ntrail; q += W) {
-        const int t = q - npanel;
+      auto locate = [&](int qq, int& i, int& j) {
+        const int t = qq - npanel;
         while (t >= base + (m - jj - (jj == 0 ? 1 : 0))) {
           base += m - jj - (jj == 0 ? 1 : 0);
           ++jj;
         }
-        const int j = k + 1 + jj;
-        const int i = k + 1 + (jj == 0 ? 1 : jj) + (t - base);
-        const float* Li = fp.R + (int64_t)i * FB * np_ + (int64_t)k * FB;
-        const float* Lj = fp.R + (int64_t)j * FB * np_ + (int64_t)k * FB;
-        load_tile_t(X, Li, np_);
-        if (i != j) load_tile_t(Y, Lj, np_);
-        __syncthreads();
-        tile_product(X, i != j ? Y : X, acc);
-        float* Ct = fp.R + (int64_t)i * FB * np_ + (int64_t)j * FB;
-        const int r0 = (threadIdx.x / 16) * 4, c0 = (threadIdx.x % 16) * 4;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float4* cp = reinterpret_cast<float4*>(Ct + (int64_t)(r0 + u) * np_ + c0);
-          float4 cv = __ldcg(cp);
-          cv.x -= acc[u][0];
-          cv.y -= acc[u][1];
-          cv.z -= acc[u][2];
-          cv.w -= acc[u][3];
-          *cp = cv;
-        }
-        __syncthreads();
+        j = k + 1 + jj;
+        i = k + 1 + (jj == 0 ? 1 : jj) + (t - base);
+      };
+      auto prefetch = [&](int b, int i, int j) {
+        prefetch_tile(Xb(b), tile(i, k), np_);
+        if (i != j) prefetch_tile(Yb(b), tile(j, k), np_);
+        prefetch_tile(Cb(b), tile(i, j), np_);
+      };
+      int ic = 0, jc = 0;
+      if (q < total) {
+        locate(q, ic, jc);
+        prefetch(0, ic, jc);
+        cp_async_commit();
       }
+      int b = 0;
+      for (; q < total; q += W) {
+        int in_ = 0, jn = 0;
+        const bool more = q + W < total;
+        if (more) {
+          locate(q + W, in_, jn);
+          prefetch(b ^ 1, in_, jn);
+        }
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        tile_product(Xb(b), ic != jc ? Yb(b) : Xb(b), acc);
+        float* Ct = tile(ic, jc);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int r = tr + 16 * u, c = tc + 16 * v;
+            Ct[(int64_t)r * np_ + c] = Cb(b)[r * TP + c] - acc[u][v];
+          }
+        __syncthreads();
+        b ^= 1;
+        ic = in_;
+        jc = jn;
+      }
+      cp_async_wait<0>();
     }
     if (!grid_barrier(fp)) return;
   }
 }
 
-size_t factor_smem_bytes() { return sizeof(float) * (3 * FB * TP + 2 * FB * FP + 32 * 32 + 32 + 32); }
+size_t factor_smem_bytes() { return sizeof(float) * (7 * FB * TP + 2 * FB * FP + 32 * 32 + 32 + 32); }
 
 // Mt[o1 + c][o2 + r] = M[o2 + r][o1 + c] for the merged blocks of one level.
 __global__ void __launch_bounds__(256) transpose_blocks_kernel(const float* __restrict__ Mh,
