@@ -139,8 +139,8 @@ size_t gptq_workspace_bytes(int64_t out, int64_t in, const gptq_config_t* cfg);
  *   tokens   >= 0; 0 is a no-op.
  *   n_accum  host pointer or NULL; *n_accum += tokens on success.
  * fp16/bf16 X with a 16-byte aligned base and (ldx * 2) % 16 == 0 runs on the
- * tensor cores (exact products, fp32 accumulation, drained into S every 8192
- * tokens so the accumulation error stays near 2e-5 relative for any token
+ * tensor cores (exact products, fp32 accumulation, drained into S every 32768
+ * tokens so the accumulation error stays below 5e-5 relative for any token
  * count); fp32 X and other layouts run on CUDA cores in fp32.  Asynchronous.
  * Accumulation order is fixed for a given (in, tokens, device), so repeated
  * calls give identical S.
