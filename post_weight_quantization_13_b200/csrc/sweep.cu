@@ -33,6 +33,7 @@ constexpr int ROWS = 16;         // rows per sweep CTA (4 lanes per row)
 constexpr int NT = ROWS * 4;     // threads per sweep CTA
 constexpr int UPITCH = 36;       // floats per (j, lane) slice of U in smem
 constexpr int EPITCH = BW + 1;
+constexpr int CPITCH = BW + 4;   // bytes per row of staged codes (no bank conflicts)
 // interleaved diagonal block of U (BW x 4 x UPITCH floats) followed by 1/U_jj
 constexpr uint32_t kDiagBlockFloats = BW * 4 * UPITCH + BW;
 constexpr uint32_t kDiagBlockBytes = kDiagBlockFloats * 4;
@@ -82,6 +83,18 @@ __device__ __forceinline__ void group_params(float lo, float hi, float amax, int
   }
 }
 
+// rint(x / s) with x / s an IEEE division, from the product with the
+// rounded reciprocal: the product is within 3 units in the last place of the
+// quotient, so its rounding gives the same integer unless the quotient lies
+// within a few units of a half-integer; there (and for non-finite products)
+// the exact quotient is rounded instead.
+__device__ __forceinline__ float round_div(float x, float s, float inv_s) {
+  const float y = x * inv_s;
+  const float fr = y - floorf(y);
+  if (fabsf(fr - 0.5f) > fmaf(fabsf(y), 0x1p-20f, 0x1p-24f)) return rintf(y);
+  return rintf(__fdiv_rn(x, s));
+}
+
 // One sweep block of BW = 128 processed columns.  Each row is handled by 4
 // lanes; lane q of a row holds the block's columns 4m + q (m = 0..31) in
 // registers w[].  The 128 columns are processed in 8 passes of 16; after a
@@ -95,7 +108,7 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
   float* rd = Us + BW * 4 * UPITCH;                // [128] 1 / U_jj
   float* Esh = rd + BW;                            // [ROWS][EPITCH]
   float* Esl = Esh + ROWS * EPITCH;                // [ROWS][EPITCH]
-  uint8_t* Cs = reinterpret_cast<uint8_t*>(Esl + ROWS * EPITCH);  // [ROWS][BW]
+  uint8_t* Cs = reinterpret_cast<uint8_t*>(Esl + ROWS * EPITCH);  // [ROWS][CPITCH]
   const int tid = threadIdx.x;
   __shared__ uint64_t ubar;
   // U's diagonal block, already laid out for this kernel by pack_diag_kernel:
@@ -125,7 +138,7 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
     for (int i = 0; i < 32; ++i) w[i] = live ? src[4 * i + q] : 0.f;
   }
   const float fmaxq = (float)sp.maxq;
-  float s = 1.f, z = 0.f, lsum = 0.f;
+  float s = 1.f, z = 0.f, inv_s = 1.f, lsum = 0.f;
   if (!mbar_wait(&ubar, 0)) raise_status(sp.status, ST_TIMEOUT);
   // a group that started in an earlier block keeps that block's scale/zero
   if (GSB == BW && !sp.gstart0 && live) {
@@ -133,6 +146,7 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
     s = sp.scales[row * sp.ngroups + g];
     z = (float)sp.zeros[row * sp.ngroups + g];
   }
+  inv_s = __frcp_rn(s);
   __syncthreads();
   for (int mo = 0; mo < 32; mo += 4) {  // pass: columns 4*mo .. 4*mo + 15
     if (4 * mo >= sp.ncols) break;
@@ -172,6 +186,7 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
           am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
         }
         group_params(lo, hi, am, sp.sym, fmaxq, s, z);
+        inv_s = __frcp_rn(s);
         if (q == 0 && live) {
           const int64_t g = sp.gs == -1 ? 0 : (sp.kB + cbase) / sp.gs;
           sp.scales[row * sp.ngroups + g] = s;
@@ -185,12 +200,12 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
         float e = 0.f;
         if (q == t) {
           const float x = w[mi];
-          float qf = rintf(__fdiv_rn(x, s)) + z;
+          float qf = round_div(x, s, inv_s) + z;
           qf = fminf(fmaxf(qf, 0.f), fmaxq);
           const float deq = s * (qf - z);
           e = (x - deq) * rd[j];
           lsum = fmaf(e, e, lsum);
-          Cs[rl * BW + j] = (uint8_t)qf;
+          Cs[rl * CPITCH + j] = (uint8_t)qf;
           float eh, el;
           split_tf32(e, eh, el);
           Esh[rl * EPITCH + j] = eh;
@@ -226,7 +241,7 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
     if (gr >= sp.out) continue;
     sp.Eh[gr * sp.lde + sp.e_col0 + c] = Esh[r * EPITCH + c];
     sp.El[gr * sp.lde + sp.e_col0 + c] = Esl[r * EPITCH + c];
-    if (c < sp.ncols) sp.codes_p[gr * sp.ldw + sp.kB + c] = Cs[r * BW + c];
+    if (c < sp.ncols) sp.codes_p[gr * sp.ldw + sp.kB + c] = Cs[r * CPITCH + c];
   }
 }
 
@@ -348,7 +363,7 @@ cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
 
 template <int GSB>
 cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st) {
-  const size_t smem = (size_t)(BW * 4 * UPITCH + BW + 2 * ROWS * EPITCH) * sizeof(float) + ROWS * BW;
+  const size_t smem = (size_t)(BW * 4 * UPITCH + BW + 2 * ROWS * EPITCH) * sizeof(float) + ROWS * CPITCH;
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(sweep_kernel<GSB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
