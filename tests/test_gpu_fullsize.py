@@ -169,3 +169,79 @@ def test_fullsize_act_order(lib, full, qi):
     if np.array_equal(perm, prep["perm"]):
         rate, _ = code_report(g["codes"][rows], codes)
         assert rate >= 0.999, rate
+
+
+def _solve_layer_case(lib, wl, layer, q, tokens, rows=None):
+    """GPU solve (the bench's call sequence) and the float64 oracle from the
+    same seeded inputs; the oracle sweeps ``rows`` (all when None)."""
+    import torch
+    W = gen.weight(wl, layer)
+    X = gen.x_full(wl, layer.site, tokens=tokens)
+    Xd = torch.from_numpy(X).cuda()
+    S = torch.zeros((layer.in_, layer.in_), dtype=torch.float32, device="cuda")
+    n = lib.gptq_hessian_accumulate(S, Xd, 0)
+    del Xd
+    full = dict(W=W, X=X, S=S, n=n, layer=layer)
+    g = _gpu_solve(lib, full, q)
+    S64 = np.zeros((layer.in_, layer.in_), dtype=np.float64)
+    for c0 in range(0, X.shape[1], 8192):
+        O.hessian_accumulate(S64, X[:, c0:c0 + 8192])
+    full["S64"] = S64
+    if rows is None:
+        rows = np.arange(layer.out)
+    prep, res, codes = _oracle_rows(full, q, rows)
+    return full, g, prep, res, codes, rows
+
+
+def test_correlated_channels_all_rows(lib):
+    """q_proj shape with strongly correlated channels (X = s (z + P y), rank
+    16): the case where error compensation changes most codes relative to
+    rounding.  Every row is compared."""
+    wl = gen.WORKLOADS["q_proj_correlated"]
+    layer, q = wl.layers[0], wl.quant[0]
+    full, g, prep, res, codes, rows = _solve_layer_case(lib, wl, layer, q, wl.tokens)
+    if np.array_equal(g["perm"], prep["perm"]):
+        rate, eq = code_report(g["codes"], codes)
+        assert rate >= 0.999, rate
+        compare_groups(g["scales"], g["zeros"], res["scales"], res["zeros"],
+                       eq[:, prep["perm"]], q.group_size)
+    H0 = prep["H0"]
+    e_gpu = _row_error(full["W"], g["codes"], g["scales"], g["zeros"], g["g_idx"], H0)
+    e_ref = _row_error(full["W"], codes, res["scales"], res["zeros"],
+                       O.g_index(prep["perm"], q.group_size), H0)
+    assert abs(e_gpu - e_ref) <= 0.01 * e_ref, (e_gpu, e_ref)
+    # compensation matters here: GPTQ beats round-to-nearest clearly
+    r_codes, r_scales, r_zeros = O.rtn(np.asarray(full["W"], np.float64), q.bits, q.group_size,
+                                       q.sym, prep["perm"])
+    e_rtn = _row_error(full["W"], r_codes, r_scales, r_zeros, O.g_index(prep["perm"], q.group_size), H0)
+    assert e_gpu < 0.9 * e_rtn, (e_gpu, e_rtn)
+
+
+def test_mlp_down_proj_11008_wide(lib):
+    """Llama-7B down_proj shape: 11008 input channels (SiLU-gated
+    activations), 3-bit symmetric, group 128, act-order.  The layer shape is
+    the benchmark's; the calibration set is cut to 32768 tokens so that the
+    float64 oracle's Hessian (11008^2 x tokens) stays within a test's time."""
+    wl = gen.WORKLOADS["llama7b_mlp"]
+    layer, q = wl.layer("down_proj"), wl.quant[0]
+    rows = np.random.default_rng(17).choice(layer.out, ROWS, replace=False)
+    full, g, prep, res, codes, rows = _solve_layer_case(lib, wl, layer, q, 32768, rows)
+    n_in = layer.in_
+    perm = g["perm"]
+    assert np.array_equal(np.sort(perm), np.arange(n_in))
+    d = np.diag(full["S64"])[perm]
+    assert np.all(d[1:] <= d[:-1] * (1 + 1e-4) + 1e-12)
+    if np.array_equal(perm, prep["perm"]):
+        U_gpu = g["U"].T
+        rel = np.linalg.norm(U_gpu - prep["U"]) / np.linalg.norm(prep["U"])
+        assert rel < 1e-3, rel
+        rate, _ = code_report(g["codes"][rows], codes)
+        assert rate >= 0.999, rate
+    maxq = 2 ** q.bits - 1
+    assert g["codes"].min() >= 0 and g["codes"].max() <= maxq
+    H0 = prep["H0"]
+    e_gpu = _row_error(full["W"][rows], g["codes"][rows], g["scales"][rows], g["zeros"][rows],
+                       g["g_idx"], H0)
+    e_ref = _row_error(full["W"][rows], codes, res["scales"], res["zeros"],
+                       O.g_index(prep["perm"], q.group_size), H0)
+    assert abs(e_gpu - e_ref) <= 0.01 * e_ref, (e_gpu, e_ref)
