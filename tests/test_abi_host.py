@@ -88,7 +88,7 @@ def test_workspace_bytes(g):
     c = _cfg(g)
     prep = g.gptq_workspace_bytes(0, 4096, c)
     full = g.gptq_workspace_bytes(4096, 4096, c)
-    assert prep > 8 * 4096 * 4096 * 4
+    assert prep >= 2 * 4096 * 4096 * 4   # R (then L) and M = L^-1, fp32
     assert full >= prep
     assert g.gptq_workspace_bytes(4096, 0, c) == 0
     assert g.gptq_workspace_bytes(11008, 4096, c) >= full
