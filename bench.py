@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--no-dequant", action="store_true")
     return ap.parse_args()
 
 
@@ -424,6 +425,32 @@ def run_ours(args):
                "ms_per_step": e_ms / args.e2e_steps, "steps": args.e2e_steps,
                "pipeline": f"{nch} host batches of {chunk} tokens, copy overlapped with the SYRK"}
 
+    # dequantisation of the solved layer back to fp16 (HBM-bound), each launch
+    # timed alone after an L2 flush (a read of 256 MiB, so that no dirty lines
+    # are left for the timed kernel to write back)
+    deq = None
+    if not args.no_dequant:
+        Wq = torch.empty((out, in_), dtype=torch.float16, device=dev)
+        flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        times = []
+        for it in range(8):
+            flush.sum()
+            d0, d1 = ev(), ev()
+            d0.record(stream)
+            g.gptq_dequantize_layer(qweight, scales, zeros, g_idx, q.bits, Wq, stream)
+            d1.record(stream)
+            torch.cuda.synchronize(dev)
+            if it >= 3:
+                times.append(d0.elapsed_time(d1))
+        dq_ms = statistics.median(times)
+        dq_bytes = (out * in_ * q.bits // 8 + out * ng * 8 + in_ * 4 + out * in_ * 2)
+        bw_peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+        deq = {"kernel": "dequant_kernel<f16>", "ms": dq_ms, "bytes": dq_bytes,
+               "GB/s": dq_bytes / (dq_ms / 1e3) / 1e9, "peak": bw_peak,
+               "frac": dq_bytes / (dq_ms / 1e3) / 1e9 / bw_peak, "bound": "hbm",
+               "note": "each launch timed alone (launch latency included) after reading 256 MiB to clear L2"}
+        del flush
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         setup = oracle_setup(wl, layer, q, Wh.numpy(), Xh.numpy())
@@ -450,6 +477,7 @@ def run_ours(args):
                          "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16)",
                          "flops_per_launch": flops},
             "step_roofline": step_roof,
+            "dequant": deq,
             "gpu_launches": launches,
             "clocks": clocks,
             "e2e": e2e,

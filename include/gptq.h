@@ -210,6 +210,27 @@ gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out,
                                   int32_t* zeros, int32_t* g_idx, float* loss,
                                   void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * Dequantize: Wq[r][c] = scales[r][g] * (code[r][c] - zeros[r][g]) with
+ * g = g_idx[c], the inverse of the group quantizer ("gptq" agent-skill page,
+ * Group-wise quantization; "gptq" glossary page: weights stored as low-bit
+ * codes with a scale and zero point per group).  The product is formed in
+ * fp32 and rounded once to wt.
+ * Inputs (device, as written by gptq_quantize_layer): qweight uint32
+ *   [out][in*bits/32] (LSB-first fields, original column order); scales fp32
+ *   and zeros int32 [out][ngroups]; g_idx int32[in], 16-byte aligned.
+ * Output (device, caller-owned): Wq, out x in, element type wt, row stride
+ *   ldw >= in.
+ * Needs in % 8 == 0 and (in * bits) % 32 == 0 (GPTQ_ERR_UNSUPPORTED
+ * otherwise).  Asynchronous.  out == 0 is a no-op.
+ */
+gptq_status_t gptq_dequantize_layer(const uint32_t* qweight,
+                                    const float* scales, const int32_t* zeros,
+                                    const int32_t* g_idx, int64_t out,
+                                    int64_t in, int bits, int ngroups,
+                                    void* Wq, gptq_dtype_t wt, int64_t ldw,
+                                    void* stream);
+
 /* Size of the fixed device scratch used by gptq_quantize_layer_noalloc:
  * 16 MiB, enough for layers up to 1024 x 1024 at block_size 128. */
 #define GPTQ_STATIC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -24,6 +24,7 @@ __all__ = [
     "gptq_abi_version", "gptq_last_error", "gptq_kernel_launches", "gptq_validate_config",
     "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "GPTQ_STATIC_SCRATCH_BYTES",
+    "gptq_dequantize_layer",
     "solve_layer", "STATUS_NAMES",
 ]
 
@@ -73,6 +74,10 @@ lib.gptq_quantize_layer.restype = ctypes.c_int
 lib.gptq_quantize_layer_noalloc.argtypes = [_p, ctypes.c_int, _i64, _i64, _i64, _p, _p, _p,
                                             ctypes.POINTER(_Config), _p, _p, _p, _p, _p, _p, _p]
 lib.gptq_quantize_layer_noalloc.restype = ctypes.c_int
+
+lib.gptq_dequantize_layer.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p,
+                                      ctypes.c_int, _i64, _p]
+lib.gptq_dequantize_layer.restype = ctypes.c_int
 
 # bytes of the library's static scratch (GPTQ_STATIC_SCRATCH_BYTES in gptq.h)
 GPTQ_STATIC_SCRATCH_BYTES = 16 << 20
@@ -197,6 +202,16 @@ def gptq_quantize_layer_noalloc(W, U, perm, dead, cfg, scales, zeros, g_idx, cod
                                            _ptr(U), _ptr(perm), _ptr(dead), ctypes.byref(c),
                                            _ptr(codes), _ptr(qweight), _ptr(scales), _ptr(zeros),
                                            _ptr(g_idx), _ptr(loss), _stream(stream)))
+
+
+def gptq_dequantize_layer(qweight, scales, zeros, g_idx, bits, Wq, stream=None) -> None:
+    """Wq (out x in; f16, bf16 or f32) <- scales * (code - zeros) from the
+    packed codes gptq_quantize_layer wrote."""
+    _rowmajor(Wq, "Wq")
+    out, in_ = Wq.shape
+    _check(lib.gptq_dequantize_layer(_ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(g_idx), out, in_,
+                                     int(bits), scales.shape[1], _ptr(Wq), _dt(Wq), Wq.stride(0),
+                                     _stream(stream)))
 
 
 def solve_layer(W, X=None, cfg=None, S=None, n=None, with_codes=True, stream=None):

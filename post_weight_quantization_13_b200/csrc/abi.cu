@@ -210,4 +210,28 @@ gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, i
                         ws_bytes, (cudaStream_t)stream);
 }
 
+gptq_status_t gptq_dequantize_layer(const uint32_t* qweight, const float* scales, const int32_t* zeros,
+                                    const int32_t* g_idx, int64_t out, int64_t in, int bits, int ngroups,
+                                    void* Wq, gptq_dtype_t wt, int64_t ldw, void* stream) {
+  clear_error();
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
+    return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8 (got %d)", bits);
+  if (out < 0 || in < 1 || in > kMaxIn || out > kMaxOut)
+    return fail(GPTQ_ERR_INVALID_ARG, "layer %lld x %lld is outside this build's limits", (long long)out,
+                (long long)in);
+  if (in % 8 != 0 || (in * bits) % 32 != 0)
+    return fail(GPTQ_ERR_UNSUPPORTED, "dequantize needs in %% 8 == 0 and in*bits %% 32 == 0 (in=%lld, bits=%d)",
+                (long long)in, bits);
+  if (ngroups < 1 || ngroups > in) return fail(GPTQ_ERR_INVALID_ARG, "ngroups must be in [1, in] (got %d)", ngroups);
+  if (!dtype_ok(wt)) return fail(GPTQ_ERR_INVALID_ARG, "unknown output dtype %d", (int)wt);
+  if (ldw < in) return fail(GPTQ_ERR_INVALID_ARG, "ldw (%lld) < in (%lld)", (long long)ldw, (long long)in);
+  if (out == 0) return GPTQ_OK;
+  if (!qweight || !scales || !zeros || !g_idx || !Wq)
+    return fail(GPTQ_ERR_INVALID_ARG, "qweight, scales, zeros, g_idx and Wq must be non-NULL");
+  if (((uintptr_t)g_idx & 15u) != 0) return fail(GPTQ_ERR_INVALID_ARG, "g_idx must be 16-byte aligned");
+  gptq_status_t s = check_device();
+  if (s != GPTQ_OK) return s;
+  return dequantize_layer(qweight, scales, zeros, g_idx, out, in, bits, ngroups, Wq, wt, ldw, (cudaStream_t)stream);
+}
+
 }  // extern "C"

@@ -46,6 +46,9 @@ size_t quantize_ws_bytes(int64_t out, int64_t in, const gptq_config_t* cfg);
 
 gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_config_t* cfg, float* U,
                            int32_t* perm, uint8_t* dead, void* ws, size_t ws_bytes, cudaStream_t st);
+gptq_status_t dequantize_layer(const uint32_t* qweight, const float* scales, const int32_t* zeros,
+                               const int32_t* g_idx, int64_t out, int64_t in, int bits, int ngroups, void* Wq,
+                               gptq_dtype_t wt, int64_t ldw, cudaStream_t st);
 gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_t in, int64_t ldw, const float* U,
                              const int32_t* perm, const uint8_t* dead, const gptq_config_t* cfg, int32_t* codes,
                              uint32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, float* loss, void* ws,
