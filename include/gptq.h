@@ -231,6 +231,17 @@ gptq_status_t gptq_dequantize_layer(const uint32_t* qweight,
                                     void* Wq, gptq_dtype_t wt, int64_t ldw,
                                     void* stream);
 
+/*
+ * Diagnostic with no counterpart in the method: every wait inside this
+ * library's kernels (pipeline barriers, copy completion, grid barriers) is
+ * bounded and, when it gives up, raises GPTQ_ERR_TIMEOUT through a status
+ * word instead of hanging or trapping.  This call runs that path on purpose:
+ * one thread waits on a barrier that nothing ever completes, gives up after
+ * limit_ns nanoseconds (1 .. 2e9), and the call returns GPTQ_ERR_TIMEOUT.
+ * The device stays usable afterwards.  Synchronises the stream.
+ */
+gptq_status_t gptq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
+
 /* Size of the fixed device scratch used by gptq_quantize_layer_noalloc:
  * 16 MiB, enough for layers up to 1024 x 1024 at block_size 128. */
 #define GPTQ_STATIC_SCRATCH_BYTES ((size_t)16 << 20)

@@ -24,7 +24,7 @@ __all__ = [
     "gptq_abi_version", "gptq_last_error", "gptq_kernel_launches", "gptq_validate_config",
     "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "GPTQ_STATIC_SCRATCH_BYTES",
-    "gptq_dequantize_layer",
+    "gptq_dequantize_layer", "gptq_selftest_wait_timeout",
     "solve_layer", "STATUS_NAMES",
 ]
 
@@ -78,6 +78,9 @@ lib.gptq_quantize_layer_noalloc.restype = ctypes.c_int
 lib.gptq_dequantize_layer.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p,
                                       ctypes.c_int, _i64, _p]
 lib.gptq_dequantize_layer.restype = ctypes.c_int
+
+lib.gptq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _p]
+lib.gptq_selftest_wait_timeout.restype = ctypes.c_int
 
 # bytes of the library's static scratch (GPTQ_STATIC_SCRATCH_BYTES in gptq.h)
 GPTQ_STATIC_SCRATCH_BYTES = 16 << 20
@@ -212,6 +215,12 @@ def gptq_dequantize_layer(qweight, scales, zeros, g_idx, bits, Wq, stream=None) 
     _check(lib.gptq_dequantize_layer(_ptr(qweight), _ptr(scales), _ptr(zeros), _ptr(g_idx), out, in_,
                                      int(bits), scales.shape[1], _ptr(Wq), _dt(Wq), Wq.stride(0),
                                      _stream(stream)))
+
+
+def gptq_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
+    """Run the bounded-wait timeout path once; returns the status code
+    (GPTQ_ERR_TIMEOUT = 6 when the path works)."""
+    return lib.gptq_selftest_wait_timeout(int(limit_ns), _stream(stream))
 
 
 def solve_layer(W, X=None, cfg=None, S=None, n=None, with_codes=True, stream=None):
