@@ -488,10 +488,99 @@ def run_ours(args):
         pg.destroy_process_group()
 
 
+def run_block(args):
+    """A whole decoder block (4 activation sites, 7 layers) through
+    solve_block: one Hessian and one prepare per site, the layers of a site
+    quantized concurrently.  Prints one JSON line; rank 0 of N replicas."""
+    import torch
+
+    import gen
+    import post_weight_quantization_13_b200 as g
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        pg = dist
+    wl = gen.WORKLOADS[args.workload]
+    n_tok = args.tokens or wl.tokens
+    q = wl.quant[0]
+    acts = {}
+    for site in wl.sites:
+        Xh = torch.empty((site.in_, n_tok), dtype=torch.float16, pin_memory=True)
+        gen.x_full(wl, site, tokens=n_tok, out=Xh.numpy())
+        acts[site.name] = Xh.to(dev)
+        del Xh
+    layers = [(l.name, torch.from_numpy(gen.weight(wl, l)).to(dev), l.site) for l in wl.layers]
+    weights = sum(W.shape[0] * W.shape[1] for _, W, _ in layers)
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    for _ in range(args.warmup):
+        g.solve_block(layers, acts, q.as_dict())
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(gpu_id_for(local), enabled=not args.no_clocks)
+    if pg:
+        pg.barrier()
+    launches0 = g.gptq_kernel_launches()
+    e0, e1 = ev(), ev()
+    e0.record()
+    for _ in range(args.steps):
+        g.solve_block(layers, acts, q.as_dict())
+    e1.record()
+    torch.cuda.synchronize(dev)
+    launches = g.gptq_kernel_launches() - launches0
+    clocks = sampler.stop()
+    elapsed = max_over_ranks(e0.elapsed_time(e1), pg, dev)
+    ms_step = elapsed / args.steps
+
+    # the same block on one stream, and as seven independent layer solves
+    # (each with its own Hessian and prepare), one timed pass each
+    def timed(fn):
+        torch.cuda.synchronize(dev)
+        a, b = ev(), ev()
+        a.record()
+        fn()
+        b.record()
+        torch.cuda.synchronize(dev)
+        return max_over_ranks(a.elapsed_time(b), pg, dev)
+
+    one_stream_ms = timed(lambda: g.solve_block(layers, acts, q.as_dict(), streams=False))
+    naive_ms = timed(lambda: [g.solve_layer(W, acts[site], q.as_dict(), with_codes=False)
+                              for _, W, site in layers])
+    peaks, peak_src = load_peaks()
+    pf = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]) * 1e12
+    syrk_floor = sum(s.in_ * (s.in_ + 1) * n_tok for s in wl.sites) / pf * 1e3
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": job_throughput(world, weights, args.steps, elapsed),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": wl.name, "layers": [(l.name, l.out, l.in_, l.site) for l in wl.layers],
+                       "tokens": n_tok, "bits": q.bits, "group_size": q.group_size,
+                       "desc_act": q.desc_act, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2"},
+            "block_roofline": {"syrk_floor_ms": syrk_floor, "frac": syrk_floor / ms_step,
+                               "peak_source": f"{peak_src} bf16 sustained"},
+            "compare_ms": {"one_stream": one_stream_ms, "seven_independent_solves": naive_ms},
+            "gpu_launches": launches, "clocks": clocks, "e2e": None, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload == "llama7b_block":
+        run_block(args)
     else:
         run_ours(args)
 

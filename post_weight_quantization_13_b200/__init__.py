@@ -25,7 +25,7 @@ __all__ = [
     "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "GPTQ_STATIC_SCRATCH_BYTES",
     "gptq_dequantize_layer", "gptq_selftest_wait_timeout",
-    "solve_layer", "STATUS_NAMES",
+    "solve_layer", "solve_block", "STATUS_NAMES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
@@ -252,3 +252,68 @@ def solve_layer(W, X=None, cfg=None, S=None, n=None, with_codes=True, stream=Non
                         qweight=qweight, loss=loss, stream=stream)
     return dict(S=S, n=n, U=U, perm=perm, dead=dead, scales=scales, zeros=zeros, g_idx=g_idx,
                 loss=loss, codes=codes, qweight=qweight)
+
+
+def solve_block(layers, activations, cfg=None, streams=True):
+    """Quantize the linear layers of one decoder block.
+
+    layers: list of (name, W, site) with W an (out x in) device tensor and
+      site the name of the activation stream feeding it (layers that read the
+      same activations, e.g. q/k/v or gate/up, share one site).
+    activations: dict site -> X (in x tokens device tensor) or an iterable of
+      such token batches.
+
+    For each site the Hessian is accumulated and prepared (U, perm, dead)
+    once; every layer of the site is then quantized against that shared U.
+    With ``streams``, each site's Hessian and prepare run on a stream of
+    their own and the layers of a site are quantized concurrently on
+    separate streams, so that latency-bound sweeps of different layers fill
+    the GPU together.  Returns {name: dict(...)} as solve_layer does, plus
+    {"site:" + site: dict(S, n, U, perm, dead)}; synchronises the device.
+    """
+    import torch
+    cfg = GptqConfig.of(cfg or GptqConfig())
+    sites = {}
+    for name, W, site in layers:
+        sites.setdefault(site, []).append((name, W))
+    dev = layers[0][1].device
+    cur = torch.cuda.current_stream(dev)
+    results = {}
+    pending = []
+    for site, members in sites.items():
+        s_site = torch.cuda.Stream(dev) if streams else cur
+        s_site.wait_stream(cur)
+        in_ = members[0][1].shape[1]
+        with torch.cuda.stream(s_site):
+            S = torch.zeros((in_, in_), dtype=torch.float32, device=dev)
+            n = 0
+            X = activations[site]
+            for Xb in ([X] if torch.is_tensor(X) else X):
+                n = gptq_hessian_accumulate(S, Xb, n, s_site)
+            ws = torch.empty(gptq_workspace_bytes(0, in_, cfg), dtype=torch.uint8, device=dev)
+            U = torch.empty((in_, in_), dtype=torch.float32, device=dev)
+            perm = torch.empty(in_, dtype=torch.int32, device=dev)
+            dead = torch.empty(in_, dtype=torch.uint8, device=dev)
+        gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, s_site)
+        results["site:" + site] = dict(S=S, n=n, U=U, perm=perm, dead=dead)
+        for name, W in members:
+            s_layer = torch.cuda.Stream(dev) if streams else s_site
+            s_layer.wait_stream(s_site)
+            out = W.shape[0]
+            ng = 1 if cfg.group_size == -1 else in_ // cfg.group_size
+            with torch.cuda.stream(s_layer):
+                wsq = torch.empty(gptq_workspace_bytes(out, in_, cfg), dtype=torch.uint8, device=dev)
+                r = dict(scales=torch.empty((out, ng), dtype=torch.float32, device=dev),
+                         zeros=torch.empty((out, ng), dtype=torch.int32, device=dev),
+                         g_idx=torch.empty(in_, dtype=torch.int32, device=dev),
+                         loss=torch.empty(out, dtype=torch.float32, device=dev),
+                         codes=torch.empty((out, in_), dtype=torch.int32, device=dev),
+                         qweight=(torch.empty((out, in_ * cfg.bits // 32), dtype=torch.int32, device=dev)
+                                  if (in_ * cfg.bits) % 32 == 0 else None))
+            gptq_quantize_layer(W, U, perm, dead, cfg, r["scales"], r["zeros"], r["g_idx"], wsq,
+                                codes=r["codes"], qweight=r["qweight"], loss=r["loss"], stream=s_layer)
+            r.update(perm=perm, dead=dead, U=U, n=n)
+            results[name] = r
+            pending.append((s_layer, wsq))
+    torch.cuda.synchronize(dev)
+    return results
