@@ -36,6 +36,10 @@ namespace gptq {
 namespace {
 
 constexpr int NB = 128;
+// Larger matrices are factored in super-blocks of this size: one cooperative
+// launch per diagonal super-block, the panel below it and the trailing
+// update of the rest as tensor-core GEMMs (their work grows as np^3).
+constexpr int64_t kSuperBlock = 4096;
 
 // ------------------------------------------------------------------ diag
 // One CTA: hd[i] = fixed diagonal of H (dead -> 1), dead flags, and
@@ -124,6 +128,26 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
       }
       *reinterpret_cast<float4*>(R + a * np_ + b0) = make_float4(v[0], v[1], v[2], v[3]);
     }
+  }
+}
+
+// Ph/Pl[r][c] = split(R[r0 + r][c0 + c]) for c < width: a panel of R as a
+// 3xTF32 operand (rows x width, row stride width).
+__global__ void __launch_bounds__(256) split_panel_kernel(const float* __restrict__ R, int64_t np_, int64_t r0,
+                                                          int64_t c0, int64_t rows, int64_t width,
+                                                          float* __restrict__ Ph, float* __restrict__ Pl) {
+  const int64_t q = width / 4;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * q;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / q, c4 = (e % q) * 4;
+    const float4 v = *reinterpret_cast<const float4*>(R + (r0 + r) * np_ + c0 + c4);
+    float4 h, l;
+    split_tf32(v.x, h.x, l.x);
+    split_tf32(v.y, h.y, l.y);
+    split_tf32(v.z, h.z, l.z);
+    split_tf32(v.w, h.w, l.w);
+    *reinterpret_cast<float4*>(Ph + r * width + c4) = h;
+    *reinterpret_cast<float4*>(Pl + r * width + c4) = l;
   }
 }
 
@@ -644,6 +668,8 @@ size_t prepare_ws_bytes(int64_t in) {
   b += 9 * round_up((int64_t)sizeof(float) * np_ * np_, 256);    // R; L, M, Mt, X^T (hi, lo)
   b += round_up((int64_t)sizeof(float) * np_ * FB, 256);         // diagonal blocks of M
   b += round_up((int64_t)sizeof(int) * (np_ / FB + 4), 256);      // barrier and panel flags
+  if (np_ > kSuperBlock)                                          // split panel below a super-block
+    b += 2 * round_up((int64_t)sizeof(float) * (np_ - kSuperBlock) * kSuperBlock, 256);
   return b;
 }
 
@@ -668,7 +694,14 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   float* Xl = (float*)p; p += mat;
   float* MD = (float*)p; p += round_up((int64_t)sizeof(float) * np_ * FB, 256);
   unsigned* sync = (unsigned*)p;  // [0..2] barrier, then panel flags
-  const int T = (int)(np_ / FB);
+  p += round_up((int64_t)sizeof(int) * (np_ / FB + 4), 256);
+  float* Pkh = nullptr;
+  float* Pkl = nullptr;
+  if (np_ > kSuperBlock) {
+    Pkh = (float*)p;
+    p += round_up((int64_t)sizeof(float) * (np_ - kSuperBlock) * kSuperBlock, 256);
+    Pkl = (float*)p;
+  }
   const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
 
   CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
@@ -686,40 +719,18 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
-  // blocked Cholesky of R and the inverses of its diagonal blocks
-  {
-    static bool factor_cfg = false;
-    const size_t fsmem = factor_smem_bytes();
-    if (!factor_cfg) {
-      CUDA_TRY(cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem));
-      factor_cfg = true;
-    }
-    CUDA_TRY(cudaMemsetAsync(sync, 0, sizeof(int) * (T + 4), st));
-    FactorParams fp;
-    fp.R = R;
-    fp.np_ = np_;
-    fp.T = T;
-    fp.MD = MD;
-    fp.Lh = Lh;
-    fp.Ll = Ll;
-    fp.Mh = Mh;
-    fp.Ml = Ml;
-    fp.Mth = Mth;
-    fp.Mtl = Mtl;
-    fp.sync = sync;
-    fp.pdone = (int*)(sync + 4);
-    fp.hdr = hdr;
-    int per_sm = 0;
-    CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, factor_kernel, FNT, fsmem));
-    if (per_sm < 1) return fail(GPTQ_ERR_CUDA, "factor_kernel does not fit on an SM");
-    const int grid = std::max(2, std::min(dev.sms, T * T));
-    void* args[] = {&fp};
-    CUDA_TRY(cudaLaunchCooperativeKernel((const void*)factor_kernel, dim3(grid), dim3(FNT), args, fsmem, st));
-    note_launch();
+  // blocked Cholesky of R, one cooperative launch per diagonal super-block
+  static bool factor_cfg = false;
+  const size_t fsmem = factor_smem_bytes();
+  if (!factor_cfg) {
+    CUDA_TRY(cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem));
+    factor_cfg = true;
   }
+  int per_sm = 0;
+  CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, factor_kernel, FNT, fsmem));
+  if (per_sm < 1) return fail(GPTQ_ERR_CUDA, "factor_kernel does not fit on an SM");
   // triangular inverse: merge groups pairwise, M21 = -M22 (L21 M11)
-  std::vector<std::pair<int64_t, int64_t>> groups;  // (offset, size)
-  for (int k = 0; k < T; ++k) groups.push_back({(int64_t)k * FB, FB});
+  auto merge = [&](std::vector<std::pair<int64_t, int64_t>> groups) -> gptq_status_t {  // (offset, size)
   while (groups.size() > 1) {
     std::vector<std::pair<int64_t, int64_t>> next;
     size_t i = 0;
@@ -790,6 +801,89 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     }
     if (i < groups.size()) next.push_back(groups[i]);
     groups.swap(next);
+  }
+  return GPTQ_OK;
+  };
+  std::vector<std::pair<int64_t, int64_t>> supers;
+  for (int64_t o = 0; o < np_; o += kSuperBlock) {
+    const int64_t B = std::min<int64_t>(kSuperBlock, np_ - o);
+    const int T = (int)(B / FB);
+    supers.push_back({o, B});
+    CUDA_TRY(cudaMemsetAsync(sync, 0, sizeof(int) * (T + 4), st));
+    const int64_t off = o * np_ + o;
+    FactorParams fp;
+    fp.R = R + off;
+    fp.np_ = np_;
+    fp.T = T;
+    fp.MD = MD;
+    fp.Lh = Lh + off;
+    fp.Ll = Ll + off;
+    fp.Mh = Mh + off;
+    fp.Ml = Ml + off;
+    fp.Mth = Mth + off;
+    fp.Mtl = Mtl + off;
+    fp.sync = sync;
+    fp.pdone = (int*)(sync + 4);
+    fp.hdr = hdr;
+    const int grid = std::max(2, std::min(dev.sms, T * T));
+    void* args[] = {&fp};
+    CUDA_TRY(cudaLaunchCooperativeKernel((const void*)factor_kernel, dim3(grid), dim3(FNT), args, fsmem, st));
+    note_launch();
+    // the inverse of this super-block's L (merging its 64-blocks)
+    std::vector<std::pair<int64_t, int64_t>> groups;
+    for (int k = 0; k < T; ++k) groups.push_back({o + (int64_t)k * FB, FB});
+    gptq_status_t ms = merge(groups);
+    if (ms != GPTQ_OK) return ms;
+    const int64_t r0 = o + B, m = np_ - r0;
+    if (m <= 0) break;
+    // panel below the super-block, L21 = R21 M_sb^T (split), then the
+    // trailing update R22 -= L21 L21^T (lower tiles), both on tensor cores
+    split_panel_kernel<<<(unsigned)std::min<int64_t>((m * (B / 4) + 255) / 256, (int64_t)dev.sms * 8), 256, 0,
+                         st>>>(R, np_, r0, o, m, B, Pkh, Pkl);
+    note_launch();
+    CUDA_TRY(cudaGetLastError());
+    GemmArgs pg;
+    pg.op = OP_TF32X3;
+    pg.P = {Pkh, Pkl, m, B, B};
+    pg.Q = {Mh, Ml, np_, np_, np_};
+    pg.R = m;
+    pg.Cn = B;
+    pg.K = B;
+    pg.q_row0 = o;
+    pg.q_k0 = o;
+    pg.C = Lh;
+    pg.C_lo = Ll;
+    pg.ldc = np_;
+    pg.c_row0 = r0;
+    pg.c_col0 = o;
+    pg.alpha = 1.f;
+    pg.beta = 0.f;
+    pg.status = &hdr->status;
+    CUDA_TRY(run_gemm(pg, st, dev.sms, force_simt));
+    GemmArgs tg;
+    tg.op = OP_TF32X3;
+    tg.P = {Lh, Ll, np_, np_, np_};
+    tg.Q = tg.P;
+    tg.R = m;
+    tg.Cn = m;
+    tg.K = B;
+    tg.p_row0 = r0;
+    tg.p_k0 = o;
+    tg.q_row0 = r0;
+    tg.q_k0 = o;
+    tg.C = R;
+    tg.ldc = np_;
+    tg.c_row0 = r0;
+    tg.c_col0 = r0;
+    tg.alpha = -1.f;
+    tg.beta = 1.f;
+    tg.mask = 2;
+    tg.status = &hdr->status;
+    CUDA_TRY(run_gemm(tg, st, dev.sms, force_simt));
+  }
+  if (supers.size() > 1) {
+    gptq_status_t ms = merge(supers);
+    if (ms != GPTQ_OK) return ms;
   }
   {
     const unsigned grid = (unsigned)std::min<int64_t>(in, (int64_t)dev.sms * 8);

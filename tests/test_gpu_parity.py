@@ -123,6 +123,9 @@ def _run_prepare(lib, S32, n, cfg):
     (8, 64, "scaled_normal", True, 0.01), (72, 500, "scaled_normal", False, 0.01),
     (136, 1000, "scaled_normal", True, 0.1), (256, 2048, "correlated", True, 0.01),
     (520, 4096, "scaled_normal", True, 0.01), (1000, 3000, "correlated", False, 0.01),
+    # wider than one 4096 super-block: two and three cooperative launches
+    # joined by tensor-core panel and trailing updates
+    (4500, 6000, "scaled_normal", True, 0.01), (9000, 12000, "scaled_normal", False, 0.01),
 ])
 def test_prepare_hinv(lib, in_, tokens, kind, desc_act, damp):
     S32, n = _prep_inputs(in_ + tokens, in_, tokens, kind, dead=(3, 5) if in_ > 8 else ())
@@ -134,7 +137,10 @@ def test_prepare_hinv(lib, in_, tokens, kind, desc_act, damp):
     assert np.all(np.tril(U, -1) == 0)
     assert np.all(np.diag(U) > 0)
     err = rel_fro(U, ref["U"])
-    assert err < 1e-4, err
+    # fp32 rounding in the factorisation grows with the dimension and the
+    # condition of the damped Hessian; above 1024 channels the bound is the
+    # full-size tests' 1e-3
+    assert err < (1e-4 if in_ <= 1024 else 1e-3), err
 
 
 def test_prepare_reports_not_pd_and_nonfinite(lib):
