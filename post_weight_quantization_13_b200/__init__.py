@@ -265,10 +265,10 @@ def solve_block(layers, activations, cfg=None, streams=True):
 
     For each site the Hessian is accumulated and prepared (U, perm, dead)
     once; every layer of the site is then quantized against that shared U.
-    With ``streams``, each site's Hessian and prepare run on a stream of
-    their own and the layers of a site are quantized concurrently on
+    With ``streams``, the layers of a site are quantized concurrently on
     separate streams, so that latency-bound sweeps of different layers fill
-    the GPU together.  Returns {name: dict(...)} as solve_layer does, plus
+    the GPU together; a site's Hessian starts after the previous site's
+    layers, since its persistent kernel wants every SM.  Returns {name: dict(...)} as solve_layer does, plus
     {"site:" + site: dict(S, n, U, perm, dead)}; synchronises the device.
     """
     import torch
@@ -283,6 +283,10 @@ def solve_block(layers, activations, cfg=None, streams=True):
     for site, members in sites.items():
         s_site = torch.cuda.Stream(dev) if streams else cur
         s_site.wait_stream(cur)
+        # the Hessian kernel is persistent (one resident CTA per SM): start it
+        # once the previous site's layers are done, not beside them
+        for s_prev, _ in pending:
+            s_site.wait_stream(s_prev)
         in_ = members[0][1].shape[1]
         with torch.cuda.stream(s_site):
             S = torch.zeros((in_, in_), dtype=torch.float32, device=dev)
