@@ -6,6 +6,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <atomic>
+#include <map>
 #include <mutex>
 #include <string>
 
@@ -36,6 +37,20 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 }
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+cudaError_t ensure_smem_limit(const void* func, int bytes) {
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;  // (kernel, device) -> bytes
+  int d = 0;
+  cudaError_t e = cudaGetDevice(&d);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  int& cur = done[{func, d}];
+  if (cur >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) cur = bytes;
+  return e;
+}
 
 const DeviceInfo& device_info() {
   static DeviceInfo infos[64];

@@ -50,6 +50,10 @@ struct GemmArgs {
 
 void note_launch();
 
+// Raise the dynamic shared-memory limit of kernel `func` to `bytes` on the
+// current device, once per (kernel, device, size); thread-safe.
+cudaError_t ensure_smem_limit(const void* func, int bytes);
+
 // Returns cudaSuccess or the launch error.  Asynchronous.
 cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t stream, int num_sms);
 cudaError_t simt_gemm(const GemmArgs& a, cudaStream_t stream);

@@ -720,12 +720,8 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     CUDA_TRY(cudaGetLastError());
   }
   // blocked Cholesky of R, one cooperative launch per diagonal super-block
-  static bool factor_cfg = false;
   const size_t fsmem = factor_smem_bytes();
-  if (!factor_cfg) {
-    CUDA_TRY(cudaFuncSetAttribute(factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fsmem));
-    factor_cfg = true;
-  }
+  CUDA_TRY(ensure_smem_limit((const void*)factor_kernel, (int)fsmem));
   int per_sm = 0;
   CUDA_TRY(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, factor_kernel, FNT, fsmem));
   if (per_sm < 1) return fail(GPTQ_ERR_CUDA, "factor_kernel does not fit on an SM");

@@ -364,12 +364,8 @@ cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
 template <int GSB>
 cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st) {
   const size_t smem = (size_t)(BW * 4 * UPITCH + BW + 2 * ROWS * EPITCH) * sizeof(float) + ROWS * CPITCH;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(sweep_kernel<GSB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  cudaError_t ce = ensure_smem_limit((const void*)sweep_kernel<GSB>, (int)smem);
+  if (ce != cudaSuccess) return ce;
   const unsigned grid = (unsigned)((sp.out + ROWS - 1) / ROWS);
   sweep_kernel<GSB><<<grid, NT, smem, st>>>(sp);
   note_launch();

@@ -660,12 +660,8 @@ bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 template <int OP>
 cudaError_t launch(const TmaMaps& maps, const KParams& kp, int grid, size_t smem, cudaStream_t st) {
-  static int configured = 0;  // the attribute is per function, set it once per process
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(tc_gemm_kernel<OP>, cudaFuncAttributeMaxDynamicSharedMemorySize, 232448);
-    if (e != cudaSuccess) return e;
-    configured = 1;
-  }
+  cudaError_t ce = ensure_smem_limit((const void*)tc_gemm_kernel<OP>, 232448);
+  if (ce != cudaSuccess) return ce;
   tc_gemm_kernel<OP><<<grid, kThreads, smem, st>>>(maps, kp);
   note_launch();
   return cudaGetLastError();
