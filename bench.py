@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
     ap.add_argument("--no-dequant", action="store_true")
+    ap.add_argument("--block-size", type=int, default=0,
+                    help="lazy-batch width of the sweep (default: the workload's)")
     return ap.parse_args()
 
 
@@ -256,6 +258,9 @@ def run_ours(args):
         wl = dataclasses.replace(wl, tokens=args.tokens)
     layer = wl.layers[0]
     q = wl.quant[0]
+    if args.block_size:
+        import dataclasses
+        q = dataclasses.replace(q, block_size=args.block_size)
     cfg = g.GptqConfig(**q.as_dict())
     out, in_ = layer.out, layer.in_
     n_tok = wl.tokens
