@@ -336,23 +336,31 @@ __global__ void invperm_kernel(const int32_t* __restrict__ perm, int64_t in, int
 __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ codes_p, int64_t ldc_p, int64_t out,
                                                    int64_t in, int bits, const int32_t* __restrict__ inv,
                                                    uint32_t* __restrict__ qweight, int32_t* __restrict__ codes) {
-  const int64_t r = blockIdx.y;
+  // one row at a time per block: the row's codes (processing order) are
+  // staged in shared memory with 16-byte loads, then gathered into original
+  // column order through inv (read-only, shared by all rows)
+  extern __shared__ __align__(16) uint8_t srow[];
   const int64_t nwords = (in * bits + 31) / 32;
-  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nwords; w += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t bit0 = w * 32;
-    int64_t c = bit0 / bits;
-    uint64_t acc = 0;
-    for (; c < in && c * bits < bit0 + 32; ++c) {
-      const uint32_t v = codes_p[r * ldc_p + inv[c]];
-      const int64_t off = c * bits - bit0;  // may be negative for the field straddling in
-      if (off >= 0) {
-        acc |= (uint64_t)v << off;
-        if (codes) codes[r * in + c] = (int32_t)v;
-      } else {
-        acc |= (uint64_t)v >> (-off);
+  for (int64_t r = blockIdx.x; r < out; r += gridDim.x) {
+    __syncthreads();
+    for (int64_t e = (int64_t)threadIdx.x * 16; e < ldc_p; e += (int64_t)blockDim.x * 16)
+      *reinterpret_cast<uint4*>(srow + e) = *reinterpret_cast<const uint4*>(codes_p + r * ldc_p + e);
+    __syncthreads();
+    if (qweight) {
+      for (int64_t w = threadIdx.x; w < nwords; w += blockDim.x) {
+        const int64_t bit0 = w * 32;
+        int64_t c = bit0 / bits;
+        uint64_t acc = 0;
+        for (; c < in && c * bits < bit0 + 32; ++c) {
+          const uint32_t v = srow[__ldg(inv + c)];
+          const int64_t off = c * bits - bit0;  // negative for the field straddling in
+          acc |= off >= 0 ? (uint64_t)v << off : (uint64_t)v >> (-off);
+        }
+        qweight[r * nwords + w] = (uint32_t)acc;
       }
     }
-    if (qweight) qweight[r * nwords + w] = (uint32_t)acc;
+    if (codes)
+      for (int64_t c = threadIdx.x; c < in; c += blockDim.x) codes[r * in + c] = (int32_t)srow[__ldg(inv + c)];
   }
 }
 
@@ -563,9 +571,8 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
   note_launch();
   CUDA_TRY(cudaGetLastError());
   if (qweight || codes) {
-    const int64_t nwords = (in * cfg->bits + 31) / 32;
-    dim3 grid((unsigned)std::min<int64_t>((nwords + 255) / 256, 32), (unsigned)out);
-    pack_kernel<<<grid, 256, 0, st>>>(codes_p, np_, out, in, cfg->bits, inv, qweight, codes);
+    const unsigned grid = (unsigned)std::min<int64_t>(out, (int64_t)dev.sms * 8);
+    pack_kernel<<<grid, 256, (size_t)np_, st>>>(codes_p, np_, out, in, cfg->bits, inv, qweight, codes);
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
