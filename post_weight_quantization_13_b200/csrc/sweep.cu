@@ -347,16 +347,28 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ c
       *reinterpret_cast<uint4*>(srow + e) = *reinterpret_cast<const uint4*>(codes_p + r * ldc_p + e);
     __syncthreads();
     if (qweight) {
-      for (int64_t w = threadIdx.x; w < nwords; w += blockDim.x) {
-        const int64_t bit0 = w * 32;
-        int64_t c = bit0 / bits;
-        uint64_t acc = 0;
-        for (; c < in && c * bits < bit0 + 32; ++c) {
-          const uint32_t v = srow[__ldg(inv + c)];
-          const int64_t off = c * bits - bit0;  // negative for the field straddling in
-          acc |= off >= 0 ? (uint64_t)v << off : (uint64_t)v >> (-off);
+      const int nw = (int)nwords, n_in = (int)in;
+      uint32_t* qrow = qweight + r * nwords;
+      if (32 % bits == 0) {
+        // 2, 4 and 8 bits: each word holds 32 / bits whole fields
+        const int per = 32 / bits;
+        for (int w = threadIdx.x; w < nw; w += blockDim.x) {
+          uint32_t acc = 0;
+          for (int u = 0; u < per; ++u) acc |= (uint32_t)srow[__ldg(inv + w * per + u)] << (u * bits);
+          qrow[w] = acc;
         }
-        qweight[r * nwords + w] = (uint32_t)acc;
+      } else {
+        // 3 bits: fields may straddle words
+        for (int w = threadIdx.x; w < nw; w += blockDim.x) {
+          const int bit0 = w * 32;
+          uint64_t acc = 0;
+          for (int c = bit0 / bits; c < n_in && c * bits < bit0 + 32; ++c) {
+            const uint32_t v = srow[__ldg(inv + c)];
+            const int off = c * bits - bit0;  // negative for the field straddling in
+            acc |= off >= 0 ? (uint64_t)v << off : (uint64_t)v >> (-off);
+          }
+          qrow[w] = (uint32_t)acc;
+        }
       }
     }
     if (codes)
