@@ -106,18 +106,20 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
                                                      const uint8_t* __restrict__ dead, PrepHeader* hdr,
                                                      float* __restrict__ R) {
   const float lam = hdr->lambda;
-  for (int64_t a = blockIdx.x; a < np_; a += gridDim.x) {
-    const int64_t i = a < in ? perm[in - 1 - a] : -1;
-    for (int64_t b0 = (int64_t)threadIdx.x * 4; b0 <= a; b0 += (int64_t)blockDim.x * 4) {
+  // in <= 32768, so in * in fits 32-bit index arithmetic
+  const int n = (int)in, np = (int)np_;
+  for (int a = blockIdx.x; a < np; a += gridDim.x) {
+    const int i = a < n ? __ldg(perm + n - 1 - a) : -1;
+    for (int b0 = threadIdx.x * 4; b0 <= a; b0 += blockDim.x * 4) {
       float v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int64_t b = b0 + u;
+        const int b = b0 + u;
         float x = 0.f;
-        if (a < in && b < in) {
-          const int64_t j = perm[in - 1 - b];
-          const int64_t lo = min(i, j), hi = max(i, j);
-          const float sv = S[lo * in + hi];
+        if (a < n && b < n) {
+          const int j = __ldg(perm + n - 1 - b);
+          const unsigned lo = (unsigned)min(i, j), hi = (unsigned)max(i, j);
+          const float sv = __ldg(S + (lo * (unsigned)n + hi));
           if (!isfinite(sv)) raise_status(&hdr->status, ST_NONFINITE);
           x = sv * scale;
           if (i == j) x = (dead[i] ? 1.f : x) + lam;
@@ -126,7 +128,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
         }
         v[u] = x;
       }
-      *reinterpret_cast<float4*>(R + a * np_ + b0) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(R + (int64_t)a * np_ + b0) = make_float4(v[0], v[1], v[2], v[3]);
     }
   }
 }

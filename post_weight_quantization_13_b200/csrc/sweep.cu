@@ -277,18 +277,21 @@ template <typename T>
 __global__ void __launch_bounds__(256) gather_w_kernel(const T* __restrict__ W, int64_t ldw_in, int64_t out,
                                                        int64_t in, int64_t np_, const int32_t* __restrict__ perm,
                                                        const uint8_t* __restrict__ dead, float* __restrict__ Wp) {
+  const int n = (int)in, np = (int)np_;
   for (int64_t r = blockIdx.x; r < out; r += gridDim.x) {
-    for (int64_t p = (int64_t)threadIdx.x * 4; p < np_; p += (int64_t)blockDim.x * 4) {
+    const T* Wr = W + r * ldw_in;
+    float* dst = Wp + r * np_;
+    for (int p = threadIdx.x * 4; p < np; p += blockDim.x * 4) {
       float v[4];
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         v[t] = 0.f;
-        if (p + t < in) {
-          const int32_t c = perm[p + t];
-          if (!dead[c]) v[t] = to_f32(W[r * ldw_in + c]);
+        if (p + t < n) {
+          const int c = __ldg(perm + p + t);
+          if (!__ldg(dead + c)) v[t] = to_f32(Wr[c]);
         }
       }
-      *reinterpret_cast<float4*>(Wp + r * np_ + p) = make_float4(v[0], v[1], v[2], v[3]);
+      *reinterpret_cast<float4*>(dst + p) = make_float4(v[0], v[1], v[2], v[3]);
     }
   }
 }
