@@ -13,6 +13,11 @@
  *   gptq_quantize_layer      the blocked column sweep with error
  *                            compensation, group quantization and packing
  *
+ * and, around them: gptq_dequantize_layer (codes back to weights),
+ * gptq_quantize_layer_noalloc (quantize on a fixed library scratch),
+ * gptq_workspace_bytes / gptq_validate_config (host-side sizing and checks)
+ * and gptq_selftest_wait_timeout (the bounded-wait failure path).
+ *
  * What is computed follows the GPTQ pages: "gptq" glossary page (Method and
  * Algorithm: layer-wise, Hessian from calibration data, quantize each weight
  * in order and compensate the error with H^-1; Group quantization), "Using
@@ -28,7 +33,8 @@
  *     allocates device memory itself: scratch space is the caller's
  *     workspace, sized by gptq_workspace_bytes().
  *   - stream is a cudaStream_t passed as void* (NULL = the legacy default
- *     stream).  Work is enqueued on it; only gptq_prepare_hinv waits for it.
+ *     stream).  Work is enqueued on it; only gptq_prepare_hinv and
+ *     gptq_selftest_wait_timeout wait for it.
  *   - Matrices are row-major unless stated otherwise; leading dimensions are
  *     in elements.
  *   - Every call returns a gptq_status_t.  Nothing aborts or traps.  On an
