@@ -479,6 +479,8 @@ def run_ours(args):
             "roofline": {"kernel": "tc_gemm_kernel<f16> (Hessian S += X X^T, tcgen05)",
                          "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
+                         "frac_of_burst_peak": achieved / peaks.get("bf16_tflops",
+                                                                    PEAKS_FALLBACK["bf16_tflops"]),
                          "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16)",
                          "flops_per_launch": flops},
             "step_roofline": step_roof,
