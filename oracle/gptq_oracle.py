@@ -43,6 +43,9 @@ named at the function that makes it:
   broken by ascending column index.
 * codes are packed LSB-first into little-endian uint32 words, row by row, in
   original column order.
+* the loaders' checkpoint layout (``checkpoint_layout``) is the transpose:
+  codes packed along the input dimension, zeros along the output dimension
+  less an offset of 1, scales in float16.
 
 Every function here is pinned by ``tests/test_oracle_*.py`` against closed
 forms, brute force on tiny layers, invariances and hand-worked examples.
@@ -57,7 +60,7 @@ __all__ = [
     "group_params", "quantize_codes", "dequantize_codes", "sweep_unblocked",
     "sweep_blocked", "prepare", "gptq_layer", "rtn", "pack_rows", "unpack_rows",
     "g_index", "dequantize_layer", "layer_error", "brute_force_sweep",
-    "maxq_of",
+    "maxq_of", "checkpoint_layout",
 ]
 
 
@@ -316,6 +319,54 @@ def unpack_rows(words: np.ndarray, bits: int, n: int) -> np.ndarray:
         codes[:, c] = (v & mask).astype(np.int64)
     return codes
 
+
+
+# ------------------------------------------------------- checkpoint layout
+def _stream_words(fields: np.ndarray, bits: int) -> np.ndarray:
+    """Words of the LSB-first stream of ``bits``-wide fields taken along the
+    last axis: field i fills stream bits [i bits, (i + 1) bits) from its least
+    significant bit up, and stream bit t is bit t % 32 of word t // 32.  Built
+    bit by bit, independently of ``pack_rows``."""
+    f = np.asarray(fields, np.uint64)
+    n = f.shape[-1]
+    if (n * bits) % 32:
+        raise ValueError("the packed axis times bits must be a multiple of 32")
+    one = np.uint64(1)
+    stream = (f[..., None] >> np.arange(bits, dtype=np.uint64)) & one
+    stream = stream.reshape(*f.shape[:-1], n * bits // 32, 32)
+    return (stream << np.arange(32, dtype=np.uint64)).sum(axis=-1).astype(np.uint32)
+
+
+def checkpoint_layout(codes, scales, zeros, g_idx, bits: int, zero_offset: int = 1):
+    """The quantized layer in the checkpoint layout of the GPTQ loaders.
+
+    Reading (the "AutoGPTQ" artifact page, "Why AutoGPTQ Matters", names the
+    GPTQ format that ExLlamaV2 and vLLM load, and the "gptq" agent-skill page,
+    "Marlin", loads it from disk; neither prints the layout): tensors are
+    stored input-dimension-major, the transpose of this solver's row-major
+    outputs --
+
+    * qweight uint32 [in bits/32][out]: column o is the LSB-first stream of
+      row o's codes along the input dimension, in original column order;
+    * qzeros uint32 [ngroups][out bits/32]: row g is the LSB-first stream,
+      along the output dimension, of (zeros[:, g] - zero_offset) mod 2^bits
+      (zero_offset 1 is the convention of the format's first version, whose
+      readers add the 1 back; a zero of 0 then wraps to maxq);
+    * scales float16 [ngroups][out]: scales^T rounded to nearest, ties to
+      even;
+    * g_idx int32 [in], unchanged.
+    """
+    codes = np.asarray(codes, np.int64)
+    zeros = np.asarray(zeros, np.int64)
+    if zero_offset not in (0, 1):
+        raise ValueError("zero_offset must be 0 or 1")
+    if np.any(codes < 0) or np.any(codes >= (1 << bits)):
+        raise ValueError("code out of range")
+    qweight = _stream_words(codes, bits).T.copy()
+    qzeros = _stream_words(np.mod(zeros.T - zero_offset, 1 << bits), bits)
+    return dict(qweight=qweight, qzeros=qzeros,
+                scales=np.asarray(scales, np.float32).T.astype(np.float16),
+                g_idx=np.asarray(g_idx).astype(np.int32))
 
 def g_index(perm: np.ndarray, group_size: int) -> np.ndarray:
     """g_idx[c] = group of original column c = (its processing position) //
