@@ -61,7 +61,20 @@ def parse():
     ap.add_argument("--no-dequant", action="store_true")
     ap.add_argument("--block-size", type=int, default=0,
                     help="lazy-batch width of the sweep (default: the workload's)")
+    ap.add_argument("--desc-act", action="store_true",
+                    help="process columns in act-order (default: the workload's, off)")
     return ap.parse_args()
+
+
+def quant_of(wl, args):
+    """The workload's quantization settings with the command-line overrides."""
+    import dataclasses
+    q = wl.quant[0]
+    if getattr(args, "block_size", 0):
+        q = dataclasses.replace(q, block_size=args.block_size)
+    if getattr(args, "desc_act", False):
+        q = dataclasses.replace(q, desc_act=True)
+    return q
 
 
 def load_peaks():
@@ -191,7 +204,7 @@ def run_reference(args):
         return
     wl = gen.WORKLOADS[args.workload]
     layer = wl.layers[0]
-    q = wl.quant[0]
+    q = quant_of(wl, args)
     W = gen.weight(wl, layer)
     X = gen.x_full(wl, layer.site, tokens=2048)
     setup = oracle_setup(wl, layer, q, W, X)
@@ -257,10 +270,7 @@ def run_ours(args):
         import dataclasses
         wl = dataclasses.replace(wl, tokens=args.tokens)
     layer = wl.layers[0]
-    q = wl.quant[0]
-    if args.block_size:
-        import dataclasses
-        q = dataclasses.replace(q, block_size=args.block_size)
+    q = quant_of(wl, args)
     cfg = g.GptqConfig(**q.as_dict())
     out, in_ = layer.out, layer.in_
     n_tok = wl.tokens
@@ -517,7 +527,7 @@ def run_block(args):
         pg = dist
     wl = gen.WORKLOADS[args.workload]
     n_tok = args.tokens or wl.tokens
-    q = wl.quant[0]
+    q = quant_of(wl, args)
     acts = {}
     for site in wl.sites:
         Xh = torch.empty((site.in_, n_tok), dtype=torch.float16, pin_memory=True)

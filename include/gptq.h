@@ -14,6 +14,7 @@
  *                            compensation, group quantization and packing
  *
  * and, around them: gptq_dequantize_layer (codes back to weights),
+ * gptq_export_checkpoint (the outputs in the loaders' checkpoint layout),
  * gptq_quantize_layer_noalloc (quantize on a fixed library scratch),
  * gptq_workspace_bytes / gptq_validate_config (host-side sizing and checks)
  * and gptq_selftest_wait_timeout (the bounded-wait failure path).
@@ -236,6 +237,42 @@ gptq_status_t gptq_dequantize_layer(const uint32_t* qweight,
                                     int64_t in, int bits, int ngroups,
                                     void* Wq, gptq_dtype_t wt, int64_t ldw,
                                     void* stream);
+
+/*
+ * Export: the solver's outputs rewritten in the checkpoint layout of the
+ * GPTQ loaders ("AutoGPTQ" artifact page, Why AutoGPTQ Matters: the GPTQ
+ * format that ExLlamaV2 and vLLM load; "gptq" agent-skill page, Marlin:
+ * quantized models saved and loaded in it).  The pages print no bit layout;
+ * the one written here stores every tensor input-dimension-major:
+ *   qweight_t uint32 [in*bits/32][out]: column o is row o's codes in
+ *             original column order as an LSB-first stream of bits-wide
+ *             fields (fields may straddle words) -- the transpose of the
+ *             qweight gptq_quantize_layer writes.  Needs (in*bits) % 32 == 0.
+ *   qzeros    uint32 [ngroups][out*bits/32]: row g is the LSB-first stream,
+ *             along the output dimension, of (zeros[o][g] - zero_offset)
+ *             mod 2^bits.  Needs (out*bits) % 32 == 0.  zero_offset 1 is
+ *             the convention of the format's first version (readers add 1
+ *             back; a zero of 0 wraps to 2^bits - 1, which such a reader
+ *             cannot tell from 2^bits - 1); 0 stores the zeros as they are.
+ *   scales_h  float16 bits (uint16) [ngroups][out]: scales^T rounded to
+ *             nearest, ties to even (values above 65504 become infinity).
+ * g_idx needs no rewrite: the loaders read the int32[in] that
+ * gptq_quantize_layer writes.
+ * Inputs (device, as written by gptq_quantize_layer): qweight uint32
+ *   [out][in*bits/32], scales fp32 and zeros int32 [out][ngroups].
+ * Outputs (device, caller-owned, not aliasing the inputs): any may be NULL
+ *   to skip it; each requested output needs its input non-NULL.
+ * Errors: GPTQ_ERR_INVALID_ARG for bits outside {2, 3, 4, 8}, sizes outside
+ * the limits, ngroups outside [1, in], zero_offset outside {0, 1} or a
+ * missing input; GPTQ_ERR_UNSUPPORTED for the divisibility rules above.
+ * Asynchronous.  out == 0 or no requested output is a no-op.
+ */
+gptq_status_t gptq_export_checkpoint(const uint32_t* qweight,
+                                     const float* scales, const int32_t* zeros,
+                                     int64_t out, int64_t in, int bits,
+                                     int ngroups, int zero_offset,
+                                     uint32_t* qweight_t, uint32_t* qzeros,
+                                     uint16_t* scales_h, void* stream);
 
 /*
  * Diagnostic with no counterpart in the method: every wait inside this

@@ -24,8 +24,8 @@ __all__ = [
     "gptq_abi_version", "gptq_last_error", "gptq_kernel_launches", "gptq_validate_config",
     "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "GPTQ_STATIC_SCRATCH_BYTES",
-    "gptq_dequantize_layer", "gptq_selftest_wait_timeout",
-    "solve_layer", "solve_block", "STATUS_NAMES",
+    "gptq_dequantize_layer", "gptq_export_checkpoint", "gptq_selftest_wait_timeout",
+    "solve_layer", "solve_block", "export_checkpoint", "STATUS_NAMES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgptq.so")
@@ -78,6 +78,10 @@ lib.gptq_quantize_layer_noalloc.restype = ctypes.c_int
 lib.gptq_dequantize_layer.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p,
                                       ctypes.c_int, _i64, _p]
 lib.gptq_dequantize_layer.restype = ctypes.c_int
+
+lib.gptq_export_checkpoint.argtypes = [_p, _p, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       _p, _p, _p, _p]
+lib.gptq_export_checkpoint.restype = ctypes.c_int
 
 lib.gptq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _p]
 lib.gptq_selftest_wait_timeout.restype = ctypes.c_int
@@ -217,6 +221,17 @@ def gptq_dequantize_layer(qweight, scales, zeros, g_idx, bits, Wq, stream=None) 
                                      _stream(stream)))
 
 
+def gptq_export_checkpoint(qweight, scales, zeros, out: int, in_: int, bits: int, ngroups: int,
+                           zero_offset: int, qweight_t=None, qzeros=None, scales_h=None,
+                           stream=None) -> None:
+    """The solver's outputs in the loaders' checkpoint layout: qweight_t
+    (in*bits/32 x out), qzeros (ngroups x out*bits/32), scales_h (float16,
+    ngroups x out).  Any output may be None to skip it."""
+    _check(lib.gptq_export_checkpoint(_ptr(qweight), _ptr(scales), _ptr(zeros), int(out), int(in_),
+                                      int(bits), int(ngroups), int(zero_offset), _ptr(qweight_t),
+                                      _ptr(qzeros), _ptr(scales_h), _stream(stream)))
+
+
 def gptq_selftest_wait_timeout(limit_ns: int, stream=None) -> int:
     """Run the bounded-wait timeout path once; returns the status code
     (GPTQ_ERR_TIMEOUT = 6 when the path works)."""
@@ -252,6 +267,23 @@ def solve_layer(W, X=None, cfg=None, S=None, n=None, with_codes=True, stream=Non
                         qweight=qweight, loss=loss, stream=stream)
     return dict(S=S, n=n, U=U, perm=perm, dead=dead, scales=scales, zeros=zeros, g_idx=g_idx,
                 loss=loss, codes=codes, qweight=qweight)
+
+
+def export_checkpoint(res, bits: int, zero_offset: int = 1, stream=None):
+    """A solve_layer result in the loaders' checkpoint layout: a dict of
+    device tensors qweight (int32, in*bits/32 x out), qzeros (int32,
+    ngroups x out*bits/32), scales (float16, ngroups x out) and g_idx."""
+    import torch
+    scales, zeros, qweight = res["scales"], res["zeros"], res["qweight"]
+    out, ng = scales.shape
+    in_ = res["g_idx"].shape[0]
+    dev = scales.device
+    qweight_t = torch.empty((in_ * bits // 32, out), dtype=torch.int32, device=dev)
+    qzeros = torch.empty((ng, out * bits // 32), dtype=torch.int32, device=dev)
+    scales_h = torch.empty((ng, out), dtype=torch.float16, device=dev)
+    gptq_export_checkpoint(qweight, scales, zeros, out, in_, bits, ng, zero_offset,
+                           qweight_t, qzeros, scales_h, stream)
+    return dict(qweight=qweight_t, qzeros=qzeros, scales=scales_h, g_idx=res["g_idx"])
 
 
 def solve_block(layers, activations, cfg=None, streams=True):

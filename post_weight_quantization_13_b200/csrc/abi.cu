@@ -249,4 +249,29 @@ gptq_status_t gptq_dequantize_layer(const uint32_t* qweight, const float* scales
   return dequantize_layer(qweight, scales, zeros, g_idx, out, in, bits, ngroups, Wq, wt, ldw, (cudaStream_t)stream);
 }
 
+gptq_status_t gptq_export_checkpoint(const uint32_t* qweight, const float* scales, const int32_t* zeros, int64_t out,
+                                     int64_t in, int bits, int ngroups, int zero_offset, uint32_t* qweight_t,
+                                     uint32_t* qzeros, uint16_t* scales_h, void* stream) {
+  clear_error();
+  if (bits != 2 && bits != 3 && bits != 4 && bits != 8)
+    return fail(GPTQ_ERR_INVALID_ARG, "bits must be 2, 3, 4 or 8 (got %d)", bits);
+  if (out < 0 || in < 1 || in > kMaxIn || out > kMaxOut)
+    return fail(GPTQ_ERR_INVALID_ARG, "layer %lld x %lld is outside this build's limits", (long long)out,
+                (long long)in);
+  if (ngroups < 1 || ngroups > in) return fail(GPTQ_ERR_INVALID_ARG, "ngroups must be in [1, in] (got %d)", ngroups);
+  if (zero_offset != 0 && zero_offset != 1)
+    return fail(GPTQ_ERR_INVALID_ARG, "zero_offset must be 0 or 1 (got %d)", zero_offset);
+  if (qweight_t && (in * bits) % 32 != 0)
+    return fail(GPTQ_ERR_UNSUPPORTED, "qweight_t needs in*bits %% 32 == 0 (in=%lld, bits=%d)", (long long)in, bits);
+  if (qzeros && (out * bits) % 32 != 0)
+    return fail(GPTQ_ERR_UNSUPPORTED, "qzeros needs out*bits %% 32 == 0 (out=%lld, bits=%d)", (long long)out, bits);
+  if ((qweight_t && !qweight) || (qzeros && !zeros) || (scales_h && !scales))
+    return fail(GPTQ_ERR_INVALID_ARG, "each requested output needs its input (qweight, zeros, scales)");
+  if (out == 0 || (!qweight_t && !qzeros && !scales_h)) return GPTQ_OK;
+  gptq_status_t s = check_device();
+  if (s != GPTQ_OK) return s;
+  return export_checkpoint(qweight, scales, zeros, out, in, bits, ngroups, zero_offset, qweight_t, qzeros, scales_h,
+                           (cudaStream_t)stream);
+}
+
 }  // extern "C"

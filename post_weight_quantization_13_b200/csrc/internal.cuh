@@ -53,6 +53,9 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
                              const int32_t* perm, const uint8_t* dead, const gptq_config_t* cfg, int32_t* codes,
                              uint32_t* qweight, float* scales, int32_t* zeros, int32_t* g_idx, float* loss, void* ws,
                              size_t ws_bytes, cudaStream_t st);
+gptq_status_t export_checkpoint(const uint32_t* qweight, const float* scales, const int32_t* zeros, int64_t out,
+                                int64_t in, int bits, int ngroups, int zero_offset, uint32_t* qweight_t,
+                                uint32_t* qzeros, uint16_t* scales_h, cudaStream_t st);
 gptq_status_t hessian_accumulate(float* S, int64_t in, const void* X, gptq_dtype_t xt, int64_t tokens, int64_t ldx,
                                  cudaStream_t st);
 

@@ -124,3 +124,21 @@ def test_calls_reject_bad_arguments_before_any_launch(g):
                                    ctypes.byref(c3), None, ctypes.c_void_p(256),
                                    *([ctypes.c_void_p(256)] * 3), None, None, 0, None) == 1
     assert "multiple of 32" in g.gptq_last_error()
+
+
+def test_export_checkpoint_rejects_bad_arguments_before_any_launch(g):
+    lib = g.lib
+    p = ctypes.c_void_p(256)
+    # bits, ngroups, zero_offset, missing input, divisibility of in*bits and out*bits
+    assert lib.gptq_export_checkpoint(p, p, p, 8, 32, 5, 1, 1, p, p, p, None) == 1
+    assert lib.gptq_export_checkpoint(p, p, p, 8, 32, 4, 0, 1, p, p, p, None) == 1
+    assert lib.gptq_export_checkpoint(p, p, p, 8, 32, 4, 33, 1, p, p, p, None) == 1
+    assert lib.gptq_export_checkpoint(p, p, p, 8, 32, 4, 1, 2, p, p, p, None) == 1
+    assert "zero_offset" in g.gptq_last_error()
+    assert lib.gptq_export_checkpoint(None, p, p, 8, 32, 4, 1, 1, p, None, None, None) == 1
+    assert lib.gptq_export_checkpoint(p, p, p, 8, 36, 3, 1, 1, p, None, None, None) == 7
+    assert lib.gptq_export_checkpoint(p, p, p, 12, 32, 3, 1, 1, None, p, None, None) == 7
+    assert "out*bits" in g.gptq_last_error()
+    # nothing requested, or out == 0: a no-op that needs no GPU
+    assert lib.gptq_export_checkpoint(p, p, p, 8, 32, 4, 1, 1, None, None, None, None) == 0
+    assert lib.gptq_export_checkpoint(p, p, p, 0, 32, 4, 1, 1, p, p, p, None) == 0
