@@ -368,6 +368,7 @@ def checkpoint_layout(codes, scales, zeros, g_idx, bits: int, zero_offset: int =
                 scales=np.asarray(scales, np.float32).T.astype(np.float16),
                 g_idx=np.asarray(g_idx).astype(np.int32))
 
+
 def g_index(perm: np.ndarray, group_size: int) -> np.ndarray:
     """g_idx[c] = group of original column c = (its processing position) //
     group_size; 0 for group_size = -1."""

@@ -24,3 +24,13 @@ def lib():
         pytest.skip("no CUDA device")
     import post_weight_quantization_13_b200 as g
     return g
+
+
+def pytest_sessionstart(session):
+    """With GPTQ_ORACLE_MUTANT set (only by test_oracle_mutants.py, in a
+    child process), plant that mistake in the oracle before any test runs."""
+    name = os.environ.get("GPTQ_ORACLE_MUTANT")
+    if name:
+        sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
+        import oracle_mutants
+        oracle_mutants.apply(name)

@@ -138,6 +138,27 @@ def test_dead_channels():
         assert np.all(deq[:, c] == 0)
 
 
+def test_fix_dead_sets_unit_diagonal_before_dampening():
+    """A channel with H_ii = 0 gets H_ii = 1 and nothing else changes; with no
+    dampening the fixed Hessian still has a Cholesky factor, and the damping
+    mean counts the fixed 1."""
+    H = np.array([[2.0, 0.0, 0.5],
+                  [0.0, 0.0, 0.0],
+                  [0.5, 0.0, 3.0]])
+    F, dead = O.fix_dead(H)
+    assert dead.tolist() == [False, True, False]
+    assert F[1, 1] == 1.0
+    keep = np.ones_like(H, dtype=bool)
+    keep[1, 1] = False
+    assert np.array_equal(F[keep], H[keep])
+    O.upper_cholesky_of_inverse(O.dampen(F, 0.0))   # positive definite
+    # lambda = 0.3 * mean(2, 1, 3) = 0.6 (the fixed diagonal counts)
+    np.testing.assert_allclose(np.diag(O.dampen(F, 0.3)), [2.6, 1.6, 3.6])
+    S = H * 5.0
+    r = O.prepare(S, 10, 0.0, False)     # H0 = 2 S / 10 = H
+    assert r["dead"].tolist() == [False, True, False] and r["Hp"][1, 1] == 1.0
+
+
 # ------------------------------------------------------------- step 3: act order
 def test_act_order_is_stable_descending_permutation():
     d = np.array([3.0, 1.0, 3.0, 7.0, 1.0, 0.5, 7.0])
@@ -223,12 +244,36 @@ def test_quantizer_range_and_grid(bits, sym):
     assert np.all(np.abs(w - deq)[inside] <= 0.5 * s.astype(np.float64)[:, None].repeat(16, 1)[inside] * (1 + 1e-6))
     if sym:
         assert np.all(z == (maxq + 1) // 2)
+        # the grid spans [-max|w|, max|w|]: scale = 2 max|w| / maxq
+        a_ = np.max(np.abs(w.astype(np.float32)), axis=1)
+        a_[a_ == 0] = 1
+        assert np.array_equal(s, (np.float32(2) * a_) / np.float32(maxq))
     else:
         # zero is exactly representable
         zq = O.quantize_codes(np.zeros(50), s, z, bits)
         assert np.all(O.dequantize_codes(zq, s, z) == 0)
         # asym range covers [min, max] of the group
         assert np.all(deq.min(1) <= w.min(1) + 0.5 * s + 1e-12)
+
+
+def test_quantizer_hand_values():
+    """Worked by hand.  sym, 4 bits, w = (0.3, -0.6, 0.1): max|w| = 0.6,
+    scale = 1.2 / 15 = 0.08, zero = 8; w / scale = 3.75, -7.5, 1.25 round
+    (half to even) to 4, -8, 1, so the codes are 12, 0, 9.  asym, 2 bits,
+    w = (-0.2, 0.1, 0.4): range [-0.2, 0.4], scale = 0.6 / 3 = 0.2, zero =
+    rint(0.2 / 0.2) = 1; w / scale = -1, 0.5, 2 round to -1, 0, 2, so the
+    codes are 0, 1, 3."""
+    w = np.array([[0.3, -0.6, 0.1]])
+    s, z = O.group_params(w, 4, True)
+    np.testing.assert_allclose(s, [0.08], rtol=1e-6)
+    assert z.tolist() == [8]
+    q = [O.quantize_codes(w[:, j], s, z, 4)[0] for j in range(3)]
+    assert q == [12, 0, 9]
+    w = np.array([[-0.2, 0.1, 0.4]])
+    s, z = O.group_params(w, 2, False)
+    np.testing.assert_allclose(s, [0.2], rtol=1e-6)
+    assert z.tolist() == [1]
+    assert [O.quantize_codes(w[:, j], s, z, 2)[0] for j in range(3)] == [0, 1, 3]
 
 
 # ------------------------------------------------------------- step 5: sweep
