@@ -365,9 +365,10 @@ def run_ours(args):
     if os.path.exists(tpath):
         with open(tpath) as f:
             t = json.load(f).get(f"hessian_syrk:{wl.name}")
-        # counters taken on an older build of the kernel no longer apply
+        # counters taken on an older build of the kernel no longer apply; X is
+        # read once per drain, so the traffic scales with the tokens
         if t and t.get("kernel_sources_sha256") == kernel_sources_sha256():
-            traffic = t.get("bytes_per_launch")
+            traffic = int(t.get("bytes_per_launch") * n_tok // t.get("tokens", n_tok))
 
     # e2e: host buffers in, results out, every step, through the same ABI
     # calls.  Calibration tokens arrive as host batches (chunk-major pinned
