@@ -45,6 +45,7 @@ struct GemmArgs {
   int batch = 1;
   int64_t bs_p_row = 0, bs_p_k = 0, bs_q_row = 0, bs_q_k = 0, bs_c_row = 0, bs_c_col = 0;
   int tri = 0;                                  // upper-triangle SYRK schedule (P == Q)
+  int p_tile = 256;                             // grid schedule: P rows per output tile (256 or 128)
   uint32_t* status = nullptr;                   // device status word (may be null)
 };
 

@@ -545,6 +545,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
         g.R = out;
         g.Cn = o1 - c0;
         g.K = BW;
+        g.p_tile = 128;
         g.p_row0 = 0;
         g.p_k0 = k - o0;
         g.q_row0 = c0;
@@ -568,6 +569,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
       g.R = out;
       g.Cn = in - o1;
       g.K = o1 - o0;
+      g.p_tile = 128;
       g.p_row0 = 0;
       g.p_k0 = 0;
       g.q_row0 = o1;

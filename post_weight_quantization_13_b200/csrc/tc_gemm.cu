@@ -68,6 +68,7 @@ struct KParams {
   int R, Cn;
   // grid schedule
   int nq, npt, ntiles;
+  int ptile;  // P rows per output tile: 256, or 128 for more and smaller pipeline stages
   int64_t bs_p_row, bs_p_k, bs_q_row, bs_q_k, bs_c_row, bs_c_col;
   // tri schedule
   int n_in, nss;
@@ -161,8 +162,8 @@ __host__ __device__ int round_pieces(const KParams& kp, int cta, int round, Piec
   Piece& p = pc[0];
   p.q0 = qt * 128;
   p.nh = 1;
-  p.p0 = pt * 256;
-  const int rows = min(256, kp.R - p.p0);
+  p.p0 = pt * kp.ptile;
+  const int rows = min(kp.ptile, kp.R - p.p0);
   p.np = (rows + 15) & ~15;
   p.qslot = 0;
   p.prow = 0;
@@ -747,10 +748,14 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
     kp.slot_bytes = 2 * kQTileBytes * split;
     kp.p_rows_max = 256;
   } else {
+    // 128-row tiles halve a stage (three stages fit instead of two for
+    // 3xTF32); the banded schedule below keeps 256-row tiles
+    const bool lower = a.mask == 2 && a.batch == 1;
+    kp.ptile = (!lower && a.p_tile == 128) ? 128 : 256;
     kp.nq = (int)((a.Cn + 127) / 128);
-    kp.npt = (int)((a.R + 255) / 256);
+    kp.npt = (int)((a.R + kp.ptile - 1) / kp.ptile);
     kp.ntiles = kp.nq * kp.npt * a.batch;
-    if (a.mask == 2 && a.batch == 1) {  // skip tiles entirely above the kept band
+    if (lower) {  // skip tiles entirely above the kept band
       kp.lower = 1;
       kp.mask_off = a.mask_off;
       kp.ntiles = 0;
@@ -768,7 +773,7 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
     kp.rounds = (kp.ntiles + grid - 1) / grid;
     kp.qslots = 1;
     kp.slot_bytes = kQTileBytes * split;
-    kp.p_rows_max = 256;
+    kp.p_rows_max = kp.ptile;
   }
   // TMA epilogue when the output allows it: beta 0 (store) or 1 (reduce-add),
   // 16-byte aligned rows, and masks only where masked elements can add 0.
