@@ -35,13 +35,26 @@ UNIT = "weights/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def kernel_sources_sha256():
-    """Hash of the sources the SYRK kernel is built from."""
+def strip_comments(src):
+    """C/C++ source without comments and blank space, so that a change to a
+    comment alone keeps a kernel's recorded counters valid."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
+def kernel_sources_sha256(texts=None):
+    """Hash of the code (comments excluded) the SYRK kernel is built from."""
     import hashlib
     h = hashlib.sha256()
     for name in ("tc_gemm.cu", "gemm.cuh", "common.cuh"):
-        with open(os.path.join(ROOT, "post_weight_quantization_13_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        if texts is None:
+            with open(os.path.join(ROOT, "post_weight_quantization_13_b200", "csrc", name)) as f:
+                src = f.read()
+        else:
+            src = texts[name]
+        h.update(strip_comments(src).encode())
     return h.hexdigest()
 
 

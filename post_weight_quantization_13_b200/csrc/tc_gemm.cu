@@ -2,9 +2,10 @@
 //
 // One persistent CTA per SM, warp-specialised:
 //   warp 0      TMA producer: fills a ring of shared-memory stages with
-//               K-major operand tiles (64-byte rows, 64-byte swizzle).  Row
-//               ranges are cut into power-of-two boxes (256/128/64/32/16
-//               rows), so a stage needs only a handful of copies.
+//               K-major operand tiles (128-byte rows, 128-byte swizzle: 64
+//               16-bit or 32 tf32 elements of k per row).  Row ranges are
+//               cut into power-of-two boxes (256/128/64/32/16 rows), so a
+//               stage needs only a handful of copies.
 //   warp 1      owns the tensor memory (all 512 columns) and issues
 //               tcgen05.mma from one thread; completion is signalled back to
 //               the producer (stage free) and to the epilogue (accumulator
@@ -22,11 +23,13 @@
 //         super-strips; super-strip s needs rows [0, 256(s+1)), i.e. s + 1
 //         pieces of 256 rows.  One piece per CTA and round; all CTAs stream
 //         the same k-window of X together, which keeps X L2-resident.  With
-//         one 256 x 256 piece per round a stage is 32 KB, so seven stages
+//         one 256 x 256 piece per round a stage is 64 KB, so three stages
 //         fit in shared memory.
-//   grid  regular 128 x 256 tiles (optionally batched), one per round, with
-//         two tensor-memory buffers so a tile's epilogue overlaps the next
-//         tile's main loop.
+//   grid  regular tiles of 128 C columns by 256 (or, on request, 128) C
+//         rows (optionally batched), one per round, with two tensor-memory
+//         buffers so a tile's epilogue overlaps the next tile's main loop.
+//         128-row tiles halve a stage, so a 3xTF32 product keeps three
+//         stages in flight instead of two.
 // Long k ranges are cut into chunks; after each chunk the accumulators are
 // drained into C with round-to-nearest adds, which bounds the error of the
 // tensor core's in-place fp32 accumulation.
