@@ -24,6 +24,15 @@ __device__ __forceinline__ void raise_status(uint32_t* st, uint32_t flag) {
   if (st) atomicOr(st, flag);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel in the stream is still
+// running; this waits until that kernel has completed and its writes are
+// visible.  For an ordinary launch it returns at once.  Every thread of a
+// kernel that can be launched this way calls it before its first access to
+// memory the previous kernels write, and before it exits, so that the
+// ordering stays transitive along the stream.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Upper bound on any device-side spin (nanoseconds of %globaltimer).  A
 // legitimate wait in these kernels lasts well under 100 ms; a wait that
 // reaches the bound is a bug, and the kernel records ST_TIMEOUT and unwinds.

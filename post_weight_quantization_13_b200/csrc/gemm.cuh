@@ -46,6 +46,8 @@ struct GemmArgs {
   int64_t bs_p_row = 0, bs_p_k = 0, bs_q_row = 0, bs_q_k = 0, bs_c_row = 0, bs_c_col = 0;
   int tri = 0;                                  // upper-triangle SYRK schedule (P == Q)
   int p_tile = 256;                             // grid schedule: P rows per output tile (256 or 128)
+  int pdl = 0;                                  // 1: programmatic dependent launch (prologue overlaps
+                                                //    the previous kernel of the stream)
   uint32_t* status = nullptr;                   // device status word (may be null)
 };
 

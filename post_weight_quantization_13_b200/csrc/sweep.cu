@@ -126,6 +126,10 @@ __global__ void __launch_bounds__(NT) sweep_kernel(const SweepParams sp) {
     Esh[e] = 0.f;
     Esl[e] = 0.f;
   }
+  // U's diagonal blocks were written before the first sweep of the layer,
+  // which is an ordinary launch; W, the scales and E come from the kernels
+  // just before this one, so a dependent launch waits here for them
+  grid_dependency_wait();
   const int warp = tid >> 5, lane = tid & 31;
   const int rl = warp * 8 + (lane >> 2);
   const int q = lane & 3;
@@ -384,15 +388,27 @@ cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
   return simt_gemm(g, st);
 }
 
+// pdl: programmatic dependent launch.  Only for a sweep that follows a
+// kernel of the same layer's sweep chain (a lazy update): its bulk copy of
+// U's diagonal block is issued before it waits on that kernel.
 template <int GSB>
-cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st) {
+cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st, bool pdl) {
   const size_t smem = (size_t)(BW * 4 * UPITCH + BW + 2 * ROWS * EPITCH) * sizeof(float) + ROWS * CPITCH;
   cudaError_t ce = ensure_smem_limit((const void*)sweep_kernel<GSB>, (int)smem);
   if (ce != cudaSuccess) return ce;
-  const unsigned grid = (unsigned)((sp.out + ROWS - 1) / ROWS);
-  sweep_kernel<GSB><<<grid, NT, smem, st>>>(sp);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((sp.out + ROWS - 1) / ROWS));
+  cfg.blockDim = dim3(NT);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  ce = cudaLaunchKernelEx(&cfg, sweep_kernel<GSB>, sp);
   note_launch();
-  return cudaGetLastError();
+  return ce != cudaSuccess ? ce : cudaGetLastError();
 }
 
 }  // namespace
@@ -517,19 +533,19 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
       cudaError_t e;
       switch (gsb) {
         case 8:
-          e = launch_sweep<8>(sp, st);
+          e = launch_sweep<8>(sp, st, k > 0);
           break;
         case 16:
-          e = launch_sweep<16>(sp, st);
+          e = launch_sweep<16>(sp, st, k > 0);
           break;
         case 32:
-          e = launch_sweep<32>(sp, st);
+          e = launch_sweep<32>(sp, st, k > 0);
           break;
         case 64:
-          e = launch_sweep<64>(sp, st);
+          e = launch_sweep<64>(sp, st, k > 0);
           break;
         case 128:
-          e = launch_sweep<128>(sp, st);
+          e = launch_sweep<128>(sp, st, k > 0);
           break;
         default:
           return fail(GPTQ_ERR_UNSUPPORTED, "group_size %d is not supported by the sweep kernel", gs);
@@ -546,6 +562,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
         g.Cn = o1 - c0;
         g.K = BW;
         g.p_tile = 128;
+        g.pdl = 1;
         g.p_row0 = 0;
         g.p_k0 = k - o0;
         g.q_row0 = c0;
@@ -570,6 +587,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
       g.Cn = in - o1;
       g.K = o1 - o0;
       g.p_tile = 128;
+      g.pdl = 1;
       g.p_row0 = 0;
       g.p_k0 = 0;
       g.q_row0 = o1;

@@ -244,6 +244,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = *tmem_slot;
+  // everything above touches only this CTA's shared and tensor memory and the
+  // kernel parameters: under a dependent launch (the 3xTF32 lazy updates of
+  // the sweep) it overlaps the previous kernel, and the operand loads and
+  // output writes below wait for it
+  if constexpr (OP == OP_TF32X3) grid_dependency_wait();
 
   const uint32_t q_region = (uint32_t)(kp.qslots * kp.slot_bytes);
   const uint32_t p_comp = (uint32_t)kp.p_rows_max * kRowBytes;  // one component of the P region
@@ -663,12 +668,22 @@ int bk_of(int op) { return op == OP_TF32X3 ? 32 : 64; }  // elements per 128-byt
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
 template <int OP>
-cudaError_t launch(const TmaMaps& maps, const KParams& kp, int grid, size_t smem, cudaStream_t st) {
+cudaError_t launch(const TmaMaps& maps, const KParams& kp, int grid, size_t smem, cudaStream_t st, bool pdl) {
   cudaError_t ce = ensure_smem_limit((const void*)tc_gemm_kernel<OP>, 232448);
   if (ce != cudaSuccess) return ce;
-  tc_gemm_kernel<OP><<<grid, kThreads, smem, st>>>(maps, kp);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  ce = cudaLaunchKernelEx(&cfg, tc_gemm_kernel<OP>, maps, kp);
   note_launch();
-  return cudaGetLastError();
+  return ce != cudaSuccess ? ce : cudaGetLastError();
 }
 
 }  // namespace
@@ -808,11 +823,11 @@ cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t st, int num_sms) {
   const size_t smem = 1024 + (size_t)kp.stages * kp.stage_bytes + (kp.epi_tma ? 2 * kStageTileBytes : 0) + 256;
   switch (a.op) {
     case OP_F16:
-      return launch<OP_F16>(maps, kp, grid, smem, st);
+      return launch<OP_F16>(maps, kp, grid, smem, st, false);
     case OP_BF16:
-      return launch<OP_BF16>(maps, kp, grid, smem, st);
-    default:
-      return launch<OP_TF32X3>(maps, kp, grid, smem, st);
+      return launch<OP_BF16>(maps, kp, grid, smem, st, false);
+    default:  // only this instantiation waits on the previous kernel
+      return launch<OP_TF32X3>(maps, kp, grid, smem, st, a.pdl != 0);
   }
 }
 
