@@ -207,7 +207,12 @@ gptq_status_t gptq_prepare_hinv(const float* S, int64_t n, int64_t in,
  *   loss     fp32[out] or NULL: sum over columns of e^2 for each row (the
  *            quadratic error (W - deq) H (W - deq)^T with the damped H).
  * ws / ws_bytes: workspace from gptq_workspace_bytes(out, in, cfg).
- * Asynchronous.  out == 0 is a no-op.
+ * Asynchronous.  out == 0 is a no-op.  Inside the call, the kernels of the
+ * sweep chain after the first are programmatic dependent launches on the
+ * caller's stream.  Each waits for the kernel before it, so the call's
+ * work is ordered after everything already queued on the stream and before
+ * everything queued after it, as with ordinary launches (also under stream
+ * capture).
  */
 gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out,
                                   int64_t in, int64_t ldw, const float* U,
