@@ -211,8 +211,7 @@ gptq_status_t gptq_prepare_hinv(const float* S, int64_t n, int64_t in,
  * sweep chain after the first are programmatic dependent launches on the
  * caller's stream.  Each waits for the kernel before it, so the call's
  * work is ordered after everything already queued on the stream and before
- * everything queued after it, as with ordinary launches (also under stream
- * capture).
+ * everything queued after it, as with ordinary launches.
  */
 gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out,
                                   int64_t in, int64_t ldw, const float* U,
