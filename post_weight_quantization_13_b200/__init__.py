@@ -275,6 +275,8 @@ def export_checkpoint(res, bits: int, zero_offset: int = 1, stream=None):
     ngroups x out*bits/32), scales (float16, ngroups x out) and g_idx."""
     import torch
     scales, zeros, qweight = res["scales"], res["zeros"], res["qweight"]
+    if qweight is None:
+        raise ValueError("the result has no packed qweight (in * bits is not a multiple of 32)")
     out, ng = scales.shape
     in_ = res["g_idx"].shape[0]
     dev = scales.device
