@@ -76,6 +76,8 @@ def parse():
                     help="lazy-batch width of the sweep (default: the workload's)")
     ap.add_argument("--desc-act", action="store_true",
                     help="process columns in act-order (default: the workload's, off)")
+    ap.add_argument("--unsampled", action="store_true",
+                    help="with --impl reference: time one whole oracle layer solve instead of samples")
     return ap.parse_args()
 
 
@@ -177,64 +179,117 @@ def oracle_setup(wl, layer, q, W, X):
     return dict(S=S, nt=nt, U=prep["U"], perm=prep["perm"])
 
 
-def oracle_sample(wl, layer, q, W, X, setup, tokens, prep_n, rows):
+# The one sampling recipe both oracle legs use (the GPU line's cpu_baseline
+# and the reference arm): the Hessian over SAMPLE_TOKENS tokens, the whole
+# prepare, and the sweep of SAMPLE_ROWS rows over all columns.
+SAMPLE_TOKENS = 4096
+SAMPLE_ROWS = 64
+
+
+def oracle_sample(wl, layer, q, W, X, setup, tokens=SAMPLE_TOKENS, rows=SAMPLE_ROWS):
     """The float64 oracle, as it stands, on a bounded sample of one layer
     solve, scaled to the whole layer: the Hessian over ``tokens`` tokens
-    (x all/tokens), the prepare on a ``prep_n`` x ``prep_n`` principal block
-    (x (in/prep_n)^3, its cost being cubic) and the column sweep of ``rows``
-    rows over all columns (x out/rows).  Returns (weights/s, detail)."""
+    (x all/tokens), the whole prepare (unscaled), and the column sweep of
+    ``rows`` rows over all columns (x out/rows).  Returns (weights/s,
+    detail)."""
     import numpy as np
     import oracle as O
     n = wl.tokens
     t0 = time.perf_counter()
     O.hessian([np.asarray(X[:, :tokens])])
     t_h = time.perf_counter() - t0
-    pn = min(prep_n, layer.in_)
     t0 = time.perf_counter()
-    O.prepare(setup["S"][:pn, :pn], setup["nt"], q.damp_percent, q.desc_act)
+    O.prepare(setup["S"], setup["nt"], q.damp_percent, q.desc_act)
     t_p = time.perf_counter() - t0
     r = min(rows, layer.out)
     Wp = np.asarray(W[:r], dtype=np.float64)[:, setup["perm"]]
     t0 = time.perf_counter()
     O.sweep_blocked(Wp, setup["U"], q.bits, q.group_size, q.sym, q.block_size)
     t_s = time.perf_counter() - t0
-    sh, sp, ss = n / tokens, (layer.in_ / pn) ** 3, layer.out / r
-    total = t_h * sh + t_p * sp + t_s * ss
-    sample = (f"Hessian over {tokens} of {n} tokens (x{sh:.0f}), prepare on a {pn}x{pn} block "
-              f"(x{sp:.0f}), sweep of {r} of {layer.out} rows (x{ss:.0f}); "
+    sh, ss = n / tokens, layer.out / r
+    total = t_h * sh + t_p + t_s * ss
+    sample = (f"Hessian over {tokens} of {n} tokens (x{sh:.0f}), the whole {layer.in_}x{layer.in_} "
+              f"prepare (x1), sweep of {r} of {layer.out} rows (x{ss:.0f}); "
               f"{t_h + t_p + t_s:.2f} s measured")
     return layer.out * layer.in_ / total, dict(
         cores=_blas_threads(), sample=sample, est_s_per_layer=total,
-        split_s=dict(hessian=t_h * sh, prepare=t_p * sp, sweep=t_s * ss))
+        split_s=dict(hessian=t_h * sh, prepare=t_p, sweep=t_s * ss))
+
+
+def oracle_unsampled(wl, layer, q, W, X):
+    """One whole layer solve by the oracle, nothing sampled: the Hessian over
+    every token (in 16384-token chunks), the prepare and the sweep of every
+    row.  Returns (seconds, split)."""
+    import numpy as np
+    import oracle as O
+    t0 = time.perf_counter()
+    S = np.zeros((layer.in_, layer.in_), np.float64)
+    for c0 in range(0, X.shape[1], 16384):
+        O.hessian_accumulate(S, X[:, c0:c0 + 16384])
+    t1 = time.perf_counter()
+    prep = O.prepare(S, X.shape[1], q.damp_percent, q.desc_act)
+    t2 = time.perf_counter()
+    Wd = np.asarray(W, np.float64)
+    Wd[:, prep["dead"]] = 0.0
+    O.sweep_blocked(Wd[:, prep["perm"]], prep["U"], q.bits, q.group_size, q.sym, q.block_size)
+    t3 = time.perf_counter()
+    return t3 - t0, dict(hessian=t1 - t0, prepare=t2 - t1, sweep=t3 - t2)
+
+
+def config_of(wl, layer, q, world, x_bytes=None):
+    """The line's config, identical in both arms."""
+    return {"workload": wl.name, "out": layer.out, "in": layer.in_, "tokens": wl.tokens,
+            "bits": q.bits, "group_size": q.group_size, "sym": q.sym, "desc_act": q.desc_act,
+            "damp_percent": q.damp_percent, "block_size": q.block_size, "x_dtype": wl.x_dtype,
+            "l2": ("inputs larger than L2 (X %.2f GiB)" % ((x_bytes if x_bytes is not None else
+                   layer.in_ * wl.tokens * (2 if wl.x_dtype == "float16" else 4)) / 2**30)),
+            "parallelism": f"replicas x{world}"}
 
 
 def run_reference(args):
     """--impl reference: the CPU oracle (float64 numpy) on the host cores,
-    each step a bounded sample of the same layer solve."""
+    each step one bounded sample of the same layer solve (the recipe the GPU
+    line's cpu_baseline uses).  With --unsampled: one whole layer solve by the
+    oracle instead, timed once, beside the recipe's estimate."""
     import gen
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     wl = gen.WORKLOADS[args.workload]
     layer = wl.layers[0]
     q = quant_of(wl, args)
     W = gen.weight(wl, layer)
-    X = gen.x_full(wl, layer.site, tokens=2048)
+    if getattr(args, "unsampled", False):
+        X = gen.x_full(wl, layer.site)
+        setup = oracle_setup(wl, layer, q, W, X)
+        v_est, d_est = oracle_sample(wl, layer, q, W, X, setup)
+        secs, split = oracle_unsampled(wl, layer, q, W, X)
+        print(json.dumps({"impl": "reference", "unsampled": True, "config": config_of(wl, layer, q, world),
+                          "seconds_per_layer": secs, "split_s": split, "cores": _blas_threads(),
+                          "recipe_estimate_s": d_est["est_s_per_layer"], "recipe_split_s": d_est["split_s"],
+                          "recipe_sample": d_est["sample"]}), flush=True)
+        return
+    X = gen.x_full(wl, layer.site, tokens=max(2048, SAMPLE_TOKENS))
     setup = oracle_setup(wl, layer, q, W, X)
     vals, detail = [], None
+    t_run = time.perf_counter()
     for i in range(args.warmup + args.steps):
-        v, detail = oracle_sample(wl, layer, q, W, X, setup, tokens=512, prep_n=1024, rows=16)
+        v, detail = oracle_sample(wl, layer, q, W, X, setup)
         if i >= args.warmup:
             vals.append(v)
+    t_run = time.perf_counter() - t_run
     v = statistics.median(vals)
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * layer.out * layer.in_ / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": wl.name, "out": layer.out, "in": layer.in_, "tokens": wl.tokens,
-                       "bits": q.bits, "group_size": q.group_size, "desc_act": q.desc_act},
+            "config": config_of(wl, layer, q, world),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": detail["cores"], "kind": "oracle",
-                             "sample": detail["sample"]},
+                             "sample": detail["sample"],
+                             "note": ("value and ms_per_step are the whole layer's oracle time "
+                                      "estimated from each step's sample; the run itself took "
+                                      f"{t_run:.1f} s for {args.warmup + args.steps} samples")},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -359,14 +414,18 @@ def run_ours(args):
     hess_ms = statistics.mean(phase_ms["syrk"])
     flops = in_ * (in_ + 1) * n_tok
     peaks, peak_src = load_peaks()
-    peak = peaks.get("bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"])
+    # the burst peak for a timed region under a second (the GPU has not yet
+    # settled at its power cap), the sustained one for a longer run
+    burst = elapsed < 1000.0
+    peak_key = "bf16_tflops" if burst else "bf16_tflops_sustained"
+    peak = peaks.get(peak_key, PEAKS_FALLBACK[peak_key])
     achieved = flops / (hess_ms / 1e3) / 1e12
     # whole-step roofline: each step at the slower of its tensor-core and HBM
     # floors (a1 Hessian and a4 factorisation on tensor cores, a6 lazy
     # update and the gathers/packing on HBM), against the measured peaks
     bw = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"]) * 1e9
     pf = peak * 1e12
-    nblk = -(-in_ // q.block_size)
+    nblk = -(-in_ // 128)
     terms = {"a1_hessian": flops / pf, "a4_factor": (2.0 / 3.0) * in_ ** 3 / pf,
              "a6_lazy_update": 4.0 * out * in_ * max(nblk - 1, 0) / bw,
              "a2_a3_a7_bytes": (8.0 * in_ * in_ + out * in_ * (2 + 4 + q.bits / 8)) / bw}
@@ -483,8 +542,7 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         setup = oracle_setup(wl, layer, q, Wh.numpy(), Xh.numpy())
-        v, d = oracle_sample(wl, layer, q, Wh.numpy(), Xh.numpy(), setup, tokens=4096,
-                             prep_n=layer.in_, rows=64)
+        v, d = oracle_sample(wl, layer, q, Wh.numpy(), Xh.numpy(), setup)
         cpu = {"value": v, "unit": UNIT, "cores": d["cores"], "kind": "oracle", "sample": d["sample"],
                "est_s_per_layer": d["est_s_per_layer"], "split_s": d["split_s"]}
 
@@ -493,19 +551,15 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
-            "config": {"workload": wl.name, "out": out, "in": in_, "tokens": n_tok,
-                       "bits": q.bits, "group_size": q.group_size, "sym": q.sym,
-                       "desc_act": q.desc_act, "damp_percent": q.damp_percent,
-                       "block_size": q.block_size, "x_dtype": wl.x_dtype,
-                       "l2": f"inputs larger than L2 (X {Xh.numel() * Xh.element_size() / 2**30:.2f} GiB)",
-                       "parallelism": f"replicas x{world}"},
+            "config": config_of(wl, layer, q, world, Xh.numel() * Xh.element_size()),
             "split_ms": {k: statistics.mean(v) for k, v in phase_ms.items()},
             "roofline": {"kernel": "tc_gemm_kernel<f16> (Hessian S += X X^T, tcgen05)",
                          "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "frac_of_burst_peak": achieved / peaks.get("bf16_tflops",
-                                                                    PEAKS_FALLBACK["bf16_tflops"]),
-                         "peak_source": f"{peak_src} bf16 sustained (fp16 dense rate = bf16)",
+                         "frac_of_sustained_peak": achieved / peaks.get(
+                             "bf16_tflops_sustained", PEAKS_FALLBACK["bf16_tflops_sustained"]),
+                         "peak_source": (f"{peak_src} bf16 {'burst' if burst else 'sustained'} "
+                                         f"(timed region {elapsed / 1e3:.2f} s; fp16 dense rate = bf16)"),
                          "flops_per_launch": flops},
             "step_roofline": step_roof,
             "dequant": deq,

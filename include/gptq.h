@@ -212,6 +212,11 @@ gptq_status_t gptq_prepare_hinv(const float* S, int64_t n, int64_t in,
  * caller's stream.  Each waits for the kernel before it, so the call's
  * work is ordered after everything already queued on the stream and before
  * everything queued after it, as with ordinary launches.
+ * The call returns before its kernels run, so a failure inside them (a
+ * bounded device-side wait that gave up: GPTQ_ERR_TIMEOUT) is not in its
+ * return value: it is raised in the status word at the start of ws, which
+ * gptq_workspace_status(ws, ws_bytes, stream) reads back once the stream has
+ * finished the call.
  */
 gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out,
                                   int64_t in, int64_t ldw, const float* U,
@@ -220,6 +225,26 @@ gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out,
                                   uint32_t* qweight, float* scales,
                                   int32_t* zeros, int32_t* g_idx, float* loss,
                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Device-side status of the last gptq_prepare_hinv or gptq_quantize_layer
+ * call that used workspace ws.  Each of those calls clears a 32-bit status
+ * word at the start of ws on its stream before its first kernel; its kernels
+ * only ever raise flags in it.  This call waits for stream, reads the word
+ * and returns:
+ *   GPTQ_ERR_TIMEOUT    a bounded device-side wait gave up (the call's
+ *                       outputs are incomplete);
+ *   GPTQ_ERR_NONFINITE  S held NaN or Inf (prepare);
+ *   GPTQ_ERR_NOT_PD     a pivot of the factorisation was not positive
+ *                       (prepare);
+ *   GPTQ_OK             none of these.
+ * Pass the stream the call was made on (or one ordered after it).  ws must
+ * be 256-byte aligned and ws_bytes >= 256.  gptq_prepare_hinv already
+ * returns this status itself; for gptq_quantize_layer this call is the only
+ * way to see it.
+ */
+gptq_status_t gptq_workspace_status(const void* ws, size_t ws_bytes,
+                                    void* stream);
 
 /*
  * Dequantize: Wq[r][c] = scales[r][g] * (code[r][c] - zeros[r][g]) with
@@ -316,11 +341,21 @@ gptq_status_t gptq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
  * need gptq_quantize_layer with a caller workspace.
  *
  * Device and setup: the call works on the calling thread's current device;
- * stream must belong to it.  The first call on each device looks up the
- * scratch's address with cudaGetSymbolAddress (which may also load the
- * library's device code on that device) and caches it; make that first call
- * before any stream capture begins.  Later calls only read the cached
- * address.
+ * stream must belong to it.  The first call on each device (more precisely,
+ * on each CUDA context of a device: after cudaDeviceReset the next call sets
+ * up again) is the set-up.  It looks up the scratch's address with
+ * cudaGetSymbolAddress, which creates the device's primary context if the
+ * thread has none yet, and makes the driver load every kernel the call can
+ * launch.  Loading device code reserves device memory inside the driver, so
+ * make the first call on each device outside the situations this entry point
+ * is for (allocator callbacks, out-of-memory handlers) and before any stream
+ * capture begins; gptq_quantize_layer_noalloc_status also does the set-up
+ * and can serve as that first call.  Later calls on the same context read
+ * the cached address and load nothing.
+ *
+ * Device-side status: as for gptq_quantize_layer, a failure inside the
+ * kernels is raised in a status word, here at the start of the static
+ * scratch; gptq_quantize_layer_noalloc_status(stream) reads it back.
  *
  * Zero state: no byte of the scratch has to start at zero.  Each call clears
  * the scratch's 256-byte status header itself, on stream, before its first
@@ -343,6 +378,16 @@ gptq_status_t gptq_quantize_layer_noalloc(const void* W, gptq_dtype_t wt,
                                           float* scales, int32_t* zeros,
                                           int32_t* g_idx, float* loss,
                                           void* stream);
+
+/*
+ * gptq_workspace_status for gptq_quantize_layer_noalloc: waits for stream
+ * and returns the device-side status of the last noalloc call on the
+ * current device (GPTQ_OK or GPTQ_ERR_TIMEOUT), read from the status word at
+ * the start of the static scratch.  Like that call, it has no counterpart in
+ * the GPTQ paper.  On a device with no earlier noalloc call it performs the
+ * set-up and returns GPTQ_OK.
+ */
+gptq_status_t gptq_quantize_layer_noalloc_status(void* stream);
 
 #ifdef __cplusplus
 }

@@ -24,6 +24,7 @@ __all__ = [
     "gptq_abi_version", "gptq_last_error", "gptq_kernel_launches", "gptq_validate_config",
     "gptq_workspace_bytes", "gptq_hessian_accumulate", "gptq_prepare_hinv",
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "GPTQ_STATIC_SCRATCH_BYTES",
+    "gptq_workspace_status", "gptq_quantize_layer_noalloc_status",
     "gptq_dequantize_layer", "gptq_export_checkpoint", "gptq_selftest_wait_timeout",
     "solve_layer", "solve_block", "export_checkpoint", "STATUS_NAMES",
 ]
@@ -74,6 +75,10 @@ lib.gptq_quantize_layer.restype = ctypes.c_int
 lib.gptq_quantize_layer_noalloc.argtypes = [_p, ctypes.c_int, _i64, _i64, _i64, _p, _p, _p,
                                             ctypes.POINTER(_Config), _p, _p, _p, _p, _p, _p, _p]
 lib.gptq_quantize_layer_noalloc.restype = ctypes.c_int
+lib.gptq_workspace_status.argtypes = [_p, ctypes.c_size_t, _p]
+lib.gptq_workspace_status.restype = ctypes.c_int
+lib.gptq_quantize_layer_noalloc_status.argtypes = [_p]
+lib.gptq_quantize_layer_noalloc_status.restype = ctypes.c_int
 
 lib.gptq_dequantize_layer.argtypes = [_p, _p, _p, _p, _i64, _i64, ctypes.c_int, ctypes.c_int, _p,
                                       ctypes.c_int, _i64, _p]
@@ -211,6 +216,18 @@ def gptq_quantize_layer_noalloc(W, U, perm, dead, cfg, scales, zeros, g_idx, cod
                                            _ptr(g_idx), _ptr(loss), _stream(stream)))
 
 
+def gptq_workspace_status(ws, stream=None) -> None:
+    """Wait for the stream and raise GptqError if the last prepare or
+    quantize call on workspace ``ws`` raised a device-side status (a bounded
+    wait that gave up, NaN/Inf in S, a non-positive pivot)."""
+    _check(lib.gptq_workspace_status(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def gptq_quantize_layer_noalloc_status(stream=None) -> None:
+    """The same for the last gptq_quantize_layer_noalloc call on this device."""
+    _check(lib.gptq_quantize_layer_noalloc_status(_stream(stream)))
+
+
 def gptq_dequantize_layer(qweight, scales, zeros, g_idx, bits, Wq, stream=None) -> None:
     """Wq (out x in; f16, bf16 or f32) <- scales * (code - zeros) from the
     packed codes gptq_quantize_layer wrote."""
@@ -288,7 +305,7 @@ def export_checkpoint(res, bits: int, zero_offset: int = 1, stream=None):
     return dict(qweight=qweight_t, qzeros=qzeros, scales=scales_h, g_idx=res["g_idx"])
 
 
-def solve_block(layers, activations, cfg=None, streams=True):
+def solve_block(layers, activations=None, cfg=None, streams=True, hessians=None):
     """Quantize the linear layers of one decoder block.
 
     layers: list of (name, W, site) with W an (out x in) device tensor and
@@ -296,62 +313,82 @@ def solve_block(layers, activations, cfg=None, streams=True):
       same activations, e.g. q/k/v or gate/up, share one site).
     activations: dict site -> X (in x tokens device tensor) or an iterable of
       such token batches.
+    hessians: optional dict site -> (S, n), an accumulated S (in x in fp32
+      device tensor, upper triangle) and its token count, used instead of
+      accumulating from activations for that site.
 
     For each site the Hessian is accumulated and prepared (U, perm, dead)
     once; every layer of the site is then quantized against that shared U.
-    With ``streams``, the layers of a site are quantized concurrently on
-    separate streams, so that latency-bound sweeps of different layers fill
-    the GPU together; a site's Hessian starts after the previous site's
-    layers, since its persistent kernel wants every SM.  Returns {name: dict(...)} as solve_layer does, plus
-    {"site:" + site: dict(S, n, U, perm, dead)}; synchronises the device.
+    The Hessians of all sites run first, back to back on the caller's stream
+    (the Hessian kernel is persistent and wants every SM).  Each site's
+    prepare follows on that stream, and with ``streams`` the layers of a site
+    are then quantized concurrently on side streams, which overlap the
+    following sites' prepares.  Every workspace and output allocated for a
+    side stream is recorded on it, so its memory is not reused before that
+    stream's work is done.  Returns {name: dict(...)} as solve_layer does,
+    plus {"site:" + site: dict(S, n, U, perm, dead)}; synchronises the device.
     """
     import torch
     cfg = GptqConfig.of(cfg or GptqConfig())
+    hessians = hessians or {}
     sites = {}
     for name, W, site in layers:
         sites.setdefault(site, []).append((name, W))
     dev = layers[0][1].device
-    cur = torch.cuda.current_stream(dev)
+    main = torch.cuda.current_stream(dev)
     results = {}
-    pending = []
+    # 1. the Hessians, one site after another on the caller's stream
+    acc = {}
     for site, members in sites.items():
-        s_site = torch.cuda.Stream(dev) if streams else cur
-        s_site.wait_stream(cur)
-        # the Hessian kernel is persistent (one resident CTA per SM): start it
-        # once the previous site's layers are done, not beside them
-        for s_prev, _ in pending:
-            s_site.wait_stream(s_prev)
         in_ = members[0][1].shape[1]
-        with torch.cuda.stream(s_site):
-            S = torch.zeros((in_, in_), dtype=torch.float32, device=dev)
-            n = 0
-            X = activations[site]
-            for Xb in ([X] if torch.is_tensor(X) else X):
-                n = gptq_hessian_accumulate(S, Xb, n, s_site)
-            ws = torch.empty(gptq_workspace_bytes(0, in_, cfg), dtype=torch.uint8, device=dev)
-            U = torch.empty((in_, in_), dtype=torch.float32, device=dev)
-            perm = torch.empty(in_, dtype=torch.int32, device=dev)
-            dead = torch.empty(in_, dtype=torch.uint8, device=dev)
-        gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, s_site)
+        if site in hessians:
+            acc[site] = hessians[site]
+            continue
+        S = torch.zeros((in_, in_), dtype=torch.float32, device=dev)
+        n = 0
+        X = activations[site]
+        for Xb in ([X] if torch.is_tensor(X) else X):
+            n = gptq_hessian_accumulate(S, Xb, n, main)
+        acc[site] = (S, n)
+    # 2. per site: prepare on the caller's stream, then its layers
+    side = []
+    for site, members in sites.items():
+        S, n = acc[site]
+        in_ = members[0][1].shape[1]
+        ws = torch.empty(gptq_workspace_bytes(0, in_, cfg), dtype=torch.uint8, device=dev)
+        U = torch.empty((in_, in_), dtype=torch.float32, device=dev)
+        perm = torch.empty(in_, dtype=torch.int32, device=dev)
+        dead = torch.empty(in_, dtype=torch.uint8, device=dev)
+        gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws, main)
+        del ws
         results["site:" + site] = dict(S=S, n=n, U=U, perm=perm, dead=dead)
+        ng = 1 if cfg.group_size == -1 else in_ // cfg.group_size
         for name, W in members:
-            s_layer = torch.cuda.Stream(dev) if streams else s_site
-            s_layer.wait_stream(s_site)
+            s_layer = torch.cuda.Stream(dev) if streams else main
+            s_layer.wait_stream(main)
             out = W.shape[0]
-            ng = 1 if cfg.group_size == -1 else in_ // cfg.group_size
-            with torch.cuda.stream(s_layer):
-                wsq = torch.empty(gptq_workspace_bytes(out, in_, cfg), dtype=torch.uint8, device=dev)
-                r = dict(scales=torch.empty((out, ng), dtype=torch.float32, device=dev),
-                         zeros=torch.empty((out, ng), dtype=torch.int32, device=dev),
-                         g_idx=torch.empty(in_, dtype=torch.int32, device=dev),
-                         loss=torch.empty(out, dtype=torch.float32, device=dev),
-                         codes=torch.empty((out, in_), dtype=torch.int32, device=dev),
-                         qweight=(torch.empty((out, in_ * cfg.bits // 32), dtype=torch.int32, device=dev)
-                                  if (in_ * cfg.bits) % 32 == 0 else None))
+            wsq = torch.empty(gptq_workspace_bytes(out, in_, cfg), dtype=torch.uint8, device=dev)
+            r = dict(scales=torch.empty((out, ng), dtype=torch.float32, device=dev),
+                     zeros=torch.empty((out, ng), dtype=torch.int32, device=dev),
+                     g_idx=torch.empty(in_, dtype=torch.int32, device=dev),
+                     loss=torch.empty(out, dtype=torch.float32, device=dev),
+                     codes=torch.empty((out, in_), dtype=torch.int32, device=dev),
+                     qweight=(torch.empty((out, in_ * cfg.bits // 32), dtype=torch.int32, device=dev)
+                              if (in_ * cfg.bits) % 32 == 0 else None))
+            if s_layer is not main:
+                for t in [wsq, W, U, perm, dead] + [v for v in r.values() if v is not None]:
+                    t.record_stream(s_layer)
             gptq_quantize_layer(W, U, perm, dead, cfg, r["scales"], r["zeros"], r["g_idx"], wsq,
                                 codes=r["codes"], qweight=r["qweight"], loss=r["loss"], stream=s_layer)
-            r.update(perm=perm, dead=dead, U=U, n=n)
+            r.update(perm=perm, dead=dead, U=U, n=n, ws=wsq, stream=s_layer)
             results[name] = r
-            pending.append((s_layer, wsq))
+            side.append(s_layer)
+    for s_layer in side:
+        main.wait_stream(s_layer)
     torch.cuda.synchronize(dev)
+    for name, _, _ in layers:
+        r = results[name]
+        ws = r.pop("ws")
+        s_layer = r.pop("stream")
+        gptq_workspace_status(ws, s_layer)
     return results

@@ -33,10 +33,28 @@ gptq_status_t fail(gptq_status_t s, const char* fmt, ...) {
 
 void clear_error() { g_last_error.clear(); }
 
+gptq_status_t read_device_status(const PrepHeader* hdr, cudaStream_t st) {
+  uint32_t status = 0;
+  CUDA_TRY(cudaMemcpyAsync(&status, &hdr->status, sizeof(status), cudaMemcpyDeviceToHost, st));
+  CUDA_TRY(cudaStreamSynchronize(st));
+  if (status & ST_TIMEOUT) return fail(GPTQ_ERR_TIMEOUT, "a bounded device-side wait gave up");
+  if (status & ST_NONFINITE) return fail(GPTQ_ERR_NONFINITE, "S holds NaN or Inf");
+  if (status & ST_NOT_PD) return fail(GPTQ_ERR_NOT_PD, "the damped Hessian is not positive definite");
+  return GPTQ_OK;
+}
+
 namespace {
 std::atomic<uint64_t> g_launches{0};
 }
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+bool force_simt() {
+  static const bool on = [] {
+    const char* v = getenv("GPTQ_FORCE_SIMT");
+    return v && atoi(v) != 0;
+  }();
+  return on;
+}
 
 cudaError_t ensure_smem_limit(const void* func, int bytes) {
   static std::mutex mu;
@@ -53,20 +71,22 @@ cudaError_t ensure_smem_limit(const void* func, int bytes) {
 }
 
 const DeviceInfo& device_info() {
-  static DeviceInfo infos[64];
+  // one entry per device ordinal, created on first use; entries are never
+  // moved or freed, so the returned reference stays valid
+  static std::map<int, DeviceInfo> infos;
   static std::mutex mu;
-  int d = 0;
-  if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) d = 0;
+  static const DeviceInfo none;
+  int d = -1;
+  if (cudaGetDevice(&d) != cudaSuccess || d < 0) return none;
   std::lock_guard<std::mutex> lock(mu);
   DeviceInfo& di = infos[d];
   if (di.id != d) {
     cudaDeviceProp prop;
-    if (cudaGetDeviceProperties(&prop, d) == cudaSuccess) {
-      di.sms = prop.multiProcessorCount;
-      di.major = prop.major;
-      di.minor = prop.minor;
-      di.id = d;
-    }
+    if (cudaGetDeviceProperties(&prop, d) != cudaSuccess) return none;
+    di.sms = prop.multiProcessorCount;
+    di.major = prop.major;
+    di.minor = prop.minor;
+    di.id = d;
   }
   return di;
 }
@@ -87,9 +107,8 @@ gptq_status_t hessian_accumulate(float* S, int64_t in, const void* X, gptq_dtype
   g.beta = 1.f;
   g.mask = 1;
   g.tri = 1;
-  const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
   cudaError_t e;
-  if (xt != GPTQ_F32 && !force_simt && tc_gemm_supported(g))
+  if (xt != GPTQ_F32 && !force_simt() && tc_gemm_supported(g))
     e = tc_gemm(g, st, dev.sms);
   else
     e = simt_gemm(g, st);
@@ -223,6 +242,18 @@ gptq_status_t gptq_quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, i
   if (s != GPTQ_OK) return s;
   return quantize_layer(W, wt, out, in, ldw, U, perm, dead, cfg, codes, qweight, scales, zeros, g_idx, loss, ws,
                         ws_bytes, (cudaStream_t)stream);
+}
+
+gptq_status_t gptq_workspace_status(const void* ws, size_t ws_bytes, void* stream) {
+  clear_error();
+  if (!ws) return fail(GPTQ_ERR_WORKSPACE, "workspace pointer is NULL");
+  if (((uintptr_t)ws & 255u) != 0) return fail(GPTQ_ERR_WORKSPACE, "workspace is not 256-byte aligned");
+  if (ws_bytes < (size_t)kHeaderBytes)
+    return fail(GPTQ_ERR_WORKSPACE, "workspace too small: %zu bytes given, %lld needed", ws_bytes,
+                (long long)kHeaderBytes);
+  gptq_status_t s = check_device();
+  if (s != GPTQ_OK) return s;
+  return read_device_status((const PrepHeader*)ws, (cudaStream_t)stream);
 }
 
 gptq_status_t gptq_dequantize_layer(const uint32_t* qweight, const float* scales, const int32_t* zeros,

@@ -61,6 +61,11 @@ cudaError_t ensure_smem_limit(const void* func, int bytes);
 cudaError_t tc_gemm(const GemmArgs& a, cudaStream_t stream, int num_sms);
 cudaError_t simt_gemm(const GemmArgs& a, cudaStream_t stream);
 
+// Make the driver load the GEMM kernels on the current device now (as their
+// first launch would); cudaFuncGetAttributes on each.
+cudaError_t preload_gemm_kernels();
+cudaError_t preload_simt_kernels();
+
 // Whether the tensor-core path can take this product (alignment of bases
 // and strides for TMA, K extents compatible with the k-tile).
 bool tc_gemm_supported(const GemmArgs& a);

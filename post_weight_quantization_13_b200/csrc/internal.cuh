@@ -11,8 +11,9 @@ namespace gptq {
 // First 256 bytes of every workspace.
 struct PrepHeader {
   uint32_t status;  // ST_* flags OR-ed by kernels
-  float lambda;     // damping added to the diagonal
-  uint32_t pad[62];
+  uint32_t pad0;
+  double lambda;    // damping added to the diagonal
+  uint32_t pad[60];
 };
 constexpr int64_t kHeaderBytes = 256;
 static_assert(sizeof(PrepHeader) == kHeaderBytes, "header size");
@@ -30,9 +31,19 @@ const DeviceInfo& device_info();
 // Process-wide count of kernels this library has launched (diagnostic).
 void note_launch();
 
+// True when the environment variable GPTQ_FORCE_SIMT was set to a non-zero
+// integer at the library's first call: every GEMM then runs on the CUDA-core
+// kernel (a cross-check of the tensor-core path).  Read once per process.
+bool force_simt();
+
 // Record a message for gptq_last_error() and return s.
 gptq_status_t fail(gptq_status_t s, const char* fmt, ...);
 void clear_error();
+
+// Wait for st, read the status word of the workspace header hdr (device
+// memory) and map its flags to a status code: GPTQ_ERR_TIMEOUT before
+// GPTQ_ERR_NONFINITE before GPTQ_ERR_NOT_PD, GPTQ_OK when none is set.
+gptq_status_t read_device_status(const PrepHeader* hdr, cudaStream_t st);
 
 #define CUDA_TRY(x)                                                                           \
   do {                                                                                        \
@@ -58,6 +69,10 @@ gptq_status_t export_checkpoint(const uint32_t* qweight, const float* scales, co
                                 uint32_t* qzeros, uint16_t* scales_h, cudaStream_t st);
 gptq_status_t hessian_accumulate(float* S, int64_t in, const void* X, gptq_dtype_t xt, int64_t tokens, int64_t ldx,
                                  cudaStream_t st);
+
+// Make the driver load every kernel gptq_quantize_layer can launch on the
+// current device now, instead of at their first launch.
+cudaError_t preload_quantize_kernels();
 
 // Lazy-batch width actually used for a configuration (multiple of 128,
 // compatible with group_size, at most 1024).

@@ -1,10 +1,13 @@
 // gptq_quantize_layer_noalloc: the quantize sweep on a fixed device scratch,
 // for callers that cannot allocate device memory.  The scratch is a static
-// device array; its address is looked up once per device and cached.  The
-// work itself is gptq_quantize_layer's, called with that scratch as the
-// workspace.
+// device array.  Its address is looked up once per device context (set-up)
+// and cached together with the context's id, so a context created after a
+// device reset gets its own look-up.  The work itself is
+// gptq_quantize_layer's, called with that scratch as the workspace.
+#include <map>
 #include <mutex>
 
+#include "gemm.cuh"
 #include "internal.cuh"
 
 namespace gptq {
@@ -12,28 +15,65 @@ namespace {
 
 __device__ __align__(256) unsigned char g_static_scratch[GPTQ_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxScratchDevices = 64;
-void* g_scratch_addr[kMaxScratchDevices];
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+CtxGetIdFn ctx_get_id_fn() {
+  static CtxGetIdFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (CtxGetIdFn)p;
+  });
+  return fn;
+}
+
+struct ScratchEntry {
+  unsigned long long ctx_id = 0;
+  void* addr = nullptr;
+};
+std::map<int, ScratchEntry> g_scratch;  // device ordinal -> set-up of its current context
 std::mutex g_scratch_mu;
 
-// Address of this device's copy of g_static_scratch (the current device's).
+// Id of the calling thread's current context (false if there is none yet).
+bool current_ctx_id(unsigned long long* id) {
+  CtxGetIdFn fn = ctx_get_id_fn();
+  return fn && fn(nullptr, id) == CUDA_SUCCESS;
+}
+
+// Address of the current device's copy of g_static_scratch.  Set-up, once per
+// device context, with that device current: cudaGetSymbolAddress (which
+// creates the primary context if this thread has none yet), then every kernel
+// the quantize call can launch is loaded on the device, so that later calls
+// neither resolve symbols nor load device code.
 gptq_status_t static_scratch(void** addr) {
   int d = -1;
   cudaError_t e = cudaGetDevice(&d);
   if (e != cudaSuccess) return fail(GPTQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (d < 0 || d >= kMaxScratchDevices)
-    return fail(GPTQ_ERR_UNSUPPORTED, "device %d: the static scratch is kept for devices 0..%d only", d,
-                kMaxScratchDevices - 1);
+  unsigned long long id = 0;
+  const bool have_ctx = current_ctx_id(&id);
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_addr[d]) {
-    void* ptr = nullptr;
-    e = cudaGetSymbolAddress((void**)&ptr, g_static_scratch);
-    if (e != cudaSuccess)
-      return fail(GPTQ_ERR_CUDA, "cudaGetSymbolAddress of the static scratch on device %d: %s", d,
-                  cudaGetErrorString(e));
-    g_scratch_addr[d] = ptr;
+  ScratchEntry& ent = g_scratch[d];
+  if (have_ctx && ent.addr && ent.ctx_id == id) {
+    *addr = ent.addr;
+    return GPTQ_OK;
   }
-  *addr = g_scratch_addr[d];
+  void* ptr = nullptr;
+  e = cudaGetSymbolAddress((void**)&ptr, g_static_scratch);
+  if (e != cudaSuccess)
+    return fail(GPTQ_ERR_CUDA, "cudaGetSymbolAddress of the static scratch on device %d: %s", d,
+                cudaGetErrorString(e));
+  if (!current_ctx_id(&id)) return fail(GPTQ_ERR_CUDA, "no current CUDA context on device %d", d);
+  e = preload_quantize_kernels();
+  if (e == cudaSuccess) e = preload_gemm_kernels();
+  if (e == cudaSuccess) e = preload_simt_kernels();
+  if (e != cudaSuccess)
+    return fail(GPTQ_ERR_CUDA, "loading the quantize kernels on device %d: %s", d, cudaGetErrorString(e));
+  ent.ctx_id = id;
+  ent.addr = ptr;
+  *addr = ptr;
   return GPTQ_OK;
 }
 
@@ -62,4 +102,13 @@ extern "C" gptq_status_t gptq_quantize_layer_noalloc(const void* W, gptq_dtype_t
   if (s != GPTQ_OK) return s;
   return gptq_quantize_layer(W, wt, out, in, ldw, U, perm, dead, cfg, codes, qweight, scales, zeros, g_idx, loss,
                              ws, GPTQ_STATIC_SCRATCH_BYTES, stream);
+}
+
+extern "C" gptq_status_t gptq_quantize_layer_noalloc_status(void* stream) {
+  using namespace gptq;
+  clear_error();
+  void* ws = nullptr;
+  gptq_status_t s = static_scratch(&ws);
+  if (s != GPTQ_OK) return s;
+  return gptq_workspace_status(ws, GPTQ_STATIC_SCRATCH_BYTES, stream);
 }

@@ -42,22 +42,23 @@ constexpr int NB = 128;
 constexpr int64_t kSuperBlock = 4096;
 
 // ------------------------------------------------------------------ diag
-// One CTA: hd[i] = fixed diagonal of H (dead -> 1), dead flags, and
+// One CTA: hd[i] = fixed diagonal of H in double, hd = c * S_ii with
+// c = 2 / n rounded to double (the same two roundings as forming H = (2/n) S
+// in float64), dead channels (S_ii == 0) get 1; dead flags; and
 // lambda = damp * mean(hd).  Deterministic tree reduction in double.
-__global__ void __launch_bounds__(1024) diag_kernel(const float* __restrict__ S, int64_t in, float scale,
-                                                    float damp, float* __restrict__ hd, uint8_t* __restrict__ dead,
+__global__ void __launch_bounds__(1024) diag_kernel(const float* __restrict__ S, int64_t in, double c,
+                                                    float damp, double* __restrict__ hd, uint8_t* __restrict__ dead,
                                                     PrepHeader* hdr) {
   __shared__ double red[1024];
   double acc = 0.0;
   for (int64_t i = threadIdx.x; i < in; i += blockDim.x) {
     const float s = S[i * in + i];
     if (!isfinite(s)) raise_status(&hdr->status, ST_NONFINITE);
-    const float h = s * scale;
-    const bool d = (h == 0.f);
-    const float hf = d ? 1.f : h;
-    hd[i] = hf;
+    const bool d = (s == 0.f);
+    const double h = d ? 1.0 : __dmul_rn(c, (double)s);
+    hd[i] = h;
     dead[i] = d ? 1 : 0;
-    acc += (double)hf;
+    acc += h;
   }
   red[threadIdx.x] = acc;
   __syncthreads();
@@ -65,29 +66,31 @@ __global__ void __launch_bounds__(1024) diag_kernel(const float* __restrict__ S,
     if (threadIdx.x < s) red[threadIdx.x] += red[threadIdx.x + s];
     __syncthreads();
   }
-  if (threadIdx.x == 0) hdr->lambda = (float)((double)damp * (red[0] / (double)in));
+  if (threadIdx.x == 0) hdr->lambda = (double)damp * (red[0] / (double)in);
 }
 
 // ------------------------------------------------------------------ act order
 // perm[rank(i)] = i, rank = #{j : hd_j > hd_i} + #{j < i : hd_j == hd_i}:
-// the stable descending order.
-__global__ void __launch_bounds__(256) rank_kernel(const float* __restrict__ hd, int64_t in, int desc_act,
+// the stable descending order of the diagonal, compared in double on the
+// values diag_kernel formed (so two channels tie exactly when their H_ii
+// tie in float64).
+__global__ void __launch_bounds__(256) rank_kernel(const double* __restrict__ hd, int64_t in, int desc_act,
                                                    int32_t* __restrict__ perm) {
-  __shared__ float tile[1024];
+  __shared__ double tile[1024];
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (!desc_act) {
     if (i < in) perm[i] = (int32_t)i;
     return;
   }
-  const float key = i < in ? hd[i] : 0.f;
+  const double key = i < in ? hd[i] : 0.0;
   int64_t rank = 0;
   for (int64_t j0 = 0; j0 < in; j0 += 1024) {
     __syncthreads();
-    for (int t = threadIdx.x; t < 1024; t += blockDim.x) tile[t] = (j0 + t < in) ? hd[j0 + t] : 0.f;
+    for (int t = threadIdx.x; t < 1024; t += blockDim.x) tile[t] = (j0 + t < in) ? hd[j0 + t] : 0.0;
     __syncthreads();
     const int m = (int)((in - j0) < 1024 ? (in - j0) : 1024);
     for (int t = 0; t < m; ++t) {
-      const float v = tile[t];
+      const double v = tile[t];
       rank += (v > key) || (v == key && j0 + t < i);
     }
   }
@@ -103,9 +106,9 @@ __global__ void __launch_bounds__(256) rank_kernel(const float* __restrict__ hd,
 // coalesce; each block takes whole rows, four columns per thread.
 __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S, int64_t in, int64_t np_,
                                                      float scale, const int32_t* __restrict__ perm,
-                                                     const uint8_t* __restrict__ dead, PrepHeader* hdr,
+                                                     const double* __restrict__ hd, PrepHeader* hdr,
                                                      float* __restrict__ R) {
-  const float lam = hdr->lambda;
+  const double lam = hdr->lambda;
   // in <= 32768, so in * in fits 32-bit index arithmetic
   const int n = (int)in, np = (int)np_;
   for (int a = blockIdx.x; a < np; a += gridDim.x) {
@@ -121,8 +124,9 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
           const unsigned lo = (unsigned)min(i, j), hi = (unsigned)max(i, j);
           const float sv = __ldg(S + (lo * (unsigned)n + hi));
           if (!isfinite(sv)) raise_status(&hdr->status, ST_NONFINITE);
-          x = sv * scale;
-          if (i == j) x = (dead[i] ? 1.f : x) + lam;
+          // the diagonal from diag_kernel's fixed values (dead channels
+          // there hold 1), damped in double and rounded once
+          x = (i == j) ? (float)(__ldg(hd + i) + lam) : sv * scale;
         } else if (a == b) {
           x = 1.f;
         }
@@ -656,8 +660,8 @@ __global__ void __launch_bounds__(256) write_u_kernel(const float* __restrict__ 
   }
 }
 
-cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
-  if (!force_simt && tc_gemm_supported(g)) return tc_gemm(g, st, sms);
+cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms) {
+  if (!force_simt() && tc_gemm_supported(g)) return tc_gemm(g, st, sms);
   return simt_gemm(g, st);
 }
 
@@ -666,7 +670,7 @@ cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
 size_t prepare_ws_bytes(int64_t in) {
   const int64_t np_ = round_up(in, NB);
   size_t b = kHeaderBytes;
-  b += round_up((int64_t)sizeof(float) * in, 256);               // hd
+  b += round_up((int64_t)sizeof(double) * in, 256);              // hd
   b += 9 * round_up((int64_t)sizeof(float) * np_ * np_, 256);    // R; L, M, Mt, X^T (hi, lo)
   b += round_up((int64_t)sizeof(float) * np_ * FB, 256);         // diagonal blocks of M
   b += round_up((int64_t)sizeof(int) * (np_ / FB + 4), 256);      // barrier and panel flags
@@ -682,8 +686,8 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   uint8_t* p = (uint8_t*)ws;
   PrepHeader* hdr = (PrepHeader*)p;
   p += kHeaderBytes;
-  float* hd = (float*)p;
-  p += round_up((int64_t)sizeof(float) * in, 256);
+  double* hd = (double*)p;
+  p += round_up((int64_t)sizeof(double) * in, 256);
   const size_t mat = round_up((int64_t)sizeof(float) * np_ * np_, 256);
   float* R = (float*)p; p += mat;      // reversed, damped Hessian; Schur complements in place
   float* Lh = (float*)p; p += mat;     // L's panels (split), for the inverse
@@ -704,12 +708,12 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     p += round_up((int64_t)sizeof(float) * (np_ - kSuperBlock) * kSuperBlock, 256);
     Pkl = (float*)p;
   }
-  const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
 
   CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
   CUDA_TRY(cudaMemsetAsync(Mh, 0, 4 * mat, st));  // M, Mt (hi, lo): strictly-off-triangle blocks stay 0
-  const float scale = (float)(2.0 / (double)n);
-  diag_kernel<<<1, 1024, 0, st>>>(S, in, scale, cfg->damp_percent, hd, dead, hdr);
+  const double c = 2.0 / (double)n;
+  const float scale = (float)c;
+  diag_kernel<<<1, 1024, 0, st>>>(S, in, c, cfg->damp_percent, hd, dead, hdr);
   note_launch();
   CUDA_TRY(cudaGetLastError());
   rank_kernel<<<(unsigned)((in + 255) / 256), 256, 0, st>>>(hd, in, cfg->desc_act, perm);
@@ -717,7 +721,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   CUDA_TRY(cudaGetLastError());
   {
     const unsigned grid = (unsigned)std::min<int64_t>(np_, (int64_t)dev.sms * 8);
-    gather_kernel<<<grid, 256, 0, st>>>(S, in, np_, scale, perm, dead, hdr, R);
+    gather_kernel<<<grid, 256, 0, st>>>(S, in, np_, scale, perm, hd, hdr, R);
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
@@ -772,7 +776,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
       a.bs_c_row = stride;
       a.bs_c_col = stride;
       a.status = &hdr->status;
-      CUDA_TRY(run_gemm(a, st, dev.sms, force_simt));
+      CUDA_TRY(run_gemm(a, st, dev.sms));
       // M21[r][c] = -sum_t M[o2+r][o2+t] X^T[o1+c][o2+t]
       GemmArgs b = a;
       b.P = {Mh, Ml, np_, np_, np_};
@@ -790,7 +794,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
       b.c_col0 = o1;
       b.alpha = -1.f;
       b.transpose = 0;
-      CUDA_TRY(run_gemm(b, st, dev.sms, force_simt));
+      CUDA_TRY(run_gemm(b, st, dev.sms));
       dim3 tg((unsigned)((s1 + 31) / 32), (unsigned)((s2 + 31) / 32), (unsigned)nb);
       transpose_blocks_kernel<<<tg, 256, 0, st>>>(Mh, Ml, Mth, Mtl, np_, o1, o2, s1, s2, stride);
       note_launch();
@@ -857,7 +861,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     pg.alpha = 1.f;
     pg.beta = 0.f;
     pg.status = &hdr->status;
-    CUDA_TRY(run_gemm(pg, st, dev.sms, force_simt));
+    CUDA_TRY(run_gemm(pg, st, dev.sms));
     GemmArgs tg;
     tg.op = OP_TF32X3;
     tg.P = {Lh, Ll, np_, np_, np_};
@@ -877,7 +881,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     tg.beta = 1.f;
     tg.mask = 2;
     tg.status = &hdr->status;
-    CUDA_TRY(run_gemm(tg, st, dev.sms, force_simt));
+    CUDA_TRY(run_gemm(tg, st, dev.sms));
   }
   if (supers.size() > 1) {
     gptq_status_t ms = merge(supers);
@@ -889,13 +893,7 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
-  uint32_t status = 0;
-  CUDA_TRY(cudaMemcpyAsync(&status, &hdr->status, sizeof(status), cudaMemcpyDeviceToHost, st));
-  CUDA_TRY(cudaStreamSynchronize(st));
-  if (status & ST_TIMEOUT) return fail(GPTQ_ERR_TIMEOUT, "a bounded device-side wait gave up");
-  if (status & ST_NONFINITE) return fail(GPTQ_ERR_NONFINITE, "S holds NaN or Inf");
-  if (status & ST_NOT_PD) return fail(GPTQ_ERR_NOT_PD, "the damped Hessian is not positive definite");
-  return GPTQ_OK;
+  return read_device_status(hdr, st);
 }
 
 }  // namespace gptq

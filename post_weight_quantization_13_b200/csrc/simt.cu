@@ -123,6 +123,17 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtParams sp) {
 
 }  // namespace
 
+cudaError_t preload_simt_kernels() {
+  const void* fns[] = {(const void*)simt_gemm_kernel<__half>, (const void*)simt_gemm_kernel<__nv_bfloat16>,
+                       (const void*)simt_gemm_kernel<float>};
+  for (const void* f : fns) {
+    cudaFuncAttributes attr;
+    const cudaError_t e = cudaFuncGetAttributes(&attr, f);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t simt_gemm(const GemmArgs& a, cudaStream_t st) {
   if (a.R <= 0 || a.Cn <= 0 || a.K <= 0 || a.batch <= 0) return cudaSuccess;
   SimtParams sp;

@@ -383,8 +383,8 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t* __restrict__ c
   }
 }
 
-cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms, bool force_simt) {
-  if (!force_simt && tc_gemm_supported(g)) return tc_gemm(g, st, sms);
+cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms) {
+  if (!force_simt() && tc_gemm_supported(g)) return tc_gemm(g, st, sms);
   return simt_gemm(g, st);
 }
 
@@ -412,6 +412,21 @@ cudaError_t launch_sweep(const SweepParams& sp, cudaStream_t st, bool pdl) {
 }
 
 }  // namespace
+
+cudaError_t preload_quantize_kernels() {
+  const void* fns[] = {
+      (const void*)sweep_kernel<8>,   (const void*)sweep_kernel<16>, (const void*)sweep_kernel<32>,
+      (const void*)sweep_kernel<64>,  (const void*)sweep_kernel<128>, (const void*)pack_diag_kernel,
+      (const void*)gather_w_kernel<__half>, (const void*)gather_w_kernel<__nv_bfloat16>,
+      (const void*)gather_w_kernel<float>,  (const void*)split_u_kernel, (const void*)invperm_kernel,
+      (const void*)pack_kernel};
+  for (const void* f : fns) {
+    cudaFuncAttributes attr;
+    const cudaError_t e = cudaFuncGetAttributes(&attr, f);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 int64_t outer_block(const gptq_config_t* cfg) {
   const int64_t gs = cfg->group_size;
@@ -460,7 +475,6 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
   float* Ud = (float*)p;
   p += round_up(4 * (int64_t)kDiagBlockFloats * (np_ / BW), 256);
   int32_t* inv = (int32_t*)p;
-  const bool force_simt = getenv("GPTQ_FORCE_SIMT") && atoi(getenv("GPTQ_FORCE_SIMT")) != 0;
 
   CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
   if (loss) CUDA_TRY(cudaMemsetAsync(loss, 0, sizeof(float) * out, st));
@@ -574,7 +588,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
         g.alpha = -1.f;
         g.beta = 1.f;
         g.status = &hdr->status;
-        CUDA_TRY(run_gemm(g, st, dev.sms, force_simt));
+        CUDA_TRY(run_gemm(g, st, dev.sms));
       }
     }
     // outer lazy update: every later column
@@ -599,7 +613,7 @@ gptq_status_t quantize_layer(const void* W, gptq_dtype_t wt, int64_t out, int64_
       g.alpha = -1.f;
       g.beta = 1.f;
       g.status = &hdr->status;
-      CUDA_TRY(run_gemm(g, st, dev.sms, force_simt));
+      CUDA_TRY(run_gemm(g, st, dev.sms));
     }
   }
   invperm_kernel<<<(unsigned)((in + 255) / 256), 256, 0, st>>>(perm, in, gs, inv, g_idx);

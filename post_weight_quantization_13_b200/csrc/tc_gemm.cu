@@ -688,6 +688,17 @@ cudaError_t launch(const TmaMaps& maps, const KParams& kp, int grid, size_t smem
 
 }  // namespace
 
+cudaError_t preload_gemm_kernels() {
+  const void* fns[] = {(const void*)tc_gemm_kernel<OP_F16>, (const void*)tc_gemm_kernel<OP_BF16>,
+                       (const void*)tc_gemm_kernel<OP_TF32X3>};
+  for (const void* f : fns) {
+    cudaFuncAttributes attr;
+    const cudaError_t e = cudaFuncGetAttributes(&attr, f);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 bool tc_gemm_supported(const GemmArgs& a) {
   const int es = esize_of(a.op);
   const Operand* ops[2] = {&a.P, &a.Q};

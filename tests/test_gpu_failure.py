@@ -1,6 +1,8 @@
 """Failure handling without a GPU fault: the bounded waits every kernel of
 the library uses give up after their limit and report GPTQ_ERR_TIMEOUT
 through a status word; the context stays usable afterwards."""
+import ctypes
+
 import numpy as np
 import pytest
 
@@ -41,3 +43,45 @@ def test_bounded_wait_times_out_and_the_device_stays_usable(lib):
     assert np.array_equal(host(r["perm"]), ref["perm"])
     rate, _ = code_report(host(r["codes"]), ref["codes"])
     assert rate >= 0.999, rate
+
+
+def test_workspace_status_rejects_bad_workspaces_on_the_host(g):
+    GPTQ_ERR_WORKSPACE = 4
+    assert g.lib.gptq_workspace_status(None, 1 << 20, None) == GPTQ_ERR_WORKSPACE
+    assert g.lib.gptq_workspace_status(ctypes.c_void_p(256 + 16), 1 << 20, None) == GPTQ_ERR_WORKSPACE
+    assert g.lib.gptq_workspace_status(ctypes.c_void_p(1 << 20), 128, None) == GPTQ_ERR_WORKSPACE
+
+
+@pytest.mark.gpu
+def test_quantize_status_reaches_the_caller(lib):
+    """gptq_quantize_layer returns before its kernels run; a device-side
+    failure reaches the caller through the workspace's status word.  A clean
+    quantize reads back GPTQ_OK; a status word holding the timeout flag (the
+    flag the bounded waits raise, set here by the test) reads back
+    GPTQ_ERR_TIMEOUT; the next quantize clears it again."""
+    import torch
+    W, X = gen.small_case(42, 48, 256, 512, w_dtype="float32", x_dtype="float16")
+    cfg = lib.GptqConfig(bits=4, group_size=64, desc_act=True)
+    S = torch.zeros((256, 256), dtype=torch.float32, device="cuda")
+    n = lib.gptq_hessian_accumulate(S, dev(X, torch.float16), 0)
+    ws = torch.empty(lib.gptq_workspace_bytes(48, 256, cfg), dtype=torch.uint8, device="cuda")
+    U = torch.empty((256, 256), dtype=torch.float32, device="cuda")
+    perm = torch.empty(256, dtype=torch.int32, device="cuda")
+    dead = torch.empty(256, dtype=torch.uint8, device="cuda")
+    lib.gptq_prepare_hinv(S, n, cfg, U, perm, dead, ws)
+    scales = torch.empty((48, 4), dtype=torch.float32, device="cuda")
+    zeros = torch.empty((48, 4), dtype=torch.int32, device="cuda")
+    g_idx = torch.empty(256, dtype=torch.int32, device="cuda")
+    Wd = dev(W)
+
+    def quantize():
+        lib.gptq_quantize_layer(Wd, U, perm, dead, cfg, scales, zeros, g_idx, ws)
+
+    quantize()
+    lib.gptq_workspace_status(ws)
+    ws[:4].view(torch.int32).fill_(4)           # the timeout flag
+    with pytest.raises(lib.GptqError) as e:
+        lib.gptq_workspace_status(ws)
+    assert e.value.status == GPTQ_ERR_TIMEOUT
+    quantize()
+    lib.gptq_workspace_status(ws)

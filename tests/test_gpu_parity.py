@@ -255,19 +255,101 @@ def test_block_size_variants_agree(lib):
         assert (r == res[0]).mean() >= 0.999
 
 
-def test_tensor_core_and_cuda_core_paths_agree(lib):
+_SIMT_CHILD = """
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, sys.argv[1])
+import post_weight_quantization_13_b200 as g
+S32 = np.load(sys.argv[2])
+n, in_ = int(sys.argv[3]), S32.shape[0]
+cfg = g.GptqConfig(bits=4, group_size=128, desc_act=True)
+ws = torch.empty(g.gptq_workspace_bytes(0, in_, cfg), dtype=torch.uint8, device="cuda")
+U = torch.empty((in_, in_), dtype=torch.float32, device="cuda")
+perm = torch.empty(in_, dtype=torch.int32, device="cuda")
+dead = torch.empty(in_, dtype=torch.uint8, device="cuda")
+g.gptq_prepare_hinv(torch.from_numpy(S32).cuda(), n, cfg, U, perm, dead, ws)
+np.save(sys.argv[4], U.cpu().numpy().T)
+np.save(sys.argv[5], perm.cpu().numpy())
+"""
+
+
+def test_tensor_core_and_cuda_core_paths_agree(lib, tmp_path):
+    """The prepare's GEMMs on the tensor cores against the same GEMMs on the
+    CUDA cores.  The library reads GPTQ_FORCE_SIMT once per process, so the
+    CUDA-core run happens in a child process started with it set."""
+    import subprocess
+    import sys
     S32, n = _prep_inputs(93, 640, 2000, "correlated")
-    W32, _ = gen.small_case(94, 96, 640, 8)
-    W_t, W64 = exact_values(W32, "float16")
     cfg = _cfg(lib, bits=4, group_size=128, desc_act=True)
     U1, p1, _ = _run_prepare(lib, S32, n, cfg)
-    os.environ["GPTQ_FORCE_SIMT"] = "1"
-    try:
-        U2, p2, _ = _run_prepare(lib, S32, n, cfg)
-    finally:
-        del os.environ["GPTQ_FORCE_SIMT"]
+    np.save(tmp_path / "S.npy", S32)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, GPTQ_FORCE_SIMT="1")
+    subprocess.run([sys.executable, "-c", _SIMT_CHILD, root, str(tmp_path / "S.npy"), str(n),
+                    str(tmp_path / "U.npy"), str(tmp_path / "p.npy")], env=env, check=True, timeout=300)
+    U2 = np.load(tmp_path / "U.npy")
+    p2 = np.load(tmp_path / "p.npy")
     assert np.array_equal(p1, p2)
     assert rel_fro(U1, U2) < 1e-5
+
+
+def test_act_order_exact_on_near_tie_diagonals(lib):
+    """Act-order ranks the diagonal the way the oracle does, on the same fp32
+    S: channels whose S_ii are one fp32 ulp apart stay in strict order (a
+    product with 2/n rounded to fp32 would merge a good share of such pairs
+    and fall back to index order), exact ties keep index order, and dead
+    channels (S_ii = 0, ranked as H_ii = 1) sit where H_ii = 1 puts them."""
+    in_, n = 512, 3
+    rng = np.random.default_rng(21)
+    base = rng.uniform(0.5, 3.0, in_ // 4).astype(np.float32)
+    d = np.empty(in_, np.float32)
+    d[0::4] = base
+    d[1::4] = np.nextafter(base, np.float32(np.inf))
+    d[2::4] = base
+    d[3::4] = np.nextafter(base, np.float32(0))
+    d[7] = np.float32(1.5)                      # H_ii = 2 * 1.5 / 3: ties with a dead channel's 1
+    dead_idx = np.array([3, 100, 257, 400])
+    d[dead_idx] = 0.0
+    off = np.triu(rng.uniform(-1e-3, 1e-3, (in_, in_)), 1).astype(np.float32)
+    S32 = np.diag(d) + off + off.T             # symmetric: the oracle reads both triangles
+    S32[dead_idx, :] = 0.0
+    S32[:, dead_idx] = 0.0
+    for damp in (0.01, 0.0):
+        cfg = _cfg(lib, desc_act=True, damp_percent=damp, group_size=-1)
+        U, perm, dead = _run_prepare(lib, S32, n, cfg)
+        ref = O.prepare(S32.astype(np.float64), n, damp, True)
+        assert np.array_equal(dead, ref["dead"])
+        assert np.array_equal(perm, ref["perm"])
+        assert rel_fro(U, ref["U"]) < 1e-4
+
+
+def test_group32_damp0005_prepare_and_quantize_at_4096(lib):
+    """The agent-skill page's configuration example with group_size 32 and
+    damp_percent 0.005, through prepare and quantize on a 4096-wide layer:
+    both sides get the same fp32 S, so perm, g_idx and codes compare
+    exactly."""
+    in_, out, tokens = 4096, 256, 8192
+    S32, n = _prep_inputs(77, in_, tokens, "correlated")
+    W32, _ = gen.small_case(78, out, in_, 8)
+    W_t, W64 = exact_values(W32, "float16")
+    cfg = _cfg(lib, bits=4, group_size=32, desc_act=True, damp_percent=0.005)
+    U, perm, dead = _run_prepare(lib, S32, n, cfg)
+    ref = O.gptq_layer(W64, S32.astype(np.float64), n, bits=4, group_size=32, sym=False,
+                       desc_act=True, damp_percent=0.005, block_size=128)
+    assert np.array_equal(perm, ref["perm"])
+    assert rel_fro(U, ref["U"]) < 1e-3
+    g = _run_quantize(lib, W_t.cuda(), np.ascontiguousarray(U.T), perm, dead, cfg)
+    rate, eq = code_report(g["codes"], ref["codes"])
+    assert rate >= 0.999, rate
+    assert np.array_equal(g["g_idx"], ref["g_idx"])
+    compare_groups(g["scales"], g["zeros"], ref["scales"], ref["zeros"], eq[:, ref["perm"]], 32)
+    assert np.array_equal(g["qweight"], O.pack_rows(g["codes"], 4))
+    deq = O.dequantize_layer(g["codes"], g["scales"], g["zeros"], g["g_idx"])
+    e_gpu, _ = O.layer_error(W64, deq, ref["H0"], n)
+    e_ref, _ = O.layer_error(W64, O.dequantize_layer(ref["codes"], ref["scales"], ref["zeros"],
+                                                     ref["g_idx"]), ref["H0"], n)
+    assert abs(e_gpu - e_ref) <= 0.01 * e_ref, (e_gpu, e_ref)
 
 
 # ----------------------------------------------------------------- end to end

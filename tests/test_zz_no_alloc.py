@@ -88,9 +88,19 @@ def test_noalloc_matches_workspace_call_twice(g, out, in_, bits, gs, sym, desc_a
 
     for call in range(2):
         o = _outputs(out, in_, cfg)
+        torch.cuda.synchronize()
+        free0, _ = torch.cuda.mem_get_info()
+        alloc0 = torch.cuda.memory_allocated()
         g.gptq_quantize_layer_noalloc(W_t, U, perm, dead, cfg, o["scales"], o["zeros"], o["g_idx"],
                                       codes=o["codes"], qweight=o.get("qweight"), loss=o["loss"])
         torch.cuda.synchronize()
+        if call == 1:
+            # after the first call's set-up, a call takes no device memory:
+            # neither from the driver nor from torch's caching allocator
+            free1, _ = torch.cuda.mem_get_info()
+            assert free1 == free0, (free0, free1)
+            assert torch.cuda.memory_allocated() == alloc0
+        g.gptq_quantize_layer_noalloc_status()        # no device-side failure
         o = {k: host(v) for k, v in o.items()}
         # integer outputs bit-exact; floating point within 1e-6 relative
         for k in ("codes", "zeros", "g_idx", "qweight"):
