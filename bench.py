@@ -182,8 +182,8 @@ def oracle_setup(wl, layer, q, W, X):
 # The one sampling recipe both oracle legs use (the GPU line's cpu_baseline
 # and the reference arm): the Hessian over SAMPLE_TOKENS tokens, the whole
 # prepare, and the sweep of SAMPLE_ROWS rows over all columns.
-SAMPLE_TOKENS = 4096
-SAMPLE_ROWS = 64
+SAMPLE_TOKENS = 16384
+SAMPLE_ROWS = 512
 
 
 def oracle_sample(wl, layer, q, W, X, setup, tokens=SAMPLE_TOKENS, rows=SAMPLE_ROWS):
@@ -270,7 +270,7 @@ def run_reference(args):
                           "recipe_estimate_s": d_est["est_s_per_layer"], "recipe_split_s": d_est["split_s"],
                           "recipe_sample": d_est["sample"]}), flush=True)
         return
-    X = gen.x_full(wl, layer.site, tokens=max(2048, SAMPLE_TOKENS))
+    X = gen.x_full(wl, layer.site, tokens=SAMPLE_TOKENS)
     setup = oracle_setup(wl, layer, q, W, X)
     vals, detail = [], None
     t_run = time.perf_counter()

@@ -45,19 +45,31 @@ def code_report(gpu_codes, ref_codes):
     return float(eq.mean()), eq
 
 
-def compare_groups(gpu_s, gpu_z, ref_s, ref_z, codes_p_eq, group_size, rtol=1e-4):
-    """Compare scales (relative) and zeros (exact) on every group whose row
-    had no code mismatch before the group's first column (processing order).
-    Returns (n_compared, n_excluded)."""
+def compare_groups(gpu_s, gpu_z, ref_s, ref_z, codes_p_eq, group_size, rtol=1e-4, max_flips=1e-3):
+    """Compare scales (relative) and zeros on every group whose row had no
+    code mismatch before the group's first column (processing order).
+
+    A zero is an integer decided in fp32 from the group's current weights,
+    like the codes: where the two sides' weights differ in the last bits and
+    -lo / scale sits at a half-integer, the zero can come out one apart, and
+    then every code of the group differs by one as well.  So zeros must be
+    equal on every compared group whose codes all agree; groups whose zero
+    differs are decision flips, bounded like codes (at most ``max_flips`` of
+    the compared groups).  Returns (n_compared, n_excluded, n_zero_flips)."""
     out, ng = ref_s.shape
     n = codes_p_eq.shape[1]
     gs = n if group_size == -1 else group_size
     first_bad = np.where(codes_p_eq.all(1), n, np.argmin(codes_p_eq, axis=1))
     ok = np.zeros((out, ng), bool)
+    grp_eq = np.zeros((out, ng), bool)
     for g in range(ng):
         ok[:, g] = first_bad >= g * gs   # no mismatch strictly before the group start
+        grp_eq[:, g] = codes_p_eq[:, g * gs:(g + 1) * gs].all(1)
     gs_ = np.asarray(gpu_s, np.float64)[ok]
     rs_ = np.asarray(ref_s, np.float64)[ok]
     np.testing.assert_allclose(gs_, rs_, rtol=rtol)
-    assert np.array_equal(np.asarray(gpu_z)[ok], np.asarray(ref_z)[ok])
-    return int(ok.sum()), int((~ok).sum())
+    zeq = np.asarray(gpu_z) == np.asarray(ref_z)
+    assert np.all(zeq[ok & grp_eq]), "zero differs on a group whose codes all agree"
+    flips = int((ok & ~zeq).sum())
+    assert flips <= max_flips * max(int(ok.sum()), 1), (flips, int(ok.sum()))
+    return int(ok.sum()), int((~ok).sum()), flips
