@@ -1,0 +1,963 @@
+// Blocked Cholesky factorisation R = L L^T ("Using AutoGPTQ in Practice":
+// the Hessian's Cholesky factorization), with the inverse of every 64 x 64
+// diagonal block, in one cooperative launch.  R is the reversed, damped
+// Hessian of gptq_prepare_hinv (lower triangle, np x np, np a multiple of
+// 128); the blocked inverse of L that turns the result into U is formed
+// afterwards by tensor-core merges in prepare.cu.
+//
+// Right-looking with 64-wide blocks and a look-ahead of one block.  Step k
+// (between two grid barriers):
+//   CTA 0 (the chain)   L_{k+1,k} = R_{k+1,k} M_kk^T; R_{k+1,k+1} -= L L^T;
+//                       then the leaf of block k+1: its Cholesky factor and
+//                       the factor's inverse M_{k+1,k+1}, both in registers
+//                       of two warps (the inverse warp trails the factor warp
+//                       by a pivot or more, fed through shared memory).
+//   CTAs 1.. (workers)  tensor-core tile tasks, 3xTF32 on tcgen05:
+//                       panel tiles L_ik = R_ik M_kk^T (i >= k+2, 128 rows x
+//                       64 columns), then, once every panel tile of the step
+//                       is written, the trailing update R_ij -= L_ik L_jk^T
+//                       of the lower triangle from block k+1 on, in 128 x 128
+//                       tiles (block (k+1, k+1) excluded: CTA 0 updates it).
+// Products on the chain CTA are 64 x 64 x 64 and stay on CUDA cores.
+//
+// Worker CTAs: warps 0-3 stage the operands of a task in shared memory in
+// the tensor core's 128-byte-swizzled K-major layout (split fp32: tf32 hi
+// plus the exact remainder; L's panel tiles are stored split, R's tiles are
+// split while they are staged) and one of their threads issues the MMAs;
+// warps 4-7 read the accumulator from tensor memory and write the result.
+// Two tensor-memory accumulators let a task's epilogue overlap the next
+// task's staging and MMAs.
+//
+// Every wait is bounded by %globaltimer; a wait that gives up raises
+// ST_TIMEOUT, sets the launch-wide abort flag and unwinds.
+#include <algorithm>
+
+#include "gemm.cuh"
+#include "internal.cuh"
+
+namespace gptq {
+namespace {
+
+constexpr int FB = 64;        // block size of the factorisation
+constexpr int FNT = 256;      // threads per CTA
+constexpr int FP = FB + 1;    // pitch of the leaf's A and M tiles
+constexpr int TP = FB + 4;    // pitch of the chain's operand tiles (float4 rows)
+
+// worker shared-memory plan: four regions (A hi/lo, B hi/lo), each 128 rows x
+// two 128-byte K chunks (K = 64 tf32)
+constexpr uint32_t kChunkBytes = 128 * 128;         // 128 rows x 128 bytes
+constexpr uint32_t kRegionBytes = 2 * kChunkBytes;  // K = 64
+constexpr uint32_t kStageBytes = 32 * 128 * 4;      // one epilogue pass: 32 rows x 128 columns fp32
+constexpr int kStages = 4;                           // epilogue staging buffers (one per 32-row pass)
+constexpr uint32_t kWorkerSmem = 4 * kRegionBytes + kStages * kStageBytes;  // 192 KB
+constexpr uint32_t kTmemCols = 256;                 // two 128-column accumulators
+
+struct CholParams {
+  float* R;        // np x np (lower triangle used), updated in place
+  int64_t np_;
+  int T;           // np / 64
+  float *Lh, *Ll;  // split L: panel tiles below the diagonal blocks
+  float *Mh, *Ml;  // split diagonal blocks of M = L^-1
+  float *Mth, *Mtl;
+  unsigned* sync;  // [2] abort, [3] diagonal blocks published (M_kk for k < count)
+  int* pdone;      // [T]: panel tiles written in step k (CTA 0 adds one)
+  int* tdone;      // [T]: trailing tiles of step k whose reduce-adds have landed
+  int* t0done;     // [T]: 1 once trailing tile (0, 0) of step k has landed
+  uint32_t* status;
+};
+
+// ------------------------------------------------------------------ sync
+__device__ __forceinline__ bool aborted(const CholParams& p) {
+  return *(volatile unsigned*)(p.sync + 2) != 0;
+}
+
+__device__ __forceinline__ void give_up(const CholParams& p) {
+  raise_status(p.status, ST_TIMEOUT);
+  atomicExch(p.sync + 2, 1u);
+}
+
+// Wait until *f >= target (another CTA raises it), bounded by kWaitLimitNs;
+// false once any CTA has given up.  One thread; a __threadfence follows a
+// successful wait, so data published before the counter is then visible.
+__device__ bool wait_ge(const CholParams& p, const int* f, int target) {
+  volatile const int* vf = f;
+  if (vf[0] < target) {
+    const uint64_t t0 = globaltimer();
+    while (vf[0] < target) {
+      if (aborted(p)) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        give_up(p);
+        return false;
+      }
+      __nanosleep(64);
+    }
+  }
+  __threadfence();
+  return true;
+}
+
+// ------------------------------------------------------------------ copies
+// 16-byte global -> shared copy through L2 only (cp.async.cg): data other
+// CTAs write during the launch must not come from a stale L1 line.  With
+// valid == false the 16 bytes are zero-filled and nothing is read.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid = true) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// 2-D tiled bulk tensor reduce-add shared -> global (bulk-group completion),
+// clipped at the tensor map's bounds.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* smem_src, int32_t x,
+                                                  int32_t y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+// Order this thread's async-proxy global writes (bulk copies it waited for)
+// before its later generic-proxy operations.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Shared-memory flag between two warps of one CTA (release / acquire).
+__device__ __forceinline__ void st_release_cta(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_cta(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+
+// ------------------------------------------------------------------ chain CTA
+// S[r][t] (pitch TP) <- G[r][t] for an FB x FB tile (row stride ld), async.
+__device__ __forceinline__ void prefetch_tile(float* S, const float* G, int64_t ld) {
+  for (int e = threadIdx.x; e < FB * FB / 4; e += FNT) {
+    const int r = e / (FB / 4), t4 = (e % (FB / 4)) * 4;
+    cp_async16(S + r * TP + t4, G + (int64_t)r * ld + t4);
+  }
+}
+
+// acc[u][v] = sum_t X[tr + 16u][t] Y[tc + 16v][t]   (tr = tid / 16, tc = tid % 16)
+// X, Y row-major tiles of pitch TP.  Output rows and columns are strided by
+// 16 so that the 16 column groups of a warp read 16 consecutive rows of Y.
+__device__ __forceinline__ void tile_product(const float* X, const float* Y, float acc[4][4]) {
+  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
+#pragma unroll 2
+  for (int t = 0; t < FB; t += 4) {
+    float4 x[4], y[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = *reinterpret_cast<const float4*>(X + (tr + 16 * u) * TP + t);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) y[v] = *reinterpret_cast<const float4*>(Y + (tc + 16 * v) * TP + t);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        acc[u][v] = fmaf(x[u].x, y[v].x, acc[u][v]);
+        acc[u][v] = fmaf(x[u].y, y[v].y, acc[u][v]);
+        acc[u][v] = fmaf(x[u].z, y[v].z, acc[u][v]);
+        acc[u][v] = fmaf(x[u].w, y[v].w, acc[u][v]);
+      }
+  }
+}
+
+// The leaf: A (FB x FB, pitch FP, lower triangle read) -> M = L^-1 (pitch FP,
+// zeros above the diagonal), where A = L L^T.  Six warps, each a chain of
+// pivots over registers, fed through shared memory:
+//   warp 0  factors rows 0..31 (pivots 0..31); lane i keeps row i;
+//   warp 1  rows 32..63, columns 0..31: forms L[32+i][j] for pivots 0..31
+//           from the pivots warp 0 publishes;
+//   warp 6  rows 32..63, columns 32..63: applies the first 32 pivots' updates
+//           to the trailing block, then factors it (pivots 32..63);
+//   warp 2  inverts L00 (M00 = L00^-1 by forward substitution, lane = column),
+//           trailing warp 0 by a pivot or more;
+//   warp 3  inverts L11 (M11) behind warp 6;
+//   warp 5  zeroes the upper block of M.
+// Warp w issues on scheduler w % 4: the factor chains (warps 0, 1 and, for
+// pivots 32..63, 6) each have a scheduler to themselves while they run.
+// Then every warp forms M10 = -M11 (L10 M00).  Column j of L goes to Lc[j][.]
+// and 1/L_jj to rdiag[j]; fl[0..2] count the pivots published by warps 0, 1
+// and 6 (release / acquire, once per pass of four pivots).  Each lane keeps a 32-entry window of its row
+// (or column) that slides by four pivots per pass, so every register index is
+// a compile-time constant and the code of one pass serves all passes.  A
+// non-positive or non-finite pivot raises ST_NOT_PD (it is replaced by 1 so
+// the leaf finishes).  False if a wait gave up.
+constexpr int LCP = 64;  // pitch of Lc (one column of L per row)
+
+__device__ __forceinline__ bool wait_count(const int* f, int j) {
+  if (ld_acquire_cta(f) > j) return true;
+  const uint64_t t0 = globaltimer();
+  while (ld_acquire_cta(f) <= j) {
+    __nanosleep(32);  // leave the issue slots to the warp being waited for
+    if (globaltimer() - t0 > kWaitLimitNs) return false;
+  }
+  return true;
+}
+
+// w[t] -= s * col[t] for t in (u, 32), col 16-byte aligned (8 vector loads).
+template <int U>
+__device__ __forceinline__ void axpy_window(float (&w)[32], float s, const float* col) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 c4 = *reinterpret_cast<const float4*>(col + 4 * q);
+    if (4 * q + 0 > U) w[4 * q + 0] = fmaf(-s, c4.x, w[4 * q + 0]);
+    if (4 * q + 1 > U) w[4 * q + 1] = fmaf(-s, c4.y, w[4 * q + 1]);
+    if (4 * q + 2 > U) w[4 * q + 2] = fmaf(-s, c4.z, w[4 * q + 2]);
+    if (4 * q + 3 > U) w[4 * q + 3] = fmaf(-s, c4.w, w[4 * q + 3]);
+  }
+}
+
+__device__ __forceinline__ void shift4(float (&w)[32]) {
+#pragma unroll
+  for (int t = 0; t < 28; ++t) w[t] = w[t + 4];
+#pragma unroll
+  for (int t = 28; t < 32; ++t) w[t] = 0.f;
+}
+
+// One factor pivot on a window whose slot U holds column j of the lane's row
+// (row j itself sits on lane jl): publish column j (rows row0 + lane) and
+// 1/L_jj, then update the window with the column's rows col0 .. col0 + 31.
+// The chain from one pivot to the next runs through registers only: dn is,
+// on the lane of the pivot row, the fully updated diagonal entry.  Row j + 1's
+// lane forms its next diagonal entry from its own L[j+1][j] (w - l l), and the
+// column j + 1 entries of every lane take L[j+1][j] by shuffle; the other
+// columns are updated from shared memory, two or more pivots ahead of use.
+template <int U>
+__device__ __forceinline__ bool factor_pivot(float (&w)[32], float& dn, int j, int jl, int row0, float* Lc,
+                                             float* rdiag, const float* col) {
+  const int lane = threadIdx.x & 31;
+  float d = __shfl_sync(0xffffffffu, dn, jl);
+  bool bad = false;
+  if (!(d > 0.f) || !isfinite(d)) {
+    bad = true;
+    d = 1.f;
+  }
+  const float rs = rsqrtf(d);
+  const float l = w[U] * rs;
+  dn = fmaf(-l, l, w[U + 1]);                               // lane jl + 1: next pivot
+  const float c1 = __shfl_sync(0xffffffffu, l, (jl + 1) & 31);  // L[j+1][j]
+  w[U + 1] = fmaf(-l, c1, w[U + 1]);
+  Lc[j * LCP + row0 + lane] = l;
+  if (lane == 0) rdiag[j] = rs;
+  __syncwarp();
+  axpy_window<U + 1>(w, l, col);
+  return bad;
+}
+
+// Publish pivots up to j (inclusive) to the warps that wait on flag: once per
+// pass of four pivots, after the pass's columns are in shared memory.
+__device__ __forceinline__ void publish(int* flag, int j) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) st_release_cta(flag, j + 1);
+}
+
+// Tiles of the chain's next step, fetched by warp 7 while the leaf runs, once
+// the workers have applied every update to them.
+struct NextTiles {
+  bool active;
+  float *X, *C;               // shared destinations (pitch TP)
+  const float *gX, *gC;       // R tiles (k+2, k+1) and (k+2, k+2)
+  int k;                      // the step whose trailing tile (0, 0) must have landed
+  int tdone_target;           // tiles of step k - 1 that must have landed (0: none)
+};
+
+__device__ void fetch_next_tiles(const NextTiles& nt, int64_t np, const CholParams& p) {
+  const int lane = threadIdx.x & 31;
+  __shared__ int go;
+  if (lane == 0) {
+    bool ok = true;
+    if (nt.k >= 0) ok = wait_ge(p, &p.t0done[nt.k], 1);
+    if (ok && nt.tdone_target > 0) ok = wait_ge(p, &p.tdone[nt.k - 1], nt.tdone_target);
+    go = ok;
+  }
+  __syncwarp();
+  if (!go) return;
+  for (int e = lane; e < 2 * FB * FB / 4; e += 32) {
+    const int which = e / (FB * FB / 4), q = e % (FB * FB / 4);
+    const int r = q / (FB / 4), t4 = (q % (FB / 4)) * 4;
+    cp_async16((which ? nt.C : nt.X) + r * TP + t4, (which ? nt.gC : nt.gX) + (int64_t)r * np + t4);
+  }
+  cp_async_commit();
+  cp_async_wait<0>();
+}
+
+__device__ bool leaf64(const float* A, float* M, float* X, float* Lc, float* rdiag, int* fl, const CholParams& p,
+                       const NextTiles& nt) {
+  __shared__ int ok_s;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x < 3) fl[threadIdx.x] = 0;
+  if (threadIdx.x == 0) ok_s = 1;
+  __syncthreads();
+  bool ok = true, bad = false;
+  if (warp == 0) {
+    float w[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) w[t] = t <= lane ? A[lane * FP + t] : 0.f;
+    float dn = w[0];
+#pragma unroll 1
+    for (int m = 0; m < 8; ++m) {
+      const float* col = Lc + 4 * m;
+      bad |= factor_pivot<0>(w, dn, 4 * m + 0, 4 * m + 0, 0, Lc, rdiag, col + (4 * m + 0) * LCP);
+      bad |= factor_pivot<1>(w, dn, 4 * m + 1, 4 * m + 1, 0, Lc, rdiag, col + (4 * m + 1) * LCP);
+      bad |= factor_pivot<2>(w, dn, 4 * m + 2, 4 * m + 2, 0, Lc, rdiag, col + (4 * m + 2) * LCP);
+      bad |= factor_pivot<3>(w, dn, 4 * m + 3, 4 * m + 3, 0, Lc, rdiag, col + (4 * m + 3) * LCP);
+      publish(&fl[0], 4 * m + 3);
+      shift4(w);
+    }
+  } else if (warp == 1) {
+    // rows 32..63, columns 0..31: L[32+i][j] = A'[32+i][j] / L_jj
+    float v[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) v[t] = A[(32 + lane) * FP + t];
+#pragma unroll 1
+    for (int m = 0; m < 8 && ok; ++m) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = 4 * m + u;
+        if (!wait_count(&fl[0], j)) ok = false;
+        const float l = v[u] * rdiag[j];
+        Lc[j * LCP + 32 + lane] = l;
+        __syncwarp();
+        const float* col = Lc + j * LCP + 4 * m;
+        switch (u) {
+          case 0: axpy_window<0>(v, l, col); break;
+          case 1: axpy_window<1>(v, l, col); break;
+          case 2: axpy_window<2>(v, l, col); break;
+          default: axpy_window<3>(v, l, col); break;
+        }
+      }
+      publish(&fl[1], 4 * m + 3);
+      shift4(v);
+    }
+  } else if (warp == 6) {
+    float z[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) z[t] = t <= lane ? A[(32 + lane) * FP + 32 + t] : 0.f;
+    // the first 32 pivots' updates of the trailing block
+#pragma unroll 1
+    for (int j = 0; j < 32 && ok; ++j) {
+      if (!wait_count(&fl[1], j)) ok = false;
+      const float li = Lc[j * LCP + 32 + lane];
+      axpy_window<-1>(z, li, Lc + j * LCP + 32);
+    }
+    // then its own factorisation, pivots 32..63
+    float dn = z[0];
+#pragma unroll 1
+    for (int m = 0; m < 8; ++m) {
+      const float* col = Lc + 32 + 4 * m;
+      bad |= factor_pivot<0>(z, dn, 32 + 4 * m + 0, 4 * m + 0, 32, Lc, rdiag, col + (32 + 4 * m + 0) * LCP);
+      bad |= factor_pivot<1>(z, dn, 32 + 4 * m + 1, 4 * m + 1, 32, Lc, rdiag, col + (32 + 4 * m + 1) * LCP);
+      bad |= factor_pivot<2>(z, dn, 32 + 4 * m + 2, 4 * m + 2, 32, Lc, rdiag, col + (32 + 4 * m + 2) * LCP);
+      bad |= factor_pivot<3>(z, dn, 32 + 4 * m + 3, 4 * m + 3, 32, Lc, rdiag, col + (32 + 4 * m + 3) * LCP);
+      publish(&fl[2], 32 + 4 * m + 3);
+      shift4(z);
+    }
+  } else if (warp == 2 || warp == 3) {
+    // forward substitution M = L^-1 on one diagonal 32-block, lane = column
+    const int o = warp == 2 ? 0 : 32;
+    const int* f = warp == 2 ? &fl[0] : &fl[2];
+    float x[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) x[t] = t == lane ? 1.f : 0.f;
+#pragma unroll 1
+    for (int m = 0; m < 8 && ok; ++m) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = o + 4 * m + u;
+        if (!wait_count(f, j)) ok = false;
+        const float mj = x[u] * rdiag[j];
+        M[j * FP + o + lane] = mj;
+        const float* col = Lc + j * LCP + o + 4 * m;
+        switch (u) {
+          case 0: axpy_window<0>(x, mj, col); break;
+          case 1: axpy_window<1>(x, mj, col); break;
+          case 2: axpy_window<2>(x, mj, col); break;
+          default: axpy_window<3>(x, mj, col); break;
+        }
+      }
+      shift4(x);
+    }
+  } else if (warp == 5) {
+    for (int e = lane; e < 32 * 32; e += 32) M[(e >> 5) * FP + 32 + (e & 31)] = 0.f;
+  } else if (warp == 7 && nt.active) {
+    fetch_next_tiles(nt, p.np_, p);
+  }
+  if (bad && lane == 0) raise_status(p.status, ST_NOT_PD);
+  if (!ok && lane == 0) ok_s = 0;
+  __syncthreads();
+  // M10 = -M11 (L10 M00): X = L10 M00, then M10 = -M11 X (32 x 32 x 32 each,
+  // 2 x 2 outputs per thread)
+  {
+    const int r0 = (threadIdx.x / 16) * 2, c0 = (threadIdx.x % 16) * 2;
+    float acc[2][2] = {};
+#pragma unroll 4
+    for (int t = 0; t < 32; ++t) {
+      const float a0 = Lc[t * LCP + 32 + r0], a1 = Lc[t * LCP + 33 + r0];  // L[32 + r][t]
+      const float b0 = M[t * FP + c0], b1 = M[t * FP + c0 + 1];
+      acc[0][0] = fmaf(a0, b0, acc[0][0]);
+      acc[0][1] = fmaf(a0, b1, acc[0][1]);
+      acc[1][0] = fmaf(a1, b0, acc[1][0]);
+      acc[1][1] = fmaf(a1, b1, acc[1][1]);
+    }
+    X[r0 * FP + c0] = acc[0][0];
+    X[r0 * FP + c0 + 1] = acc[0][1];
+    X[(r0 + 1) * FP + c0] = acc[1][0];
+    X[(r0 + 1) * FP + c0 + 1] = acc[1][1];
+    __syncthreads();
+    float bcc[2][2] = {};
+#pragma unroll 4
+    for (int t = 0; t < 32; ++t) {
+      const float a0 = M[(32 + r0) * FP + 32 + t], a1 = M[(33 + r0) * FP + 32 + t];
+      const float b0 = X[t * FP + c0], b1 = X[t * FP + c0 + 1];
+      bcc[0][0] = fmaf(a0, b0, bcc[0][0]);
+      bcc[0][1] = fmaf(a0, b1, bcc[0][1]);
+      bcc[1][0] = fmaf(a1, b0, bcc[1][0]);
+      bcc[1][1] = fmaf(a1, b1, bcc[1][1]);
+    }
+    M[(32 + r0) * FP + c0] = -bcc[0][0];
+    M[(32 + r0) * FP + c0 + 1] = -bcc[0][1];
+    M[(33 + r0) * FP + c0] = -bcc[1][0];
+    M[(33 + r0) * FP + c0 + 1] = -bcc[1][1];
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// Diagonal block b of M (pitch FP) -> split Mh/Ml and, transposed, Mth/Mtl.
+__device__ void store_diag_m(const CholParams& p, const float* M, int b) {
+  const int64_t o = (int64_t)b * FB;
+  for (int e = threadIdx.x; e < FB * FB; e += FNT) {
+    const int r = e / FB, c = e % FB;
+    const float v = M[r * FP + c], vt = M[c * FP + r];
+    float h, l;
+    split_tf32(v, h, l);
+    p.Mh[(o + r) * p.np_ + o + c] = h;
+    p.Ml[(o + r) * p.np_ + o + c] = l;
+    split_tf32(vt, h, l);
+    p.Mth[(o + r) * p.np_ + o + c] = h;
+    p.Mtl[(o + r) * p.np_ + o + c] = l;
+  }
+}
+
+// ------------------------------------------------------------------ workers
+// Byte offset of 16-byte unit u (0..7) of row r in a 128-byte-swizzled
+// K-major chunk (the layout TMA's 128-byte swizzle produces): the unit index
+// is XOR-ed with the row's position inside its 8-row, 1024-byte group.
+__device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+
+// Stage rows [row0, row0 + nrows) x columns [col0, col0 + 64) of a split
+// matrix (hi, lo; row stride ld) into regions Shi, Slo: 128-byte swizzled,
+// two K chunks of 32.  Rows at or past rmax are zero-filled.  Loader threads
+// only (128).
+__device__ __forceinline__ void stage_split(uint8_t* Shi, uint8_t* Slo, const float* hi, const float* lo,
+                                            int64_t ld, int64_t row0, int nrows, int64_t col0, int64_t rmax) {
+  const int lt = threadIdx.x;  // 0..127
+  for (int e = lt; e < nrows * 16; e += 128) {
+    const int r = e >> 4, g = e & 15;  // g: 16-byte unit along K (0..15)
+    const int ch = g >> 3, u = g & 7;
+    const int64_t gr = row0 + r;
+    const bool valid = gr < rmax;
+    const int64_t off = (valid ? gr : 0) * ld + col0 + 4 * g;
+    const uint32_t so = ch * kChunkBytes + sw128(r, u);
+    cp_async16(Shi + so, hi + off, valid);
+    cp_async16(Slo + so, lo + off, valid);
+  }
+}
+
+// The same from an unsplit fp32 matrix (split while staging), 128 rows: all
+// sixteen 16-byte loads of a thread are in flight before the first store.
+__device__ __forceinline__ void stage_fp32(uint8_t* Shi, uint8_t* Slo, const float* src, int64_t ld,
+                                           int64_t row0, int64_t col0, int64_t rmax) {
+  const int lt = threadIdx.x;
+  float4 v[16];
+#pragma unroll
+  for (int it = 0; it < 16; ++it) {
+    const int e = lt + 128 * it;
+    const int r = e >> 4, g = e & 15;
+    const int64_t gr = row0 + r;
+    v[it] = gr < rmax ? __ldcg(reinterpret_cast<const float4*>(src + gr * ld + col0 + 4 * g))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+#pragma unroll
+  for (int it = 0; it < 16; ++it) {
+    const int e = lt + 128 * it;
+    const int r = e >> 4, g = e & 15;
+    const int ch = g >> 3, u = g & 7;
+    float4 h, l;
+    split_tf32(v[it].x, h.x, l.x);
+    split_tf32(v[it].y, h.y, l.y);
+    split_tf32(v[it].z, h.z, l.z);
+    split_tf32(v[it].w, h.w, l.w);
+    const uint32_t so = ch * kChunkBytes + sw128(r, u);
+    *reinterpret_cast<float4*>(Shi + so) = h;
+    *reinterpret_cast<float4*>(Slo + so) = l;
+  }
+}
+
+// 24 MMAs: D (+)= A B^T over K = 64 with split operands (hi hi + hi lo + lo hi).
+__device__ __forceinline__ void issue_mma(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi, uint32_t b_lo,
+                                          uint32_t idesc) {
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint32_t off = ch * kChunkBytes + kk * 32;
+      const uint64_t ah = smem_desc_k_sw128(a_hi + off), al = smem_desc_k_sw128(a_lo + off);
+      const uint64_t bh = smem_desc_k_sw128(b_hi + off), bl = smem_desc_k_sw128(b_lo + off);
+      umma_tf32(d, ah, bh, idesc, (ch | kk) ? 1u : 0u);
+      umma_tf32(d, ah, bl, idesc, 1u);
+      umma_tf32(d, al, bh, idesc, 1u);
+    }
+}
+
+// Task t of step k: a panel tile (t < npan) or a trailing tile.
+struct Task {
+  int kind;     // 0 panel, 1 trailing
+  int64_t r0;   // first row of the output tile
+  int64_t c0;   // first column of the output tile (trailing) / of the panel
+  int diag;     // trailing tile on the diagonal (both operands the same rows)
+};
+
+__device__ __forceinline__ Task task_of(int64_t np, int k, int t, int npan) {
+  Task x;
+  if (t < npan) {
+    x.kind = 0;
+    x.r0 = (int64_t)FB * (k + 2) + 128 * (int64_t)t;
+    x.c0 = (int64_t)FB * k;
+    x.diag = 0;
+    return x;
+  }
+  const int q = t - npan;
+  // lower-triangular tile (a, b), b <= a, numbered row by row
+  int a = (int)((sqrtf(8.f * (float)q + 1.f) - 1.f) * 0.5f);
+  while ((a + 1) * (a + 2) / 2 <= q) ++a;
+  while (a * (a + 1) / 2 > q) --a;
+  const int b = q - a * (a + 1) / 2;
+  const int64_t s = (int64_t)FB * (k + 1);
+  x.kind = 1;
+  x.r0 = s + 128 * (int64_t)a;
+  x.c0 = s + 128 * (int64_t)b;
+  x.diag = a == b;
+  return x;
+}
+
+__device__ __forceinline__ void step_tasks(int64_t np, int k, int& npan, int& ntrail) {
+  const int64_t pr0 = (int64_t)FB * (k + 2);
+  npan = pr0 < np ? (int)((np - pr0 + 127) / 128) : 0;
+  const int64_t s = (int64_t)FB * (k + 1);
+  const int64_t rem = np - s;
+  const int m = rem > FB ? (int)((rem + 127) / 128) : 0;
+  ntrail = m * (m + 1) / 2;
+}
+
+__global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CUtensorMap rmap,
+                                                      const CholParams p) {
+  extern __shared__ __align__(1024) uint8_t csm_raw[];
+  uint8_t* csm = (uint8_t*)(((uintptr_t)csm_raw + 1023) & ~(uintptr_t)1023);
+  const int64_t np = p.np_;
+  const int T = p.T;
+  const int cta = blockIdx.x;
+  const int G = gridDim.x;
+
+  if (cta == 0) {
+    // ---------------------------------------------------------------- chain
+    float* fsm = reinterpret_cast<float*>(csm);
+    float* Xb2 = fsm;                // [2][FB][TP] R_{k+1,k} (double-buffered across steps)
+    float* Cb2 = Xb2 + 2 * FB * TP;  // [2][FB][TP] R_{k+1,k+1}
+    float* Yb = Cb2 + 2 * FB * TP;   // [FB][TP] M_kk
+    float* LT = Yb + FB * TP;        // [FB][TP] L_{k+1,k}
+    float* A = LT + FB * TP;         // [FB][FP]
+    float* M = A + FB * FP;          // [FB][FP]
+    float* Xs = M + FB * FP;         // [32][FP] scratch of the leaf's merge
+    float* Lc = Xs + 32 * FP;        // [FB][LCP] columns of L (leaf), 16-byte aligned
+    float* rdiag = Lc + FB * LCP;    // [FB]
+    int* fl = reinterpret_cast<int*>(rdiag + FB);
+    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+    auto tile = [&](int i, int j) { return p.R + (int64_t)i * FB * np + (int64_t)j * FB; };
+    // the next step's tiles, for warp 7 during the leaf of step k (k = -1:
+    // the first diagonal block's leaf, whose next tiles no one updates)
+    auto next_tiles = [&](int k) {
+      NextTiles nt;
+      nt.active = k + 2 < T;
+      const int b = (k + 1) & 1;
+      nt.X = Xb2 + b * FB * TP;
+      nt.C = Cb2 + b * FB * TP;
+      nt.gX = tile(k + 2, k + 1);
+      nt.gC = tile(k + 2, k + 2);
+      nt.k = k;
+      nt.tdone_target = 0;
+      if (k >= 1) {
+        int np_, nt_;
+        step_tasks(np, k - 1, np_, nt_);
+        nt.tdone_target = nt_;
+      }
+      return nt;
+    };
+    auto publish_m = [&](int count) {
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicExch((int*)&p.sync[3], count);
+      }
+    };
+    // the first diagonal block
+    for (int e = threadIdx.x; e < FB * FB; e += FNT) {
+      const int r = e / FB, c = e % FB;
+      A[r * FP + c] = __ldcg(p.R + (int64_t)r * np + c);
+    }
+    __syncthreads();
+    if (!leaf64(A, M, Xs, Lc, rdiag, fl, p, next_tiles(-1))) give_up(p);
+    store_diag_m(p, M, 0);
+    publish_m(1);
+    for (int k = 0; k + 1 < T && !aborted(p); ++k) {
+      float acc[4][4];
+      const float* Xb = Xb2 + (k & 1) * FB * TP;
+      const float* Cb = Cb2 + (k & 1) * FB * TP;
+      // this step's tiles arrived during the previous leaf (warp 7 waited for
+      // its copies before the leaf's closing barrier)
+      for (int e = threadIdx.x; e < FB * FB; e += FNT) {
+        const int r = e / FB, c = e % FB;
+        Yb[r * TP + c] = M[r * FP + c];
+      }
+      __syncthreads();
+      // L_{k+1,k} = R_{k+1,k} M_kk^T, published split for the workers
+      tile_product(Xb, Yb, acc);
+      {
+        const int64_t base = (int64_t)(k + 1) * FB * np + (int64_t)k * FB;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int r = tr + 16 * u, c = tc + 16 * v;
+            float h, l;
+            split_tf32(acc[u][v], h, l);
+            p.Lh[base + (int64_t)r * np + c] = h;
+            p.Ll[base + (int64_t)r * np + c] = l;
+            LT[r * TP + c] = acc[u][v];
+          }
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(&p.pdone[k], 1);
+      }
+      tile_product(LT, LT, acc);  // L L^T
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int r = tr + 16 * u, c = tc + 16 * v;
+          A[r * FP + c] = Cb[r * TP + c] - acc[u][v];
+        }
+      __syncthreads();
+      if (!leaf64(A, M, Xs, Lc, rdiag, fl, p, next_tiles(k))) give_up(p);
+      store_diag_m(p, M, k + 1);
+      publish_m(k + 2);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------------ workers
+  uint8_t* SAh = csm;
+  uint8_t* SAl = SAh + kRegionBytes;
+  uint8_t* SBh = SAl + kRegionBytes;
+  uint8_t* SBl = SBh + kRegionBytes;
+  float* stg = reinterpret_cast<float*>(SBl + kRegionBytes);  // [kStages][32][128] epilogue staging
+  __shared__ uint64_t smem_free, acc_full[2], acc_empty[2], drain;
+  __shared__ uint32_t tmem_slot;
+  __shared__ int local_abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&smem_free, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(&drain, 1);
+    local_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tmem_slot, kTmemCols);
+    tmem_relinquish();
+    if (lane == 0) tma_prefetch_desc(&rmap);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tmem_slot;
+  const int W = G - 1, slot = cta - 1;
+  const uint32_t aH = smem_u32(SAh), aL = smem_u32(SAl), bH = smem_u32(SBh), bL = smem_u32(SBl);
+  int tcount = 0;    // tasks of this CTA so far (all steps): drives the barrier phases
+  int epi_pass = 0;  // epilogue staging passes (selects the staging buffer)
+  bool ok = true;
+  for (int k = 0; ok && k + 1 < T; ++k) {
+    int npan, ntrail;
+    step_tasks(np, k, npan, ntrail);
+    const int ntask = npan + ntrail;
+    if (warp < 4) {
+      // ------------------------------------------------ staging and MMA issue
+      // the step's inputs: M_kk published, and every trailing tile of the
+      // previous step landed (so column block k of R is final and the reduce-
+      // adds of consecutive steps reach each element in order)
+      if (threadIdx.x == 0) {
+        bool w = wait_ge(p, (const int*)&p.sync[3], k + 1);
+        if (w && k > 0) {
+          int pn, pt;
+          step_tasks(np, k - 1, pn, pt);
+          w = wait_ge(p, &p.tdone[k - 1], pt);
+        }
+        if (!w) local_abort = 1;
+      }
+      named_bar_sync(1, 128);
+      bool panels_seen = false;
+      int tl = tcount;
+      for (int t = slot; t < ntask && !local_abort; t += W, ++tl) {
+        const Task x = task_of(np, k, t, npan);
+        if (x.kind == 1 && !panels_seen) {
+          // every panel tile of the step (npan by workers, one by CTA 0)
+          if (threadIdx.x == 0 && !wait_ge(p, &p.pdone[k], npan + 1)) local_abort = 1;
+          named_bar_sync(1, 128);
+          panels_seen = true;
+          if (local_abort) break;
+        }
+        // the previous task's MMAs have read the staged operands
+        if (tl > 0 && !mbar_wait(&smem_free, (tl - 1) & 1)) {
+          give_up(p);
+          local_abort = 1;
+          break;
+        }
+        if (x.kind == 0) {
+          stage_fp32(SAh, SAl, p.R, np, x.r0, x.c0, np);
+          stage_split(SBh, SBl, p.Mh, p.Ml, np, x.c0, FB, x.c0, np);
+        } else {
+          stage_split(SAh, SAl, p.Lh, p.Ll, np, x.c0, 128, (int64_t)FB * k, np);
+          if (!x.diag) stage_split(SBh, SBl, p.Lh, p.Ll, np, x.r0, 128, (int64_t)FB * k, np);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 0) {
+          const int buf = tl & 1;
+          const int use = tl >> 1;
+          if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) {
+            give_up(p);
+            local_abort = 1;
+          } else {
+            tc_fence_after();
+            const uint32_t d = tbase + (uint32_t)buf * 128;
+            if (x.kind == 0) {
+              // D[r][c] = sum_t R[r][t] M[c][t]: lanes = rows, N = 64 columns
+              issue_mma(d, aH, aL, bH, bL, make_idesc(2, 128, 64));
+            } else {
+              // D[c][r] = sum_t L[c][t] L[r][t]: lanes = columns, N = 128 rows
+              const uint32_t b_hi = x.diag ? aH : bH, b_lo = x.diag ? aL : bL;
+              issue_mma(d, aH, aL, b_hi, b_lo, make_idesc(2, 128, 128));
+            }
+            umma_commit(&smem_free);
+            umma_commit(&acc_full[buf]);
+          }
+        }
+        named_bar_sync(1, 128);
+      }
+    } else {
+      // ------------------------------------------------ epilogue (warps 4-7)
+      const int quarter = warp & 3;
+      const int cl = quarter * 32 + lane;
+      int tl = tcount;
+      for (int t = slot; t < ntask; t += W, ++tl) {
+        const Task x = task_of(np, k, t, npan);
+        const int buf = tl & 1;
+        if (!mbar_wait_sleep(&acc_full[buf], (tl >> 1) & 1)) {
+          give_up(p);
+          local_abort = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
+        if (x.kind == 0) {
+          const int64_t r = x.r0 + quarter * 32 + lane;
+#pragma unroll
+          for (int n0 = 0; n0 < FB; n0 += 32) {
+            float v[32];
+            tmem_ld32(taddr + (uint32_t)n0, v);
+            if (r < np) {
+              float* dh = p.Lh + r * np + x.c0 + n0;
+              float* dl = p.Ll + r * np + x.c0 + n0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4) {
+                float4 h, l;
+                split_tf32(v[j + 0], h.x, l.x);
+                split_tf32(v[j + 1], h.y, l.y);
+                split_tf32(v[j + 2], h.z, l.z);
+                split_tf32(v[j + 3], h.w, l.w);
+                *reinterpret_cast<float4*>(dh + j) = h;
+                *reinterpret_cast<float4*>(dl + j) = l;
+              }
+            }
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
+          named_bar_sync(2, 128);
+          if (threadIdx.x == 128) {
+            __threadfence();
+            atomicAdd(&p.pdone[k], 1);
+          }
+        } else {
+          // R -= D by TMA reduce-add in L2, 32 rows per pass through one of
+          // kStages staging tiles; elements outside the update (above
+          // the diagonal, in block (k+1, k+1), past the matrix) add zero
+          const int64_t s = (int64_t)FB * (k + 1);
+          const int64_t c = x.c0 + cl;
+#pragma unroll 1
+          for (int pz = 0; pz < 4; ++pz) {
+            float v[32];
+            tmem_ld32(taddr + (uint32_t)(32 * pz), v);
+            const int64_t rb = x.r0 + 32 * pz;
+            float* sb = stg + (epi_pass % kStages) * (32 * 128);
+            if (threadIdx.x == 128) bulk_wait_read<kStages - 1>();  // the reduce that last read sb is done
+            named_bar_sync(2, 128);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int64_t r = rb + j;
+              const bool kp = r < np && c <= r && !(r < s + FB && c < s + FB);
+              sb[j * 128 + cl] = kp ? -v[j] : 0.f;
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(2, 128);
+            if (threadIdx.x == 128) {
+              tma_reduce_add_2d(&rmap, sb, (int32_t)x.c0, (int32_t)rb);
+              bulk_commit();
+            }
+            ++epi_pass;
+          }
+          tc_fence_before();
+          mbar_arrive(&acc_empty[buf]);
+          if (t == npan && threadIdx.x == 128) {
+            // trailing tile (0, 0) holds the chain's next two tiles
+            bulk_wait_all();
+            fence_proxy_async_global();
+            __threadfence();
+            atomicExch(&p.t0done[k], 1);
+          }
+        }
+      }
+    }
+    if (threadIdx.x == 128) {
+      // this CTA's reduce-adds of the step have landed: count them
+      int mine = 0;
+      for (int t = slot; t < ntask; t += W) mine += t >= npan;
+      bulk_wait_all();
+      fence_proxy_async_global();
+      __threadfence();
+      if (mine) atomicAdd(&p.tdone[k], mine);
+    }
+    // both groups walked the same task list
+    for (int t = slot; t < ntask; t += W) ++tcount;
+    ok = !local_abort && !aborted(p);
+  }
+  if (threadIdx.x == 128) bulk_wait_all();
+  __syncthreads();
+  if (local_abort || aborted(p)) {
+    // let MMAs already issued finish before the tensor memory goes away
+    if (threadIdx.x == 0) {
+      umma_commit(&drain);
+      mbar_wait(&drain, 0);
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, kTmemCols);
+  }
+}
+
+size_t chain_smem_bytes() {
+  return sizeof(float) * (6 * FB * TP + 2 * FB * FP + 32 * FP + FB * LCP + FB) + 16;
+}
+
+}  // namespace
+
+size_t chol_smem_bytes() { return 1024 + std::max<size_t>(kWorkerSmem, chain_smem_bytes()); }
+
+size_t chol_sync_bytes(int64_t np_) { return sizeof(int) * (size_t)(3 * (np_ / FB) + 4); }
+
+namespace {
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// R (np x np fp32, row-major) as a 2-D tensor with 128-column x 32-row boxes,
+// for the trailing update's reduce-add.
+bool make_r_map(CUtensorMap* m, float* R, int64_t np_) {
+  static EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return (EncodeTiledFn)f;
+  }();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {(cuuint64_t)np_, (cuuint64_t)np_};
+  cuuint64_t gstride[1] = {(cuuint64_t)(np_ * 4)};
+  cuuint32_t box[2] = {128, 32};
+  cuuint32_t estride[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, R, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, float* Ml, float* Mth, float* Mtl,
+                        unsigned* sync, uint32_t* status, int sms, cudaStream_t st) {
+  const size_t smem = chol_smem_bytes();
+  cudaError_t e = ensure_smem_limit((const void*)chol_kernel, (int)smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, chol_kernel, FNT, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  const int T = (int)(np_ / FB);
+  e = cudaMemsetAsync(sync, 0, chol_sync_bytes(np_), st);
+  if (e != cudaSuccess) return e;
+  // workers: enough for the first step's tasks (at most one CTA per SM)
+  const int64_t m = (np_ - FB + 127) / 128;
+  const int64_t tasks0 = (np_ - 2 * FB + 127) / 128 + m * (m + 1) / 2;
+  const int grid = (int)std::max<int64_t>(2, std::min<int64_t>(sms, 1 + tasks0));
+  CholParams p;
+  p.R = R;
+  p.np_ = np_;
+  p.T = T;
+  p.Lh = Lh;
+  p.Ll = Ll;
+  p.Mh = Mh;
+  p.Ml = Ml;
+  p.Mth = Mth;
+  p.Mtl = Mtl;
+  p.sync = sync;
+  p.pdone = (int*)(sync + 4);
+  p.tdone = p.pdone + T;
+  p.t0done = p.tdone + T;
+  p.status = status;
+  CUtensorMap rmap;
+  if (!make_r_map(&rmap, R, np_)) return cudaErrorInvalidValue;
+  void* args[] = {&rmap, &p};
+  e = cudaLaunchCooperativeKernel((const void*)chol_kernel, dim3(grid), dim3(FNT), args, smem, st);
+  note_launch();
+  return e;
+}
+
+}  // namespace gptq
