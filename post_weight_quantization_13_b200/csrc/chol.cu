@@ -63,6 +63,9 @@ struct CholParams {
   int* pdone;      // [T]: panel tiles written in step k (CTA 0 adds one)
   int* tdone;      // [T]: trailing tiles of step k whose reduce-adds have landed
   int* t0done;     // [T]: 1 once trailing tile (0, 0) of step k has landed
+  int* mrdone;     // [T]: tiles of block row k of M written
+  int* gdone;      // [T]: inverse-accumulator tiles of step k whose reduce-adds have landed
+  float* Gt;       // np x np: G^T, G_ij = sum over t < (current step) of L_it M_tj
   uint32_t* status;
 };
 
@@ -521,47 +524,84 @@ __device__ __forceinline__ void issue_mma(uint32_t d, uint32_t a_hi, uint32_t a_
     }
 }
 
-// Task t of step k: a panel tile (t < npan) or a trailing tile.
+// The tile tasks of step k, in this order:
+//   kind 2  M row tiles: M_kj = -M_kk G_kj for the columns before block k
+//           (128 columns each; G_kj is final once step k - 1's accumulation
+//           has landed);
+//   kind 0  panel tiles L_ik = R_ik M_kk^T, i >= k + 2 (128 rows each);
+//   kind 1  trailing tiles R_ij -= L_ik L_jk^T, lower triangle from block
+//           k + 1 on (128 x 128, block (k+1, k+1) excluded);
+//   kind 3  inverse accumulation G_ij += L_ik M_kj for the rows after block k
+//           and the columns up to block k (128 x 128).
+// So M = L^-1 is complete, block row by block row, when the factorisation
+// is; step T - 1 has only its M row tiles.
 struct Task {
-  int kind;     // 0 panel, 1 trailing
+  int kind;
   int64_t r0;   // first row of the output tile
-  int64_t c0;   // first column of the output tile (trailing) / of the panel
+  int64_t c0;   // first column of the output tile
   int diag;     // trailing tile on the diagonal (both operands the same rows)
 };
 
-__device__ __forceinline__ Task task_of(int64_t np, int k, int t, int npan) {
+struct StepTasks {
+  int nmrow, npan, ntrail, ngupd;
+  int mg;  // row tiles of the inverse accumulation
+  __host__ __device__ __forceinline__ int total() const { return nmrow + npan + ntrail + ngupd; }
+};
+
+__host__ __device__ __forceinline__ StepTasks step_tasks(int64_t np, int k) {
+  StepTasks st;
+  const int T = (int)(np / FB);
+  st.nmrow = (k + 1) / 2;  // columns [0, 64k) in 128-column tiles
+  const int64_t pr0 = (int64_t)FB * (k + 2);
+  st.npan = (k + 1 < T && pr0 < np) ? (int)((np - pr0 + 127) / 128) : 0;
+  const int64_t s = (int64_t)FB * (k + 1);
+  const int64_t rem = np - s;
+  const int m = (k + 1 < T && rem > FB) ? (int)((rem + 127) / 128) : 0;
+  st.ntrail = m * (m + 1) / 2;
+  st.mg = (k + 1 < T) ? (int)((rem + 127) / 128) : 0;
+  st.ngupd = st.mg * ((k + 2) / 2);  // columns [0, 64(k+1)) in 128-column tiles
+  return st;
+}
+
+__device__ __forceinline__ Task task_of(int64_t np, int k, int t, const StepTasks& st) {
   Task x;
-  if (t < npan) {
+  x.diag = 0;
+  if (t < st.nmrow) {
+    x.kind = 2;
+    x.r0 = (int64_t)FB * k;
+    x.c0 = 128 * (int64_t)t;
+    return x;
+  }
+  t -= st.nmrow;
+  if (t < st.npan) {
     x.kind = 0;
     x.r0 = (int64_t)FB * (k + 2) + 128 * (int64_t)t;
     x.c0 = (int64_t)FB * k;
-    x.diag = 0;
     return x;
   }
-  const int q = t - npan;
-  // lower-triangular tile (a, b), b <= a, numbered row by row
-  int a = (int)((sqrtf(8.f * (float)q + 1.f) - 1.f) * 0.5f);
-  while ((a + 1) * (a + 2) / 2 <= q) ++a;
-  while (a * (a + 1) / 2 > q) --a;
-  const int b = q - a * (a + 1) / 2;
+  t -= st.npan;
   const int64_t s = (int64_t)FB * (k + 1);
-  x.kind = 1;
-  x.r0 = s + 128 * (int64_t)a;
-  x.c0 = s + 128 * (int64_t)b;
-  x.diag = a == b;
+  if (t < st.ntrail) {
+    // lower-triangular tile (a, b), b <= a, numbered row by row
+    int a = (int)((sqrtf(8.f * (float)t + 1.f) - 1.f) * 0.5f);
+    while ((a + 1) * (a + 2) / 2 <= t) ++a;
+    while (a * (a + 1) / 2 > t) --a;
+    const int b = t - a * (a + 1) / 2;
+    x.kind = 1;
+    x.r0 = s + 128 * (int64_t)a;
+    x.c0 = s + 128 * (int64_t)b;
+    x.diag = a == b;
+    return x;
+  }
+  t -= st.ntrail;
+  x.kind = 3;
+  x.r0 = s + 128 * (int64_t)(t % st.mg);
+  x.c0 = 128 * (int64_t)(t / st.mg);
   return x;
 }
 
-__device__ __forceinline__ void step_tasks(int64_t np, int k, int& npan, int& ntrail) {
-  const int64_t pr0 = (int64_t)FB * (k + 2);
-  npan = pr0 < np ? (int)((np - pr0 + 127) / 128) : 0;
-  const int64_t s = (int64_t)FB * (k + 1);
-  const int64_t rem = np - s;
-  const int m = rem > FB ? (int)((rem + 127) / 128) : 0;
-  ntrail = m * (m + 1) / 2;
-}
-
 __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CUtensorMap rmap,
+                                                      const __grid_constant__ CUtensorMap gmap,
                                                       const CholParams p) {
   extern __shared__ __align__(1024) uint8_t csm_raw[];
   uint8_t* csm = (uint8_t*)(((uintptr_t)csm_raw + 1023) & ~(uintptr_t)1023);
@@ -597,11 +637,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       nt.gC = tile(k + 2, k + 2);
       nt.k = k;
       nt.tdone_target = 0;
-      if (k >= 1) {
-        int np_, nt_;
-        step_tasks(np, k - 1, np_, nt_);
-        nt.tdone_target = nt_;
-      }
+      if (k >= 1) nt.tdone_target = step_tasks(np, k - 1).ntrail;
       return nt;
     };
     auto publish_m = [&](int count) {
@@ -691,7 +727,10 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   if (warp == 0) {
     tmem_alloc(&tmem_slot, kTmemCols);
     tmem_relinquish();
-    if (lane == 0) tma_prefetch_desc(&rmap);
+    if (lane == 0) {
+      tma_prefetch_desc(&rmap);
+      tma_prefetch_desc(&gmap);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -702,34 +741,41 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   int tcount = 0;    // tasks of this CTA so far (all steps): drives the barrier phases
   int epi_pass = 0;  // epilogue staging passes (selects the staging buffer)
   bool ok = true;
-  for (int k = 0; ok && k + 1 < T; ++k) {
-    int npan, ntrail;
-    step_tasks(np, k, npan, ntrail);
-    const int ntask = npan + ntrail;
+  for (int k = 0; ok && k < T; ++k) {
+    const StepTasks st = step_tasks(np, k);
+    const int ntask = st.total();
+    const int t_first_trail = st.nmrow + st.npan;  // task index of trailing tile (0, 0)
     if (warp < 4) {
       // ------------------------------------------------ staging and MMA issue
-      // the step's inputs: M_kk published, and every trailing tile of the
-      // previous step landed (so column block k of R is final and the reduce-
-      // adds of consecutive steps reach each element in order)
+      // the step's inputs: M_kk published, and every trailing and inverse-
+      // accumulation tile of the previous step landed (so column block k of R
+      // and block row k of G are final, and the reduce-adds of consecutive
+      // steps reach each element in order)
       if (threadIdx.x == 0) {
         bool w = wait_ge(p, (const int*)&p.sync[3], k + 1);
         if (w && k > 0) {
-          int pn, pt;
-          step_tasks(np, k - 1, pn, pt);
-          w = wait_ge(p, &p.tdone[k - 1], pt);
+          const StepTasks pv = step_tasks(np, k - 1);
+          w = wait_ge(p, &p.tdone[k - 1], pv.ntrail) && wait_ge(p, &p.gdone[k - 1], pv.ngupd);
         }
         if (!w) local_abort = 1;
       }
       named_bar_sync(1, 128);
-      bool panels_seen = false;
+      bool panels_seen = false, mrows_seen = false;
       int tl = tcount;
       for (int t = slot; t < ntask && !local_abort; t += W, ++tl) {
-        const Task x = task_of(np, k, t, npan);
-        if (x.kind == 1 && !panels_seen) {
-          // every panel tile of the step (npan by workers, one by CTA 0)
-          if (threadIdx.x == 0 && !wait_ge(p, &p.pdone[k], npan + 1)) local_abort = 1;
+        const Task x = task_of(np, k, t, st);
+        if ((x.kind == 1 || x.kind == 3) && !panels_seen) {
+          // every panel tile of the step (by the workers, and one by CTA 0)
+          if (threadIdx.x == 0 && !wait_ge(p, &p.pdone[k], st.npan + 1)) local_abort = 1;
           named_bar_sync(1, 128);
           panels_seen = true;
+          if (local_abort) break;
+        }
+        if (x.kind == 3 && !mrows_seen) {
+          // block row k of M
+          if (threadIdx.x == 0 && !wait_ge(p, &p.mrdone[k], st.nmrow)) local_abort = 1;
+          named_bar_sync(1, 128);
+          mrows_seen = true;
           if (local_abort) break;
         }
         // the previous task's MMAs have read the staged operands
@@ -738,12 +784,24 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           local_abort = 1;
           break;
         }
-        if (x.kind == 0) {
-          stage_fp32(SAh, SAl, p.R, np, x.r0, x.c0, np);
-          stage_split(SBh, SBl, p.Mh, p.Ml, np, x.c0, FB, x.c0, np);
-        } else {
-          stage_split(SAh, SAl, p.Lh, p.Ll, np, x.c0, 128, (int64_t)FB * k, np);
-          if (!x.diag) stage_split(SBh, SBl, p.Lh, p.Ll, np, x.r0, 128, (int64_t)FB * k, np);
+        const int64_t kc = (int64_t)FB * k;  // k range of every product: block column k
+        switch (x.kind) {
+          case 0:  // L_ik = R_ik M_kk^T
+            stage_fp32(SAh, SAl, p.R, np, x.r0, kc, np);
+            stage_split(SBh, SBl, p.Mh, p.Ml, np, kc, FB, kc, np);
+            break;
+          case 1:  // (L L^T)[c][r]
+            stage_split(SAh, SAl, p.Lh, p.Ll, np, x.c0, 128, kc, np);
+            if (!x.diag) stage_split(SBh, SBl, p.Lh, p.Ll, np, x.r0, 128, kc, np);
+            break;
+          case 2:  // (M_kk G_kj)[r][c] as D[c][r] = sum_t Gt[c][t] M_kk[r][t]
+            stage_fp32(SAh, SAl, p.Gt, np, x.c0, kc, np);
+            stage_split(SBh, SBl, p.Mh, p.Ml, np, kc, FB, kc, np);
+            break;
+          default:  // (L_ik M_kj)[i][c] = sum_t L[i][t] Mt[c][t]
+            stage_split(SAh, SAl, p.Lh, p.Ll, np, x.r0, 128, kc, np);
+            stage_split(SBh, SBl, p.Mth, p.Mtl, np, x.c0, 128, kc, np);
+            break;
         }
         cp_async_commit();
         cp_async_wait<0>();
@@ -758,14 +816,9 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           } else {
             tc_fence_after();
             const uint32_t d = tbase + (uint32_t)buf * 128;
-            if (x.kind == 0) {
-              // D[r][c] = sum_t R[r][t] M[c][t]: lanes = rows, N = 64 columns
-              issue_mma(d, aH, aL, bH, bL, make_idesc(2, 128, 64));
-            } else {
-              // D[c][r] = sum_t L[c][t] L[r][t]: lanes = columns, N = 128 rows
-              const uint32_t b_hi = x.diag ? aH : bH, b_lo = x.diag ? aL : bL;
-              issue_mma(d, aH, aL, b_hi, b_lo, make_idesc(2, 128, 128));
-            }
+            const bool same = x.kind == 1 && x.diag;
+            const uint32_t n = (x.kind == 0 || x.kind == 2) ? 64u : 128u;
+            issue_mma(d, aH, aL, same ? aH : bH, same ? aL : bL, make_idesc(2, 128, n));
             umma_commit(&smem_free);
             umma_commit(&acc_full[buf]);
           }
@@ -778,7 +831,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       const int cl = quarter * 32 + lane;
       int tl = tcount;
       for (int t = slot; t < ntask; t += W, ++tl) {
-        const Task x = task_of(np, k, t, npan);
+        const Task x = task_of(np, k, t, st);
         const int buf = tl & 1;
         if (!mbar_wait_sleep(&acc_full[buf], (tl >> 1) & 1)) {
           give_up(p);
@@ -787,22 +840,30 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
         }
         tc_fence_after();
         const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
-        if (x.kind == 0) {
-          const int64_t r = x.r0 + quarter * 32 + lane;
+        if (x.kind == 0 || x.kind == 2) {
+          // 64 accumulator columns per lane, stored split with vector stores:
+          //   kind 0  lane = row r of L, Lh/Ll[r][64k + n]
+          //   kind 2  lane = column c of M, Mth/Mtl[c][64k + n] = -D
+          //           (columns of block k and past it are not this task's)
+          const int64_t row = (x.kind == 0 ? x.r0 : x.c0) + cl;
+          const bool live = row < np && (x.kind == 0 || row < (int64_t)FB * k);
+          float* const bh = x.kind == 0 ? p.Lh : p.Mth;
+          float* const bl = x.kind == 0 ? p.Ll : p.Mtl;
+          const float sg = x.kind == 0 ? 1.f : -1.f;
 #pragma unroll
           for (int n0 = 0; n0 < FB; n0 += 32) {
             float v[32];
             tmem_ld32(taddr + (uint32_t)n0, v);
-            if (r < np) {
-              float* dh = p.Lh + r * np + x.c0 + n0;
-              float* dl = p.Ll + r * np + x.c0 + n0;
+            if (live) {
+              float* dh = bh + row * np + (int64_t)FB * k + n0;
+              float* dl = bl + row * np + (int64_t)FB * k + n0;
 #pragma unroll
               for (int j = 0; j < 32; j += 4) {
                 float4 h, l;
-                split_tf32(v[j + 0], h.x, l.x);
-                split_tf32(v[j + 1], h.y, l.y);
-                split_tf32(v[j + 2], h.z, l.z);
-                split_tf32(v[j + 3], h.w, l.w);
+                split_tf32(sg * v[j + 0], h.x, l.x);
+                split_tf32(sg * v[j + 1], h.y, l.y);
+                split_tf32(sg * v[j + 2], h.z, l.z);
+                split_tf32(sg * v[j + 3], h.w, l.w);
                 *reinterpret_cast<float4*>(dh + j) = h;
                 *reinterpret_cast<float4*>(dl + j) = l;
               }
@@ -813,39 +874,54 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           named_bar_sync(2, 128);
           if (threadIdx.x == 128) {
             __threadfence();
-            atomicAdd(&p.pdone[k], 1);
+            atomicAdd(x.kind == 0 ? &p.pdone[k] : &p.mrdone[k], 1);
           }
         } else {
-          // R -= D by TMA reduce-add in L2, 32 rows per pass through one of
-          // kStages staging tiles; elements outside the update (above
-          // the diagonal, in block (k+1, k+1), past the matrix) add zero
+          // TMA reduce-add in L2, 32 accumulator columns per pass through one
+          // of kStages staging tiles; elements outside the update add zero:
+          //   kind 1  R[r][c] -= D[c][r] (lane = column c): above the diagonal,
+          //           block (k+1, k+1) and past the matrix excluded;
+          //   kind 3  Gt[c][i] += D[i][c] (lane = row i of G): columns from
+          //           block k + 1 on and rows past the matrix excluded.
           const int64_t s = (int64_t)FB * (k + 1);
-          const int64_t c = x.c0 + cl;
+          const int64_t lane_idx = (x.kind == 1 ? x.c0 : x.r0) + cl;
 #pragma unroll 1
           for (int pz = 0; pz < 4; ++pz) {
             float v[32];
             tmem_ld32(taddr + (uint32_t)(32 * pz), v);
-            const int64_t rb = x.r0 + 32 * pz;
+            const int64_t nb = (x.kind == 1 ? x.r0 : x.c0) + 32 * pz;
             float* sb = stg + (epi_pass % kStages) * (32 * 128);
             if (threadIdx.x == 128) bulk_wait_read<kStages - 1>();  // the reduce that last read sb is done
             named_bar_sync(2, 128);
+            if (x.kind == 1) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int64_t r = rb + j;
-              const bool kp = r < np && c <= r && !(r < s + FB && c < s + FB);
-              sb[j * 128 + cl] = kp ? -v[j] : 0.f;
+              for (int j = 0; j < 32; ++j) {
+                const int64_t r = nb + j, c = lane_idx;
+                const bool kp = r < np && c <= r && !(r < s + FB && c < s + FB);
+                sb[j * 128 + cl] = kp ? -v[j] : 0.f;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const int64_t c = nb + j, i = lane_idx;
+                const bool kp = i < np && c < s;
+                sb[j * 128 + cl] = kp ? v[j] : 0.f;
+              }
             }
             fence_proxy_async_smem();
             named_bar_sync(2, 128);
             if (threadIdx.x == 128) {
-              tma_reduce_add_2d(&rmap, sb, (int32_t)x.c0, (int32_t)rb);
+              if (x.kind == 1)
+                tma_reduce_add_2d(&rmap, sb, (int32_t)x.c0, (int32_t)nb);
+              else
+                tma_reduce_add_2d(&gmap, sb, (int32_t)x.r0, (int32_t)nb);
               bulk_commit();
             }
             ++epi_pass;
           }
           tc_fence_before();
           mbar_arrive(&acc_empty[buf]);
-          if (t == npan && threadIdx.x == 128) {
+          if (t == t_first_trail && threadIdx.x == 128) {
             // trailing tile (0, 0) holds the chain's next two tiles
             bulk_wait_all();
             fence_proxy_async_global();
@@ -857,12 +933,17 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
     }
     if (threadIdx.x == 128) {
       // this CTA's reduce-adds of the step have landed: count them
-      int mine = 0;
-      for (int t = slot; t < ntask; t += W) mine += t >= npan;
+      int mine_t = 0, mine_g = 0;
+      for (int t = slot; t < ntask; t += W) {
+        const int kd = task_of(np, k, t, st).kind;
+        mine_t += kd == 1;
+        mine_g += kd == 3;
+      }
       bulk_wait_all();
       fence_proxy_async_global();
       __threadfence();
-      if (mine) atomicAdd(&p.tdone[k], mine);
+      if (mine_t) atomicAdd(&p.tdone[k], mine_t);
+      if (mine_g) atomicAdd(&p.gdone[k], mine_g);
     }
     // both groups walked the same task list
     for (int t = slot; t < ntask; t += W) ++tcount;
@@ -892,15 +973,15 @@ size_t chain_smem_bytes() {
 
 size_t chol_smem_bytes() { return 1024 + std::max<size_t>(kWorkerSmem, chain_smem_bytes()); }
 
-size_t chol_sync_bytes(int64_t np_) { return sizeof(int) * (size_t)(3 * (np_ / FB) + 4); }
+size_t chol_sync_bytes(int64_t np_) { return sizeof(int) * (size_t)(5 * (np_ / FB) + 4); }
 
 namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// R (np x np fp32, row-major) as a 2-D tensor with 128-column x 32-row boxes,
-// for the trailing update's reduce-add.
+// An np x np fp32 row-major matrix (R, G^T) as a 2-D tensor with 128-column x
+// 32-row boxes, for the reduce-add epilogues.
 bool make_r_map(CUtensorMap* m, float* R, int64_t np_) {
   static EncodeTiledFn fn = [] {
     void* f = nullptr;
@@ -922,7 +1003,7 @@ bool make_r_map(CUtensorMap* m, float* R, int64_t np_) {
 }  // namespace
 
 cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, float* Ml, float* Mth, float* Mtl,
-                        unsigned* sync, uint32_t* status, int sms, cudaStream_t st) {
+                        float* Gt, unsigned* sync, uint32_t* status, int sms, cudaStream_t st) {
   const size_t smem = chol_smem_bytes();
   cudaError_t e = ensure_smem_limit((const void*)chol_kernel, (int)smem);
   if (e != cudaSuccess) return e;
@@ -934,9 +1015,10 @@ cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, 
   e = cudaMemsetAsync(sync, 0, chol_sync_bytes(np_), st);
   if (e != cudaSuccess) return e;
   // workers: enough for the first step's tasks (at most one CTA per SM)
-  const int64_t m = (np_ - FB + 127) / 128;
-  const int64_t tasks0 = (np_ - 2 * FB + 127) / 128 + m * (m + 1) / 2;
-  const int grid = (int)std::max<int64_t>(2, std::min<int64_t>(sms, 1 + tasks0));
+  // workers: enough for the busiest step's tasks (at most one CTA per SM)
+  int most = 1;
+  for (int k = 0; k < T; ++k) most = std::max(most, step_tasks(np_, k).total());
+  const int grid = std::max(2, std::min(sms, 1 + most));
   CholParams p;
   p.R = R;
   p.np_ = np_;
@@ -951,10 +1033,13 @@ cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, 
   p.pdone = (int*)(sync + 4);
   p.tdone = p.pdone + T;
   p.t0done = p.tdone + T;
+  p.mrdone = p.t0done + T;
+  p.gdone = p.mrdone + T;
+  p.Gt = Gt;
   p.status = status;
-  CUtensorMap rmap;
-  if (!make_r_map(&rmap, R, np_)) return cudaErrorInvalidValue;
-  void* args[] = {&rmap, &p};
+  CUtensorMap rmap, gmap;
+  if (!make_r_map(&rmap, R, np_) || !make_r_map(&gmap, Gt, np_)) return cudaErrorInvalidValue;
+  void* args[] = {&rmap, &gmap, &p};
   e = cudaLaunchCooperativeKernel((const void*)chol_kernel, dim3(grid), dim3(FNT), args, smem, st);
   note_launch();
   return e;

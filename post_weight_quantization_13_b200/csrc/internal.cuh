@@ -71,14 +71,16 @@ gptq_status_t hessian_accumulate(float* S, int64_t in, const void* X, gptq_dtype
                                  cudaStream_t st);
 
 // Blocked Cholesky R = L L^T of the np x np matrix R (lower triangle, np a
-// multiple of 128) in one cooperative launch (chol.cu): the panel tiles of L
-// below the 64 x 64 diagonal blocks go to Lh/Ll split (tf32 hi + remainder),
-// the inverses of the diagonal blocks of L to Mh/Ml and, transposed, to
-// Mth/Mtl; R is overwritten.  sync: chol_sync_bytes(np) bytes of scratch.
-// Device-side failures are raised in *status.
+// multiple of 128) and the inverse M = L^-1, in one cooperative launch
+// (chol.cu).  Outputs, split (tf32 hi + exact remainder): the panel tiles of L
+// below the 64 x 64 diagonal blocks in Lh/Ll, the diagonal blocks of M in
+// Mh/Ml, and all of M transposed in Mth/Mtl (Mt[c][r] = M[r][c]).  R and Gt
+// (np x np scratch) are overwritten; Mth, Mtl and Gt must hold zeros on
+// entry.  sync: chol_sync_bytes(np) bytes of scratch.  Device-side failures
+// are raised in *status.
 size_t chol_sync_bytes(int64_t np_);
 cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, float* Ml, float* Mth, float* Mtl,
-                        unsigned* sync, uint32_t* status, int sms, cudaStream_t st);
+                        float* Gt, unsigned* sync, uint32_t* status, int sms, cudaStream_t st);
 
 // Make the driver load every kernel gptq_quantize_layer can launch on the
 // current device now, instead of at their first launch.

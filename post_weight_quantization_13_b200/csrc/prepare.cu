@@ -13,30 +13,25 @@
 //
 // The matrix is padded to a multiple of 128 with identity (block-diagonal,
 // so the padding never mixes with the real channels).
-//   Cholesky:  right-looking with 64-wide blocks in one cooperative launch
-//              (chol.cu): one CTA factors and inverts each diagonal block
-//              while the others form the panel L_ik = R_ik M_kk^T and the
-//              trailing update R -= L_ik L_jk^T as 3xTF32 tensor-core tiles.
-//   Inverse:   pairs of already inverted diagonal groups are merged,
-//              M21 = -M22 (L21 M11), doubling the group size each level; all
-//              merges of one level are one batched tensor-core launch on
-//              "split" operands (hi rounded to tf32 plus the exact fp32
-//              remainder, 3xTF32 accuracy).
+//   Cholesky and inverse: right-looking with 64-wide blocks in one
+//              cooperative launch (chol.cu): one CTA factors and inverts each
+//              diagonal block while the others form, as 3xTF32 tensor-core
+//              tiles on split operands (hi rounded to tf32 plus the exact
+//              fp32 remainder), the panel L_ik = R_ik M_kk^T, the trailing
+//              update R -= L_ik L_jk^T and, block row by block row, the
+//              inverse M = L^-1.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <algorithm>
 #include <cstdlib>
-#include <vector>
 
-#include "gemm.cuh"
 #include "internal.cuh"
 
 namespace gptq {
 namespace {
 
 constexpr int NB = 128;
-constexpr int FB = 64;  // diagonal blocks of the factorisation (chol.cu)
 
 // ------------------------------------------------------------------ diag
 // One CTA: hd[i] = fixed diagonal of H in double, hd = c * S_ii with
@@ -134,34 +129,6 @@ __global__ void __launch_bounds__(256) gather_kernel(const float* __restrict__ S
   }
 }
 
-// Mt[o1 + c][o2 + r] = M[o2 + r][o1 + c] for the merged blocks of one level.
-__global__ void __launch_bounds__(256) transpose_blocks_kernel(const float* __restrict__ Mh,
-                                                               const float* __restrict__ Ml, float* __restrict__ Th,
-                                                               float* __restrict__ Tl, int64_t np_, int64_t o1,
-                                                               int64_t o2, int64_t s1, int64_t s2,
-                                                               int64_t stride) {
-  __shared__ float th[32][33], tl[32][33];
-  const int64_t b = blockIdx.z;
-  const int64_t r0 = (int64_t)blockIdx.y * 32, c0 = (int64_t)blockIdx.x * 32;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 32 x 8
-  const int64_t O1 = o1 + b * stride, O2 = o2 + b * stride;
-  for (int y = ty; y < 32; y += 8) {
-    const int64_t r = r0 + y, c = c0 + tx;
-    if (r < s2 && c < s1) {
-      th[y][tx] = Mh[(O2 + r) * np_ + O1 + c];
-      tl[y][tx] = Ml[(O2 + r) * np_ + O1 + c];
-    }
-  }
-  __syncthreads();
-  for (int y = ty; y < 32; y += 8) {
-    const int64_t c = c0 + y, r = r0 + tx;
-    if (r < s2 && c < s1) {
-      Th[(O1 + c) * np_ + O2 + r] = th[tx][y];
-      Tl[(O1 + c) * np_ + O2 + r] = tl[tx][y];
-    }
-  }
-}
-
 // U (column-major, in x in): U_cm[x][y] = Mt[in-1-x][in-1-y] for y <= x, 0 above.
 // U[x][y] = M[in-1-y][in-1-x] = Mt[in-1-x][in-1-y] for y <= x (U = J M J with
 // J the reversal), 0 above.  Rows of Mt are read backwards; with in % 4 == 0
@@ -198,18 +165,13 @@ __global__ void __launch_bounds__(256) write_u_kernel(const float* __restrict__ 
   }
 }
 
-cudaError_t run_gemm(GemmArgs& g, cudaStream_t st, int sms) {
-  if (!force_simt() && tc_gemm_supported(g)) return tc_gemm(g, st, sms);
-  return simt_gemm(g, st);
-}
-
 }  // namespace
 
 size_t prepare_ws_bytes(int64_t in) {
   const int64_t np_ = round_up(in, NB);
   size_t b = kHeaderBytes;
   b += round_up((int64_t)sizeof(double) * in, 256);              // hd
-  b += 9 * round_up((int64_t)sizeof(float) * np_ * np_, 256);    // R; L, M, Mt, X^T (hi, lo)
+  b += 8 * round_up((int64_t)sizeof(float) * np_ * np_, 256);    // R; L, M, Mt (hi, lo); G^T
   b += round_up((int64_t)chol_sync_bytes(np_), 256);             // barrier and panel counters
   return b;
 }
@@ -231,12 +193,11 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
   float* Ml = (float*)p; p += mat;
   float* Mth = (float*)p; p += mat;
   float* Mtl = (float*)p; p += mat;
-  float* Xh = (float*)p; p += mat;
-  float* Xl = (float*)p; p += mat;
+  float* Gt = (float*)p; p += mat;     // the inverse's accumulator, transposed
   unsigned* sync = (unsigned*)p;  // barrier, then the panel counters
 
   CUDA_TRY(cudaMemsetAsync(hdr, 0, kHeaderBytes, st));
-  CUDA_TRY(cudaMemsetAsync(Mh, 0, 4 * mat, st));  // M, Mt (hi, lo): strictly-off-triangle blocks stay 0
+  CUDA_TRY(cudaMemsetAsync(Mth, 0, 3 * mat, st));  // Mt (hi, lo): zeros above the diagonal; G^T starts at 0
   const double c = 2.0 / (double)n;
   const float scale = (float)c;
   diag_kernel<<<1, 1024, 0, st>>>(S, in, c, cfg->damp_percent, hd, dead, hdr);
@@ -251,89 +212,8 @@ gptq_status_t prepare_hinv(const float* S, int64_t n, int64_t in, const gptq_con
     note_launch();
     CUDA_TRY(cudaGetLastError());
   }
-  // blocked Cholesky of R with the inverses of its 64 x 64 diagonal blocks
-  CUDA_TRY(chol_factor(R, np_, Lh, Ll, Mh, Ml, Mth, Mtl, sync, &hdr->status, dev.sms, st));
-  // triangular inverse: merge groups pairwise, M21 = -M22 (L21 M11)
-  auto merge = [&](std::vector<std::pair<int64_t, int64_t>> groups) -> gptq_status_t {  // (offset, size)
-  while (groups.size() > 1) {
-    std::vector<std::pair<int64_t, int64_t>> next;
-    size_t i = 0;
-    while (i + 1 < groups.size()) {
-      // batch consecutive pairs with identical sizes
-      const int64_t s1 = groups[i].second, s2 = groups[i + 1].second;
-      size_t j = i;
-      int nb = 0;
-      while (j + 1 < groups.size() && groups[j].second == s1 && groups[j + 1].second == s2 &&
-             (nb == 0 || groups[j].first == groups[i].first + (int64_t)nb * (s1 + s2))) {
-        next.push_back({groups[j].first, s1 + s2});
-        j += 2;
-        ++nb;
-      }
-      const int64_t o1 = groups[i].first, o2 = o1 + s1, stride = s1 + s2;
-      // X^T[o1+c][o2+r] = (L21 M11)[r][c] = sum_t L[o2+r][o1+t] Mt[o1+c][o1+t]
-      GemmArgs a;
-      a.op = OP_TF32X3;
-      a.P = {Lh, Ll, np_, np_, np_};
-      a.Q = {Mth, Mtl, np_, np_, np_};
-      a.R = s2;
-      a.Cn = s1;
-      a.K = s1;
-      a.p_row0 = o2;
-      a.p_k0 = o1;
-      a.q_row0 = o1;
-      a.q_k0 = o1;
-      a.C = Xh;
-      a.C_lo = Xl;
-      a.ldc = np_;
-      a.c_row0 = o1;  // transposed store: row o1 + c, col o2 + r
-      a.c_col0 = o2;
-      a.alpha = 1.f;
-      a.beta = 0.f;
-      a.transpose = 1;
-      a.batch = nb;
-      a.bs_p_row = stride;
-      a.bs_p_k = stride;
-      a.bs_q_row = stride;
-      a.bs_q_k = stride;
-      a.bs_c_row = stride;
-      a.bs_c_col = stride;
-      a.status = &hdr->status;
-      CUDA_TRY(run_gemm(a, st, dev.sms));
-      // M21[r][c] = -sum_t M[o2+r][o2+t] X^T[o1+c][o2+t]
-      GemmArgs b = a;
-      b.P = {Mh, Ml, np_, np_, np_};
-      b.Q = {Xh, Xl, np_, np_, np_};
-      b.R = s2;
-      b.Cn = s1;
-      b.K = s2;
-      b.p_row0 = o2;
-      b.p_k0 = o2;
-      b.q_row0 = o1;
-      b.q_k0 = o2;
-      b.C = Mh;
-      b.C_lo = Ml;
-      b.c_row0 = o2;
-      b.c_col0 = o1;
-      b.alpha = -1.f;
-      b.transpose = 0;
-      CUDA_TRY(run_gemm(b, st, dev.sms));
-      dim3 tg((unsigned)((s1 + 31) / 32), (unsigned)((s2 + 31) / 32), (unsigned)nb);
-      transpose_blocks_kernel<<<tg, 256, 0, st>>>(Mh, Ml, Mth, Mtl, np_, o1, o2, s1, s2, stride);
-      note_launch();
-      CUDA_TRY(cudaGetLastError());
-      i = j;
-    }
-    if (i < groups.size()) next.push_back(groups[i]);
-    groups.swap(next);
-  }
-  return GPTQ_OK;
-  };
-  {
-    std::vector<std::pair<int64_t, int64_t>> groups;
-    for (int64_t o = 0; o < np_; o += FB) groups.push_back({o, FB});
-    gptq_status_t ms = merge(groups);
-    if (ms != GPTQ_OK) return ms;
-  }
+  // blocked Cholesky of R and the inverse M = L^-1 (transposed in Mth/Mtl)
+  CUDA_TRY(chol_factor(R, np_, Lh, Ll, Mh, Ml, Mth, Mtl, Gt, sync, &hdr->status, dev.sms, st));
   {
     const unsigned grid = (unsigned)std::min<int64_t>(in, (int64_t)dev.sms * 8);
     write_u_kernel<<<grid, 256, 0, st>>>(Mth, Mtl, np_, in, U);
