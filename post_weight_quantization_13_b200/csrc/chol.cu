@@ -18,7 +18,8 @@
 //                       is written, the trailing update R_ij -= L_ik L_jk^T
 //                       of the lower triangle from block k+1 on, in 128 x 128
 //                       tiles (block (k+1, k+1) excluded: CTA 0 updates it).
-// Products on the chain CTA are 64 x 64 x 64 and stay on CUDA cores.
+// The chain CTA's two 64 x 64 x 64 products run on the tensor cores too
+// (M = 128 with zero rows), the leaf on CUDA cores.
 //
 // Worker CTAs: warps 0-3 stage the operands of a task in shared memory in
 // the tensor core's 128-byte-swizzled K-major layout (split fp32: tf32 hi
@@ -51,6 +52,11 @@ constexpr uint32_t kStageBytes = 32 * 128 * 4;      // one epilogue pass: 32 row
 constexpr int kStages = 4;                           // epilogue staging buffers (one per 32-row pass)
 constexpr uint32_t kWorkerSmem = 4 * kRegionBytes + kStages * kStageBytes;  // 192 KB
 constexpr uint32_t kTmemCols = 256;                 // two 128-column accumulators
+// chain CTA: fp32 tiles, then (1024-aligned) the tensor-core operand regions
+constexpr uint32_t kChainFloats = 4 * FB * TP + 2 * FB * FP + 32 * FP + FB * 64 + FB + 4;
+constexpr uint32_t kChainOpOffset = (kChainFloats * 4 + 1023) / 1024 * 1024;
+constexpr uint32_t kChainOpABytes = 2 * 2 * 128 * 128;  // 128 rows x K 64, hi and lo
+constexpr uint32_t kChainOpBBytes = 2 * 2 * 64 * 128;   // 64 rows x K 64, hi and lo
 
 struct CholParams {
   float* R;        // np x np (lower triangle used), updated in place
@@ -139,42 +145,6 @@ __device__ __forceinline__ int ld_acquire_cta(const int* p) {
 }
 
 // ------------------------------------------------------------------ chain CTA
-// S[r][t] (pitch TP) <- G[r][t] for an FB x FB tile (row stride ld), async.
-__device__ __forceinline__ void prefetch_tile(float* S, const float* G, int64_t ld) {
-  for (int e = threadIdx.x; e < FB * FB / 4; e += FNT) {
-    const int r = e / (FB / 4), t4 = (e % (FB / 4)) * 4;
-    cp_async16(S + r * TP + t4, G + (int64_t)r * ld + t4);
-  }
-}
-
-// acc[u][v] = sum_t X[tr + 16u][t] Y[tc + 16v][t]   (tr = tid / 16, tc = tid % 16)
-// X, Y row-major tiles of pitch TP.  Output rows and columns are strided by
-// 16 so that the 16 column groups of a warp read 16 consecutive rows of Y.
-__device__ __forceinline__ void tile_product(const float* X, const float* Y, float acc[4][4]) {
-  const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
-#pragma unroll
-  for (int u = 0; u < 4; ++u)
-#pragma unroll
-    for (int v = 0; v < 4; ++v) acc[u][v] = 0.f;
-#pragma unroll 2
-  for (int t = 0; t < FB; t += 4) {
-    float4 x[4], y[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) x[u] = *reinterpret_cast<const float4*>(X + (tr + 16 * u) * TP + t);
-#pragma unroll
-    for (int v = 0; v < 4; ++v) y[v] = *reinterpret_cast<const float4*>(Y + (tc + 16 * v) * TP + t);
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        acc[u][v] = fmaf(x[u].x, y[v].x, acc[u][v]);
-        acc[u][v] = fmaf(x[u].y, y[v].y, acc[u][v]);
-        acc[u][v] = fmaf(x[u].z, y[v].z, acc[u][v]);
-        acc[u][v] = fmaf(x[u].w, y[v].w, acc[u][v]);
-      }
-  }
-}
-
 // The leaf: A (FB x FB, pitch FP, lower triangle read) -> M = L^-1 (pitch FP,
 // zeros above the diagonal), where A = L L^T.  Six warps, each a chain of
 // pivots over registers, fed through shared memory:
@@ -508,6 +478,24 @@ __device__ __forceinline__ void stage_fp32(uint8_t* Shi, uint8_t* Slo, const flo
   }
 }
 
+// 24 MMAs: D (+)= A B^T over K = 64 with split operands (hi hi + hi lo + lo hi);
+// the operands' two K chunks are a_chunk / b_chunk bytes apart.
+__device__ __forceinline__ void issue_mma_strided(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t a_chunk,
+                                                  uint32_t b_hi, uint32_t b_lo, uint32_t b_chunk, uint32_t idesc) {
+#pragma unroll
+  for (int ch = 0; ch < 2; ++ch)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const uint64_t ah = smem_desc_k_sw128(a_hi + ch * a_chunk + kk * 32);
+      const uint64_t al = smem_desc_k_sw128(a_lo + ch * a_chunk + kk * 32);
+      const uint64_t bh = smem_desc_k_sw128(b_hi + ch * b_chunk + kk * 32);
+      const uint64_t bl = smem_desc_k_sw128(b_lo + ch * b_chunk + kk * 32);
+      umma_tf32(d, ah, bh, idesc, (ch | kk) ? 1u : 0u);
+      umma_tf32(d, ah, bl, idesc, 1u);
+      umma_tf32(d, al, bh, idesc, 1u);
+    }
+}
+
 // 24 MMAs: D (+)= A B^T over K = 64 with split operands (hi hi + hi lo + lo hi).
 __device__ __forceinline__ void issue_mma(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi, uint32_t b_lo,
                                           uint32_t idesc) {
@@ -600,9 +588,15 @@ __device__ __forceinline__ Task task_of(int64_t np, int k, int t, const StepTask
   return x;
 }
 
+// Operand loads by TMA: the split panel columns of L and of M^T, boxes of 32
+// columns (one 128-byte swizzled K chunk) by 128 rows.
+struct OpMaps {
+  CUtensorMap lh, ll, mth, mtl;
+};
+
 __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CUtensorMap rmap,
                                                       const __grid_constant__ CUtensorMap gmap,
-                                                      const CholParams p) {
+                                                      const __grid_constant__ OpMaps om, const CholParams p) {
   extern __shared__ __align__(1024) uint8_t csm_raw[];
   uint8_t* csm = (uint8_t*)(((uintptr_t)csm_raw + 1023) & ~(uintptr_t)1023);
   const int64_t np = p.np_;
@@ -615,16 +609,62 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
     float* fsm = reinterpret_cast<float*>(csm);
     float* Xb2 = fsm;                // [2][FB][TP] R_{k+1,k} (double-buffered across steps)
     float* Cb2 = Xb2 + 2 * FB * TP;  // [2][FB][TP] R_{k+1,k+1}
-    float* Yb = Cb2 + 2 * FB * TP;   // [FB][TP] M_kk
-    float* LT = Yb + FB * TP;        // [FB][TP] L_{k+1,k}
-    float* A = LT + FB * TP;         // [FB][FP]
+    float* A = Cb2 + 2 * FB * TP;    // [FB][FP]
     float* M = A + FB * FP;          // [FB][FP]
     float* Xs = M + FB * FP;         // [32][FP] scratch of the leaf's merge
     float* Lc = Xs + 32 * FP;        // [FB][LCP] columns of L (leaf), 16-byte aligned
     float* rdiag = Lc + FB * LCP;    // [FB]
     int* fl = reinterpret_cast<int*>(rdiag + FB);
-    const int tr = threadIdx.x / 16, tc = threadIdx.x % 16;
+    // tensor-core operands of the chain's two products (split, 128-byte
+    // swizzled, K = 64 in two chunks): OPA 128 rows (rows 64..127 stay zero,
+    // the MMA's M is 128), OPB 64 rows
+    uint8_t* OPA = csm + kChainOpOffset;
+    uint8_t* OPB = OPA + kChainOpABytes;
+    constexpr uint32_t kAChunk = 128 * 128, kBChunk = 64 * 128;
+    __shared__ uint64_t cbar;
+    __shared__ uint32_t ctmem;
+    const int warp = threadIdx.x >> 5;
+    if (threadIdx.x == 0) {
+      mbar_init(&cbar, 1);
+      fence_mbar_init();
+    }
+    if (warp == 0) {
+      tmem_alloc(&ctmem, 128);
+      tmem_relinquish();
+    }
+    for (int e = threadIdx.x; e < (int)(kChainOpABytes / 16); e += FNT) {
+      // zero OPA (rows 64..127 are never written again)
+      reinterpret_cast<float4*>(OPA)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t ctb = ctmem;
+    const uint32_t oah = smem_u32(OPA), oal = oah + 2 * kAChunk;
+    const uint32_t obh = smem_u32(OPB), obl = obh + 2 * kBChunk;
+    uint32_t cphase = 0;
     auto tile = [&](int i, int j) { return p.R + (int64_t)i * FB * np + (int64_t)j * FB; };
+    // one 64-row operand into a region: element (r, t) of a row-major source
+    // with pitch ld, split, at row r of the swizzled K-major layout
+    auto stage_op = [&](uint8_t* dst, uint32_t chunk, const float* src, int ld) {
+      for (int e = threadIdx.x; e < FB * 16; e += FNT) {
+        const int r = e >> 4, g = e & 15;
+        const float* q = src + r * ld + 4 * g;
+        float4 h, l;
+        split_tf32(q[0], h.x, l.x);
+        split_tf32(q[1], h.y, l.y);
+        split_tf32(q[2], h.z, l.z);
+        split_tf32(q[3], h.w, l.w);
+        const uint32_t so = (g >> 3) * chunk + sw128(r, g & 7);
+        *reinterpret_cast<float4*>(dst + so) = h;
+        *reinterpret_cast<float4*>(dst + 2 * chunk + so) = l;
+      }
+    };
+    auto mma_wait = [&]() {
+      if (!mbar_wait(&cbar, cphase)) give_up(p);
+      cphase ^= 1;
+      tc_fence_after();
+    };
     // the next step's tiles, for warp 7 during the leaf of step k (k = -1:
     // the first diagonal block's leaf, whose next tiles no one updates)
     auto next_tiles = [&](int k) {
@@ -641,6 +681,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       return nt;
     };
     auto publish_m = [&](int count) {
+      fence_proxy_async_global();  // workers read M_kk^T by TMA
       __syncthreads();
       if (threadIdx.x == 0) {
         __threadfence();
@@ -656,50 +697,86 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
     if (!leaf64(A, M, Xs, Lc, rdiag, fl, p, next_tiles(-1))) give_up(p);
     store_diag_m(p, M, 0);
     publish_m(1);
+    const uint32_t idesc = make_idesc(2, 128, 64);
     for (int k = 0; k + 1 < T && !aborted(p); ++k) {
-      float acc[4][4];
       const float* Xb = Xb2 + (k & 1) * FB * TP;
       const float* Cb = Cb2 + (k & 1) * FB * TP;
-      // this step's tiles arrived during the previous leaf (warp 7 waited for
-      // its copies before the leaf's closing barrier)
-      for (int e = threadIdx.x; e < FB * FB; e += FNT) {
-        const int r = e / FB, c = e % FB;
-        Yb[r * TP + c] = M[r * FP + c];
-      }
-      __syncthreads();
-      // L_{k+1,k} = R_{k+1,k} M_kk^T, published split for the workers
-      tile_product(Xb, Yb, acc);
-      {
-        const int64_t base = (int64_t)(k + 1) * FB * np + (int64_t)k * FB;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int r = tr + 16 * u, c = tc + 16 * v;
-            float h, l;
-            split_tf32(acc[u][v], h, l);
-            p.Lh[base + (int64_t)r * np + c] = h;
-            p.Ll[base + (int64_t)r * np + c] = l;
-            LT[r * TP + c] = acc[u][v];
-          }
-      }
+      // L_{k+1,k} = R_{k+1,k} M_kk^T on the tensor cores: D1[r][c] =
+      // sum_t X[r][t] M[c][t], lanes = rows of X (this step's tiles arrived
+      // during the previous leaf: warp 7 waited for its copies before the
+      // leaf's closing barrier)
+      stage_op(OPA, kAChunk, Xb, TP);
+      stage_op(OPB, kBChunk, M, FP);
+      fence_proxy_async_smem();
       __syncthreads();
       if (threadIdx.x == 0) {
+        tc_fence_after();
+        issue_mma_strided(ctb, oah, oal, kAChunk, obh, obl, kBChunk, idesc);
+        umma_commit(&cbar);
+      }
+      mma_wait();
+      if (warp < 2) {
+        // lane r: row r of L, published split for the workers and staged as
+        // the operand of L L^T
+        const int r = threadIdx.x;
+        const uint32_t ta = ctb + ((uint32_t)(32 * warp) << 16);
+        float* gh = p.Lh + (int64_t)((k + 1) * FB + r) * np + (int64_t)k * FB;
+        float* gl = p.Ll + (int64_t)((k + 1) * FB + r) * np + (int64_t)k * FB;
+#pragma unroll
+        for (int n0 = 0; n0 < FB; n0 += 32) {
+          float v[32];
+          tmem_ld32(ta + (uint32_t)n0, v);
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            float4 h, l;
+            split_tf32(v[j + 0], h.x, l.x);
+            split_tf32(v[j + 1], h.y, l.y);
+            split_tf32(v[j + 2], h.z, l.z);
+            split_tf32(v[j + 3], h.w, l.w);
+            *reinterpret_cast<float4*>(gh + n0 + j) = h;
+            *reinterpret_cast<float4*>(gl + n0 + j) = l;
+            const int g = (n0 + j) >> 2;
+            const uint32_t so = (g >> 3) * kAChunk + sw128(r, g & 7);
+            *reinterpret_cast<float4*>(OPA + so) = h;
+            *reinterpret_cast<float4*>(OPA + 2 * kAChunk + so) = l;
+          }
+        }
+        fence_proxy_async_smem();
+        fence_proxy_async_global();  // workers read L_{k+1,k} by TMA
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        // L L^T: both operands are L (the first 64 rows of OPA)
+        tc_fence_after();
+        issue_mma_strided(ctb + 64, oah, oal, kAChunk, oah, oal, kAChunk, idesc);
+        umma_commit(&cbar);
+      } else if (threadIdx.x == 32) {
         __threadfence();
         atomicAdd(&p.pdone[k], 1);
       }
-      tile_product(LT, LT, acc);  // L L^T
+      mma_wait();
+      if (warp < 2) {
+        const int r = threadIdx.x;
+        const uint32_t ta = ctb + 64 + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
+        for (int n0 = 0; n0 < FB; n0 += 32) {
+          float v[32];
+          tmem_ld32(ta + (uint32_t)n0, v);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int r = tr + 16 * u, c = tc + 16 * v;
-          A[r * FP + c] = Cb[r * TP + c] - acc[u][v];
+          for (int j = 0; j < 32; ++j) A[r * FP + n0 + j] = Cb[r * TP + n0 + j] - v[j];
         }
+      }
+      tc_fence_before();
       __syncthreads();
       if (!leaf64(A, M, Xs, Lc, rdiag, fl, p, next_tiles(k))) give_up(p);
       store_diag_m(p, M, k + 1);
       publish_m(k + 2);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(ctb, 128);
     }
     return;
   }
@@ -710,7 +787,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   uint8_t* SBh = SAl + kRegionBytes;
   uint8_t* SBl = SBh + kRegionBytes;
   float* stg = reinterpret_cast<float*>(SBl + kRegionBytes);  // [kStages][32][128] epilogue staging
-  __shared__ uint64_t smem_free, acc_full[2], acc_empty[2], drain;
+  __shared__ uint64_t smem_free, acc_full[2], acc_empty[2], drain, op_full;
   __shared__ uint32_t tmem_slot;
   __shared__ int local_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -721,6 +798,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       mbar_init(&acc_empty[b], 128);
     }
     mbar_init(&drain, 1);
+    mbar_init(&op_full, 1);
     local_abort = 0;
     fence_mbar_init();
   }
@@ -730,6 +808,10 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
     if (lane == 0) {
       tma_prefetch_desc(&rmap);
       tma_prefetch_desc(&gmap);
+      tma_prefetch_desc(&om.lh);
+      tma_prefetch_desc(&om.ll);
+      tma_prefetch_desc(&om.mth);
+      tma_prefetch_desc(&om.mtl);
     }
   }
   tc_fence_before();
@@ -740,6 +822,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   const uint32_t aH = smem_u32(SAh), aL = smem_u32(SAl), bH = smem_u32(SBh), bL = smem_u32(SBl);
   int tcount = 0;    // tasks of this CTA so far (all steps): drives the barrier phases
   int epi_pass = 0;  // epilogue staging passes (selects the staging buffer)
+  uint32_t op_phase = 0;  // phase of op_full (thread 0: operands loaded by TMA)
   bool ok = true;
   for (int k = 0; ok && k < T; ++k) {
     const StepTasks st = step_tasks(np, k);
@@ -758,6 +841,8 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           w = wait_ge(p, &p.tdone[k - 1], pv.ntrail) && wait_ge(p, &p.gdone[k - 1], pv.ngupd);
         }
         if (!w) local_abort = 1;
+        // operands written by other CTAs' generic stores are read by TMA below
+        fence_proxy_async_global();
       }
       named_bar_sync(1, 128);
       bool panels_seen = false, mrows_seen = false;
@@ -766,14 +851,20 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
         const Task x = task_of(np, k, t, st);
         if ((x.kind == 1 || x.kind == 3) && !panels_seen) {
           // every panel tile of the step (by the workers, and one by CTA 0)
-          if (threadIdx.x == 0 && !wait_ge(p, &p.pdone[k], st.npan + 1)) local_abort = 1;
+          if (threadIdx.x == 0) {
+            if (!wait_ge(p, &p.pdone[k], st.npan + 1)) local_abort = 1;
+            fence_proxy_async_global();
+          }
           named_bar_sync(1, 128);
           panels_seen = true;
           if (local_abort) break;
         }
         if (x.kind == 3 && !mrows_seen) {
           // block row k of M
-          if (threadIdx.x == 0 && !wait_ge(p, &p.mrdone[k], st.nmrow)) local_abort = 1;
+          if (threadIdx.x == 0) {
+            if (!wait_ge(p, &p.mrdone[k], st.nmrow)) local_abort = 1;
+            fence_proxy_async_global();
+          }
           named_bar_sync(1, 128);
           mrows_seen = true;
           if (local_abort) break;
@@ -785,27 +876,43 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           break;
         }
         const int64_t kc = (int64_t)FB * k;  // k range of every product: block column k
-        switch (x.kind) {
-          case 0:  // L_ik = R_ik M_kk^T
+        const bool by_tma = x.kind == 1 || x.kind == 3;
+        if (!by_tma) {
+          if (x.kind == 0) {  // L_ik = R_ik M_kk^T
             stage_fp32(SAh, SAl, p.R, np, x.r0, kc, np);
-            stage_split(SBh, SBl, p.Mh, p.Ml, np, kc, FB, kc, np);
-            break;
-          case 1:  // (L L^T)[c][r]
-            stage_split(SAh, SAl, p.Lh, p.Ll, np, x.c0, 128, kc, np);
-            if (!x.diag) stage_split(SBh, SBl, p.Lh, p.Ll, np, x.r0, 128, kc, np);
-            break;
-          case 2:  // (M_kk G_kj)[r][c] as D[c][r] = sum_t Gt[c][t] M_kk[r][t]
+          } else {  // (M_kk G_kj)[r][c] as D[c][r] = sum_t Gt[c][t] M_kk[r][t]
             stage_fp32(SAh, SAl, p.Gt, np, x.c0, kc, np);
-            stage_split(SBh, SBl, p.Mh, p.Ml, np, kc, FB, kc, np);
-            break;
-          default:  // (L_ik M_kj)[i][c] = sum_t L[i][t] Mt[c][t]
-            stage_split(SAh, SAl, p.Lh, p.Ll, np, x.r0, 128, kc, np);
-            stage_split(SBh, SBl, p.Mth, p.Mtl, np, x.c0, 128, kc, np);
-            break;
+          }
+          stage_split(SBh, SBl, p.Mh, p.Ml, np, kc, FB, kc, np);
+          cp_async_commit();
+          cp_async_wait<0>();
+          fence_proxy_async_smem();
+        } else if (threadIdx.x == 0) {
+          // kind 1: (L L^T)[c][r], A = L rows c, B = L rows r;
+          // kind 3: (L_ik M_kj)[i][c] = sum_t L[i][t] Mt[c][t], A = L rows i,
+          // B = Mt rows c.  Rows past the matrix arrive as zeros.
+          const bool two = !(x.kind == 1 && x.diag);
+          const int32_t ya = (int32_t)(x.kind == 1 ? x.c0 : x.r0);
+          const int32_t yb = (int32_t)(x.kind == 1 ? x.r0 : x.c0);
+          const CUtensorMap* bhm = x.kind == 1 ? &om.lh : &om.mth;
+          const CUtensorMap* blm = x.kind == 1 ? &om.ll : &om.mtl;
+          mbar_arrive_expect_tx(&op_full, (two ? 2u : 1u) * kRegionBytes * 2u);
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            const int32_t xk = (int32_t)(kc + 32 * ch);
+            tma_load_2d(SAh + ch * kChunkBytes, &om.lh, &op_full, xk, ya);
+            tma_load_2d(SAl + ch * kChunkBytes, &om.ll, &op_full, xk, ya);
+            if (two) {
+              tma_load_2d(SBh + ch * kChunkBytes, bhm, &op_full, xk, yb);
+              tma_load_2d(SBl + ch * kChunkBytes, blm, &op_full, xk, yb);
+            }
+          }
+          if (!mbar_wait(&op_full, op_phase)) {
+            give_up(p);
+            local_abort = 1;
+          }
+          op_phase ^= 1;
         }
-        cp_async_commit();
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (threadIdx.x == 0) {
           const int buf = tl & 1;
@@ -869,6 +976,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
               }
             }
           }
+          fence_proxy_async_global();  // other CTAs read these stores by TMA
           tc_fence_before();
           mbar_arrive(&acc_empty[buf]);
           named_bar_sync(2, 128);
@@ -893,21 +1001,27 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
             float* sb = stg + (epi_pass % kStages) * (32 * 128);
             if (threadIdx.x == 128) bulk_wait_read<kStages - 1>();  // the reduce that last read sb is done
             named_bar_sync(2, 128);
+            // the kept entries of a pass are a range of j, [lo, hi)
+            int lo, hi;
+            float sg;
             if (x.kind == 1) {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int64_t r = nb + j, c = lane_idx;
-                const bool kp = r < np && c <= r && !(r < s + FB && c < s + FB);
-                sb[j * 128 + cl] = kp ? -v[j] : 0.f;
-              }
+              // r = nb + j < np, c <= r, and not both r and c in block k + 1
+              const int64_t c = lane_idx;
+              int64_t l = c - nb;
+              if (c < s + FB) l = l > s + FB - nb ? l : s + FB - nb;
+              lo = (int)(l < 0 ? 0 : (l > 32 ? 32 : l));
+              const int64_t h = np - nb;
+              hi = (int)(h < 0 ? 0 : (h > 32 ? 32 : h));
+              sg = -1.f;
             } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const int64_t c = nb + j, i = lane_idx;
-                const bool kp = i < np && c < s;
-                sb[j * 128 + cl] = kp ? v[j] : 0.f;
-              }
+              // column c = nb + j < s, row i < np
+              const int64_t h = lane_idx < np ? s - nb : 0;
+              lo = 0;
+              hi = (int)(h < 0 ? 0 : (h > 32 ? 32 : h));
+              sg = 1.f;
             }
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sb[j * 128 + cl] = (j >= lo && j < hi) ? sg * v[j] : 0.f;
             fence_proxy_async_smem();
             named_bar_sync(2, 128);
             if (threadIdx.x == 128) {
@@ -965,9 +1079,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   }
 }
 
-size_t chain_smem_bytes() {
-  return sizeof(float) * (6 * FB * TP + 2 * FB * FP + 32 * FP + FB * LCP + FB) + 16;
-}
+size_t chain_smem_bytes() { return kChainOpOffset + kChainOpABytes + kChainOpBBytes; }
 
 }  // namespace
 
@@ -980,9 +1092,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-// An np x np fp32 row-major matrix (R, G^T) as a 2-D tensor with 128-column x
-// 32-row boxes, for the reduce-add epilogues.
-bool make_r_map(CUtensorMap* m, float* R, int64_t np_) {
+// An np x np fp32 row-major matrix as a 2-D tensor: 128-column x 32-row boxes
+// without swizzle for the reduce-add epilogues (R, G^T), 32-column x 128-row
+// boxes with 128-byte swizzle for the operand loads (L, M^T; the tensor
+// core's K-major layout).
+bool make_r_map(CUtensorMap* m, float* R, int64_t np_, uint32_t box_x = 128, uint32_t box_y = 32,
+                CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
   static EncodeTiledFn fn = [] {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -994,11 +1109,10 @@ bool make_r_map(CUtensorMap* m, float* R, int64_t np_) {
   if (!fn) return false;
   cuuint64_t gdim[2] = {(cuuint64_t)np_, (cuuint64_t)np_};
   cuuint64_t gstride[1] = {(cuuint64_t)(np_ * 4)};
-  cuuint32_t box[2] = {128, 32};
+  cuuint32_t box[2] = {box_x, box_y};
   cuuint32_t estride[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, R, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 }  // namespace
 
@@ -1039,7 +1153,12 @@ cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, 
   p.status = status;
   CUtensorMap rmap, gmap;
   if (!make_r_map(&rmap, R, np_) || !make_r_map(&gmap, Gt, np_)) return cudaErrorInvalidValue;
-  void* args[] = {&rmap, &gmap, &p};
+  OpMaps om;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_r_map(&om.lh, Lh, np_, 32, 128, sw) || !make_r_map(&om.ll, Ll, np_, 32, 128, sw) ||
+      !make_r_map(&om.mth, Mth, np_, 32, 128, sw) || !make_r_map(&om.mtl, Mtl, np_, 32, 128, sw))
+    return cudaErrorInvalidValue;
+  void* args[] = {&rmap, &gmap, &om, &p};
   e = cudaLaunchCooperativeKernel((const void*)chol_kernel, dim3(grid), dim3(FNT), args, smem, st);
   note_launch();
   return e;
