@@ -128,6 +128,14 @@ __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const 
                "r"(smem_u32(smem_src)), "r"(x), "r"(y)
                : "memory");
 }
+// 2-D tiled bulk tensor store shared -> global (bulk-group completion), clipped
+// at the tensor map's bounds.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+
 // Order this thread's async-proxy global writes (bulk copies it waited for)
 // before its later generic-proxy operations.
 __device__ __forceinline__ void fence_proxy_async_global() {
@@ -496,20 +504,18 @@ __device__ __forceinline__ void issue_mma_strided(uint32_t d, uint32_t a_hi, uin
     }
 }
 
-// 24 MMAs: D (+)= A B^T over K = 64 with split operands (hi hi + hi lo + lo hi).
-__device__ __forceinline__ void issue_mma(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi, uint32_t b_lo,
-                                          uint32_t idesc) {
+// 12 MMAs: D (+)= A B^T over one K chunk of 32 with split operands (hi hi + hi
+// lo + lo hi); accumulate == false starts the accumulator.
+__device__ __forceinline__ void issue_mma_chunk(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
+                                                uint32_t b_lo, uint32_t idesc, bool accumulate) {
 #pragma unroll
-  for (int ch = 0; ch < 2; ++ch)
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk) {
-      const uint32_t off = ch * kChunkBytes + kk * 32;
-      const uint64_t ah = smem_desc_k_sw128(a_hi + off), al = smem_desc_k_sw128(a_lo + off);
-      const uint64_t bh = smem_desc_k_sw128(b_hi + off), bl = smem_desc_k_sw128(b_lo + off);
-      umma_tf32(d, ah, bh, idesc, (ch | kk) ? 1u : 0u);
-      umma_tf32(d, ah, bl, idesc, 1u);
-      umma_tf32(d, al, bh, idesc, 1u);
-    }
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint64_t ah = smem_desc_k_sw128(a_hi + kk * 32), al = smem_desc_k_sw128(a_lo + kk * 32);
+    const uint64_t bh = smem_desc_k_sw128(b_hi + kk * 32), bl = smem_desc_k_sw128(b_lo + kk * 32);
+    umma_tf32(d, ah, bh, idesc, (accumulate || kk) ? 1u : 0u);
+    umma_tf32(d, ah, bl, idesc, 1u);
+    umma_tf32(d, al, bh, idesc, 1u);
+  }
 }
 
 // The tile tasks of step k, in this order:
@@ -592,6 +598,7 @@ __device__ __forceinline__ Task task_of(int64_t np, int k, int t, const StepTask
 // columns (one 128-byte swizzled K chunk) by 128 rows.
 struct OpMaps {
   CUtensorMap lh, ll, mth, mtl;
+  CUtensorMap mth64, mtl64;  // the same with 64-row boxes (a half tile of M^T rows)
 };
 
 __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CUtensorMap rmap,
@@ -660,6 +667,14 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
         *reinterpret_cast<float4*>(dst + 2 * chunk + so) = l;
       }
     };
+    auto publish_m = [&](int count) {
+      fence_proxy_async_global();  // workers read M_kk^T by TMA
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicExch((int*)&p.sync[3], count);
+      }
+    };
     auto mma_wait = [&]() {
       if (!mbar_wait(&cbar, cphase)) give_up(p);
       cphase ^= 1;
@@ -679,14 +694,6 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       nt.tdone_target = 0;
       if (k >= 1) nt.tdone_target = step_tasks(np, k - 1).ntrail;
       return nt;
-    };
-    auto publish_m = [&](int count) {
-      fence_proxy_async_global();  // workers read M_kk^T by TMA
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        __threadfence();
-        atomicExch((int*)&p.sync[3], count);
-      }
     };
     // the first diagonal block
     for (int e = threadIdx.x; e < FB * FB; e += FNT) {
@@ -715,31 +722,31 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
         umma_commit(&cbar);
       }
       mma_wait();
-      if (warp < 2) {
-        // lane r: row r of L, published split for the workers and staged as
-        // the operand of L L^T
-        const int r = threadIdx.x;
-        const uint32_t ta = ctb + ((uint32_t)(32 * warp) << 16);
-        float* gh = p.Lh + (int64_t)((k + 1) * FB + r) * np + (int64_t)k * FB;
-        float* gl = p.Ll + (int64_t)((k + 1) * FB + r) * np + (int64_t)k * FB;
+      // warps 0, 1, 4 and 5 read the accumulator: rows 32 (w % 4) .. + 31,
+      // columns 32 (w / 4) .. + 31 (a warp reaches the lanes of its quarter)
+      const bool reader = (warp & 3) < 2;
+      const int rr = 32 * (warp & 3) + (threadIdx.x & 31);
+      const int c0 = 32 * (warp >> 2);
+      if (reader) {
+        // row rr of L (columns c0 .. c0 + 31), published split for the
+        // workers and staged as the operand of L L^T
+        float v[32];
+        tmem_ld32(ctb + (uint32_t)c0 + ((uint32_t)(32 * (warp & 3)) << 16), v);
+        float* gh = p.Lh + (int64_t)((k + 1) * FB + rr) * np + (int64_t)k * FB + c0;
+        float* gl = p.Ll + (int64_t)((k + 1) * FB + rr) * np + (int64_t)k * FB + c0;
 #pragma unroll
-        for (int n0 = 0; n0 < FB; n0 += 32) {
-          float v[32];
-          tmem_ld32(ta + (uint32_t)n0, v);
-#pragma unroll
-          for (int j = 0; j < 32; j += 4) {
-            float4 h, l;
-            split_tf32(v[j + 0], h.x, l.x);
-            split_tf32(v[j + 1], h.y, l.y);
-            split_tf32(v[j + 2], h.z, l.z);
-            split_tf32(v[j + 3], h.w, l.w);
-            *reinterpret_cast<float4*>(gh + n0 + j) = h;
-            *reinterpret_cast<float4*>(gl + n0 + j) = l;
-            const int g = (n0 + j) >> 2;
-            const uint32_t so = (g >> 3) * kAChunk + sw128(r, g & 7);
-            *reinterpret_cast<float4*>(OPA + so) = h;
-            *reinterpret_cast<float4*>(OPA + 2 * kAChunk + so) = l;
-          }
+        for (int j = 0; j < 32; j += 4) {
+          float4 h, l;
+          split_tf32(v[j + 0], h.x, l.x);
+          split_tf32(v[j + 1], h.y, l.y);
+          split_tf32(v[j + 2], h.z, l.z);
+          split_tf32(v[j + 3], h.w, l.w);
+          *reinterpret_cast<float4*>(gh + j) = h;
+          *reinterpret_cast<float4*>(gl + j) = l;
+          const int g = (c0 + j) >> 2;
+          const uint32_t so = (g >> 3) * kAChunk + sw128(rr, g & 7);
+          *reinterpret_cast<float4*>(OPA + so) = h;
+          *reinterpret_cast<float4*>(OPA + 2 * kAChunk + so) = l;
         }
         fence_proxy_async_smem();
         fence_proxy_async_global();  // workers read L_{k+1,k} by TMA
@@ -756,16 +763,11 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
         atomicAdd(&p.pdone[k], 1);
       }
       mma_wait();
-      if (warp < 2) {
-        const int r = threadIdx.x;
-        const uint32_t ta = ctb + 64 + ((uint32_t)(32 * warp) << 16);
+      if (reader) {
+        float v[32];
+        tmem_ld32(ctb + 64 + (uint32_t)c0 + ((uint32_t)(32 * (warp & 3)) << 16), v);
 #pragma unroll
-        for (int n0 = 0; n0 < FB; n0 += 32) {
-          float v[32];
-          tmem_ld32(ta + (uint32_t)n0, v);
-#pragma unroll
-          for (int j = 0; j < 32; ++j) A[r * FP + n0 + j] = Cb[r * TP + n0 + j] - v[j];
-        }
+        for (int j = 0; j < 32; ++j) A[rr * FP + c0 + j] = Cb[rr * TP + c0 + j] - v[j];
       }
       tc_fence_before();
       __syncthreads();
@@ -787,18 +789,18 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   uint8_t* SBh = SAl + kRegionBytes;
   uint8_t* SBl = SBh + kRegionBytes;
   float* stg = reinterpret_cast<float*>(SBl + kRegionBytes);  // [kStages][32][128] epilogue staging
-  __shared__ uint64_t smem_free, acc_full[2], acc_empty[2], drain, op_full;
+  __shared__ uint64_t st_full[2], st_empty[2], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tmem_slot;
   __shared__ int local_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(&smem_free, 1);
     for (int b = 0; b < 2; ++b) {
+      mbar_init(&st_full[b], 1);
+      mbar_init(&st_empty[b], 1);
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
     mbar_init(&drain, 1);
-    mbar_init(&op_full, 1);
     local_abort = 0;
     fence_mbar_init();
   }
@@ -822,7 +824,6 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   const uint32_t aH = smem_u32(SAh), aL = smem_u32(SAl), bH = smem_u32(SBh), bL = smem_u32(SBl);
   int tcount = 0;    // tasks of this CTA so far (all steps): drives the barrier phases
   int epi_pass = 0;  // epilogue staging passes (selects the staging buffer)
-  uint32_t op_phase = 0;  // phase of op_full (thread 0: operands loaded by TMA)
   bool ok = true;
   for (int k = 0; ok && k < T; ++k) {
     const StepTasks st = step_tasks(np, k);
@@ -869,15 +870,21 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           mrows_seen = true;
           if (local_abort) break;
         }
-        // the previous task's MMAs have read the staged operands
-        if (tl > 0 && !mbar_wait(&smem_free, (tl - 1) & 1)) {
-          give_up(p);
-          local_abort = 1;
-          break;
-        }
+        // The operands go through a ring of two stages, one K chunk (32 of
+        // the 64) each: the MMAs of a chunk start once it has landed, and a
+        // stage is refilled (for the next task) once its MMAs are done.
         const int64_t kc = (int64_t)FB * k;  // k range of every product: block column k
         const bool by_tma = x.kind == 1 || x.kind == 3;
         if (!by_tma) {
+          // kinds 0 and 2 split an fp32 operand while staging it: all four
+          // warps write both stages, then thread 0 marks them full
+          bool w = true;
+          if (tl > 0) w = mbar_wait(&st_empty[0], (tl - 1) & 1) && mbar_wait(&st_empty[1], (tl - 1) & 1);
+          if (!w) {
+            give_up(p);
+            local_abort = 1;
+            break;
+          }
           if (x.kind == 0) {  // L_ik = R_ik M_kk^T
             stage_fp32(SAh, SAl, p.R, np, x.r0, kc, np);
           } else {  // (M_kk G_kj)[r][c] as D[c][r] = sum_t Gt[c][t] M_kk[r][t]
@@ -887,6 +894,11 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           cp_async_commit();
           cp_async_wait<0>();
           fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (threadIdx.x == 0) {
+            mbar_arrive(&st_full[0]);
+            mbar_arrive(&st_full[1]);
+          }
         } else if (threadIdx.x == 0) {
           // kind 1: (L L^T)[c][r], A = L rows c, B = L rows r;
           // kind 3: (L_ik M_kj)[i][c] = sum_t L[i][t] Mt[c][t], A = L rows i,
@@ -896,41 +908,50 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           const int32_t yb = (int32_t)(x.kind == 1 ? x.r0 : x.c0);
           const CUtensorMap* bhm = x.kind == 1 ? &om.lh : &om.mth;
           const CUtensorMap* blm = x.kind == 1 ? &om.ll : &om.mtl;
-          mbar_arrive_expect_tx(&op_full, (two ? 2u : 1u) * kRegionBytes * 2u);
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
+            if (tl > 0 && !mbar_wait(&st_empty[ch], (tl - 1) & 1)) {
+              give_up(p);
+              local_abort = 1;
+              break;
+            }
             const int32_t xk = (int32_t)(kc + 32 * ch);
-            tma_load_2d(SAh + ch * kChunkBytes, &om.lh, &op_full, xk, ya);
-            tma_load_2d(SAl + ch * kChunkBytes, &om.ll, &op_full, xk, ya);
+            mbar_arrive_expect_tx(&st_full[ch], (two ? 4u : 2u) * kChunkBytes);
+            tma_load_2d(SAh + ch * kChunkBytes, &om.lh, &st_full[ch], xk, ya);
+            tma_load_2d(SAl + ch * kChunkBytes, &om.ll, &st_full[ch], xk, ya);
             if (two) {
-              tma_load_2d(SBh + ch * kChunkBytes, bhm, &op_full, xk, yb);
-              tma_load_2d(SBl + ch * kChunkBytes, blm, &op_full, xk, yb);
+              tma_load_2d(SBh + ch * kChunkBytes, bhm, &st_full[ch], xk, yb);
+              tma_load_2d(SBl + ch * kChunkBytes, blm, &st_full[ch], xk, yb);
             }
           }
-          if (!mbar_wait(&op_full, op_phase)) {
-            give_up(p);
-            local_abort = 1;
-          }
-          op_phase ^= 1;
         }
-        named_bar_sync(1, 128);
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 96) {
+          // the MMA issuer: chunk by chunk, as the stages land
           const int buf = tl & 1;
           const int use = tl >> 1;
-          if (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1)) {
+          bool w = !(use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1));
+          const bool same = x.kind == 1 && x.diag;
+          const uint32_t idesc = make_idesc(2, 128, (x.kind == 0 || x.kind == 2) ? 64u : 128u);
+          const uint32_t d = tbase + (uint32_t)buf * 128;
+#pragma unroll
+          for (int ch = 0; ch < 2 && w; ++ch) {
+            if (!mbar_wait(&st_full[ch], tl & 1)) {
+              w = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t off = ch * kChunkBytes;
+            issue_mma_chunk(d, aH + off, aL + off, same ? aH + off : bH + off, same ? aL + off : bL + off, idesc,
+                            ch > 0);
+            umma_commit(&st_empty[ch]);
+          }
+          if (w) {
+            umma_commit(&acc_full[buf]);
+          } else {
             give_up(p);
             local_abort = 1;
-          } else {
-            tc_fence_after();
-            const uint32_t d = tbase + (uint32_t)buf * 128;
-            const bool same = x.kind == 1 && x.diag;
-            const uint32_t n = (x.kind == 0 || x.kind == 2) ? 64u : 128u;
-            issue_mma(d, aH, aL, same ? aH : bH, same ? aL : bL, make_idesc(2, 128, n));
-            umma_commit(&smem_free);
-            umma_commit(&acc_full[buf]);
           }
         }
-        named_bar_sync(1, 128);
       }
     } else {
       // ------------------------------------------------ epilogue (warps 4-7)
@@ -948,39 +969,53 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
         tc_fence_after();
         const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
         if (x.kind == 0 || x.kind == 2) {
-          // 64 accumulator columns per lane, stored split with vector stores:
-          //   kind 0  lane = row r of L, Lh/Ll[r][64k + n]
-          //   kind 2  lane = column c of M, Mth/Mtl[c][64k + n] = -D
-          //           (columns of block k and past it are not this task's)
-          const int64_t row = (x.kind == 0 ? x.r0 : x.c0) + cl;
-          const bool live = row < np && (x.kind == 0 || row < (int64_t)FB * k);
-          float* const bh = x.kind == 0 ? p.Lh : p.Mth;
-          float* const bl = x.kind == 0 ? p.Ll : p.Mtl;
+          // 64 accumulator columns per lane, split and staged in the 128-byte
+          // swizzled layout (lane = row of the stored tile), then written by
+          // TMA tensor stores:
+          //   kind 0  rows of L: Lh/Ll[r][64k .. 64k + 63];
+          //   kind 2  rows of M^T: Mth/Mtl[c][64k ..] = -D.  With k odd the
+          //           tile's last 64 rows are block k, whose M_kk^T is
+          //           already in place: only the first 64 rows are stored.
           const float sg = x.kind == 0 ? 1.f : -1.f;
+          uint8_t* sbase = reinterpret_cast<uint8_t*>(stg);  // hi: 2 chunks, then lo: 2 chunks
+          if (threadIdx.x == 128) bulk_wait_read<0>();  // earlier bulk copies are done reading stg
+          named_bar_sync(2, 128);
 #pragma unroll
           for (int n0 = 0; n0 < FB; n0 += 32) {
             float v[32];
             tmem_ld32(taddr + (uint32_t)n0, v);
-            if (live) {
-              float* dh = bh + row * np + (int64_t)FB * k + n0;
-              float* dl = bl + row * np + (int64_t)FB * k + n0;
 #pragma unroll
-              for (int j = 0; j < 32; j += 4) {
-                float4 h, l;
-                split_tf32(sg * v[j + 0], h.x, l.x);
-                split_tf32(sg * v[j + 1], h.y, l.y);
-                split_tf32(sg * v[j + 2], h.z, l.z);
-                split_tf32(sg * v[j + 3], h.w, l.w);
-                *reinterpret_cast<float4*>(dh + j) = h;
-                *reinterpret_cast<float4*>(dl + j) = l;
-              }
+            for (int j = 0; j < 32; j += 4) {
+              float4 h, l;
+              split_tf32(sg * v[j + 0], h.x, l.x);
+              split_tf32(sg * v[j + 1], h.y, l.y);
+              split_tf32(sg * v[j + 2], h.z, l.z);
+              split_tf32(sg * v[j + 3], h.w, l.w);
+              const int g = (n0 + j) >> 2;
+              const uint32_t so = (g >> 3) * kChunkBytes + sw128(cl, g & 7);
+              *reinterpret_cast<float4*>(sbase + so) = h;
+              *reinterpret_cast<float4*>(sbase + 2 * kChunkBytes + so) = l;
             }
           }
-          fence_proxy_async_global();  // other CTAs read these stores by TMA
+          fence_proxy_async_smem();
           tc_fence_before();
           mbar_arrive(&acc_empty[buf]);
           named_bar_sync(2, 128);
           if (threadIdx.x == 128) {
+            const int64_t row0 = x.kind == 0 ? x.r0 : x.c0;
+            const bool half = x.kind == 2 && row0 + 128 > (int64_t)FB * k;
+            const CUtensorMap* mh = x.kind == 0 ? &om.lh : (half ? &om.mth64 : &om.mth);
+            const CUtensorMap* ml = x.kind == 0 ? &om.ll : (half ? &om.mtl64 : &om.mtl);
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              const int32_t xc = (int32_t)((int64_t)FB * k + 32 * ch);
+              tma_store_2d(mh, sbase + ch * kChunkBytes, xc, (int32_t)row0);
+              tma_store_2d(ml, sbase + (2 + ch) * kChunkBytes, xc, (int32_t)row0);
+            }
+            bulk_commit();
+            // published once written: other CTAs read these tiles by TMA
+            bulk_wait_all();
+            fence_proxy_async_global();
             __threadfence();
             atomicAdd(x.kind == 0 ? &p.pdone[k] : &p.mrdone[k], 1);
           }
@@ -1066,8 +1101,9 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   if (threadIdx.x == 128) bulk_wait_all();
   __syncthreads();
   if (local_abort || aborted(p)) {
-    // let MMAs already issued finish before the tensor memory goes away
-    if (threadIdx.x == 0) {
+    // let MMAs already issued (by thread 96) finish before the tensor memory
+    // goes away; copies in flight land on barriers that are never reused
+    if (threadIdx.x == 96) {
       umma_commit(&drain);
       mbar_wait(&drain, 0);
     }
@@ -1156,7 +1192,8 @@ cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, 
   OpMaps om;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
   if (!make_r_map(&om.lh, Lh, np_, 32, 128, sw) || !make_r_map(&om.ll, Ll, np_, 32, 128, sw) ||
-      !make_r_map(&om.mth, Mth, np_, 32, 128, sw) || !make_r_map(&om.mtl, Mtl, np_, 32, 128, sw))
+      !make_r_map(&om.mth, Mth, np_, 32, 128, sw) || !make_r_map(&om.mtl, Mtl, np_, 32, 128, sw) ||
+      !make_r_map(&om.mth64, Mth, np_, 32, 64, sw) || !make_r_map(&om.mtl64, Mtl, np_, 32, 64, sw))
     return cudaErrorInvalidValue;
   void* args[] = {&rmap, &gmap, &om, &p};
   e = cudaLaunchCooperativeKernel((const void*)chol_kernel, dim3(grid), dim3(FNT), args, smem, st);
