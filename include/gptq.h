@@ -91,9 +91,9 @@ typedef enum gptq_dtype {
  *   block_size    > 0; with group_size != -1 it must divide group_size or be
  *                 a multiple of it.  It is the lazy-batch width: it changes
  *                 only the order of floating-point rounding, never the
- *                 result in exact arithmetic.  The kernels sweep 128 columns
- *                 at a time and apply the deferred update of later columns
- *                 every max(128, block_size rounded down to 128) columns.
+ *                 result in exact arithmetic.  This build validates it and
+ *                 always batches 128 columns (the width its kernels are
+ *                 built around).
  * maxq = 2^bits - 1.  code = clamp(rint(w / scale) + zero, 0, maxq), the
  * division and rint in IEEE float32 (round half to even).
  * Layer size limits of this build: 1 <= in <= 32768, 0 <= out <= 65535
@@ -315,8 +315,8 @@ gptq_status_t gptq_export_checkpoint(const uint32_t* qweight,
 gptq_status_t gptq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
 /* Size of the fixed device scratch used by gptq_quantize_layer_noalloc:
- * 16 MiB, enough for layers up to 1024 x 1024 at block_size 128. */
-#define GPTQ_STATIC_SCRATCH_BYTES ((size_t)16 << 20)
+ * 32 MiB, enough for layers up to 1024 x 1024. */
+#define GPTQ_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
 
 /*
  * gptq_quantize_layer without a caller workspace and without allocating.

@@ -92,7 +92,7 @@ lib.gptq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _p]
 lib.gptq_selftest_wait_timeout.restype = ctypes.c_int
 
 # bytes of the library's static scratch (GPTQ_STATIC_SCRATCH_BYTES in gptq.h)
-GPTQ_STATIC_SCRATCH_BYTES = 16 << 20
+GPTQ_STATIC_SCRATCH_BYTES = 32 << 20
 
 
 class GptqError(RuntimeError):

@@ -1,33 +1,40 @@
 // Blocked Cholesky factorisation R = L L^T ("Using AutoGPTQ in Practice":
-// the Hessian's Cholesky factorization), with the inverse of every 64 x 64
-// diagonal block, in one cooperative launch.  R is the reversed, damped
-// Hessian of gptq_prepare_hinv (lower triangle, np x np, np a multiple of
-// 128); the blocked inverse of L that turns the result into U is formed
-// afterwards by tensor-core merges in prepare.cu.
+// the Hessian's Cholesky factorization) and the inverse M = L^-1, in one
+// cooperative launch.  R is the reversed, damped Hessian of gptq_prepare_hinv
+// (lower triangle, np x np, np a multiple of 128); U = J M J is read from M^T
+// afterwards.
 //
-// Right-looking with 64-wide blocks and a look-ahead of one block.  Step k
-// (between two grid barriers):
-//   CTA 0 (the chain)   L_{k+1,k} = R_{k+1,k} M_kk^T; R_{k+1,k+1} -= L L^T;
-//                       then the leaf of block k+1: its Cholesky factor and
-//                       the factor's inverse M_{k+1,k+1}, both in registers
-//                       of two warps (the inverse warp trails the factor warp
-//                       by a pivot or more, fed through shared memory).
-//   CTAs 1.. (workers)  tensor-core tile tasks, 3xTF32 on tcgen05:
-//                       panel tiles L_ik = R_ik M_kk^T (i >= k+2, 128 rows x
-//                       64 columns), then, once every panel tile of the step
-//                       is written, the trailing update R_ij -= L_ik L_jk^T
-//                       of the lower triangle from block k+1 on, in 128 x 128
-//                       tiles (block (k+1, k+1) excluded: CTA 0 updates it).
-// The chain CTA's two 64 x 64 x 64 products run on the tensor cores too
-// (M = 128 with zero rows), the leaf on CUDA cores.
+// Right-looking with 64-wide blocks and a look-ahead of one block.  Step k:
+//   CTA 0 (the chain)   L_{k+1,k} = R_{k+1,k} M_kk^T and R_{k+1,k+1} - L L^T
+//                       as 3xTF32 tcgen05 MMAs (M = 128 with zero rows), then
+//                       the leaf of block k+1 on six warps: its Cholesky
+//                       factor in registers (one pivot chain per 32 rows) and
+//                       the factor's inverse M_{k+1,k+1}, pipelined through
+//                       shared memory.  A seventh warp meanwhile fetches the
+//                       next step's two tiles once the workers have updated
+//                       them.
+//   CTAs 1.. (workers)  3xTF32 tcgen05 tile tasks (128 x 128 or 128 x 64,
+//                       K = 64):
+//                         M row tiles   M_kj = -M_kk G_kj   (j < k)
+//                         panel tiles   L_ik = R_ik M_kk^T  (i >= k+2)
+//                         trailing      R_ij -= L_ik L_jk^T (lower, block k+1 on)
+//                         accumulation  G_ij += L_ik M_kj   (i > k, j <= k)
+//                       where G accumulates sum_t L_it M_tj, so block row k of
+//                       M is final once step k - 1's accumulation has landed.
+// The CTAs never meet at a grid barrier: counters in global memory publish
+// the diagonal blocks, panel tiles, M row tiles, and the trailing and
+// accumulation tiles that have landed, and each task waits for exactly the
+// counters its operands depend on (the reduce-adds of consecutive steps reach
+// each element in step order).
 //
-// Worker CTAs: warps 0-3 stage the operands of a task in shared memory in
-// the tensor core's 128-byte-swizzled K-major layout (split fp32: tf32 hi
-// plus the exact remainder; L's panel tiles are stored split, R's tiles are
-// split while they are staged) and one of their threads issues the MMAs;
-// warps 4-7 read the accumulator from tensor memory and write the result.
+// Worker CTAs: warps 0-3 stage a task's split operands (tf32 hi plus the exact
+// fp32 remainder) in a two-stage ring of 128-byte-swizzled K chunks, by TMA
+// tensor copies (L, M^T) or by splitting fp32 tiles on the way (R, G^T); one
+// thread issues the MMAs chunk by chunk; warps 4-7 read the tensor-memory
+// accumulator and write the result: trailing and accumulation tiles by TMA
+// reduce-add into R and G^T in L2, panel and M row tiles by TMA tensor stores.
 // Two tensor-memory accumulators let a task's epilogue overlap the next
-// task's staging and MMAs.
+// task's MMAs.
 //
 // Every wait is bounded by %globaltimer; a wait that gives up raises
 // ST_TIMEOUT, sets the launch-wide abort flag and unwinds.
@@ -120,27 +127,6 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// 2-D tiled bulk tensor reduce-add shared -> global (bulk-group completion),
-// clipped at the tensor map's bounds.
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* smem_src, int32_t x,
-                                                  int32_t y) {
-  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
-               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
-               : "memory");
-}
-// 2-D tiled bulk tensor store shared -> global (bulk-group completion), clipped
-// at the tensor map's bounds.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
-               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
-               : "memory");
-}
-
-// Order this thread's async-proxy global writes (bulk copies it waited for)
-// before its later generic-proxy operations.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 // Shared-memory flag between two warps of one CTA (release / acquire).
 __device__ __forceinline__ void st_release_cta(int* p, int v) {
@@ -432,10 +418,6 @@ __device__ void store_diag_m(const CholParams& p, const float* M, int b) {
 }
 
 // ------------------------------------------------------------------ workers
-// Byte offset of 16-byte unit u (0..7) of row r in a 128-byte-swizzled
-// K-major chunk (the layout TMA's 128-byte swizzle produces): the unit index
-// is XOR-ed with the row's position inside its 8-row, 1024-byte group.
-__device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
 // Stage rows [row0, row0 + nrows) x columns [col0, col0 + 64) of a split
 // matrix (hi, lo; row stride ld) into regions Shi, Slo: 128-byte swizzled,
@@ -504,19 +486,6 @@ __device__ __forceinline__ void issue_mma_strided(uint32_t d, uint32_t a_hi, uin
     }
 }
 
-// 12 MMAs: D (+)= A B^T over one K chunk of 32 with split operands (hi hi + hi
-// lo + lo hi); accumulate == false starts the accumulator.
-__device__ __forceinline__ void issue_mma_chunk(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
-                                                uint32_t b_lo, uint32_t idesc, bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const uint64_t ah = smem_desc_k_sw128(a_hi + kk * 32), al = smem_desc_k_sw128(a_lo + kk * 32);
-    const uint64_t bh = smem_desc_k_sw128(b_hi + kk * 32), bl = smem_desc_k_sw128(b_lo + kk * 32);
-    umma_tf32(d, ah, bh, idesc, (accumulate || kk) ? 1u : 0u);
-    umma_tf32(d, ah, bl, idesc, 1u);
-    umma_tf32(d, al, bh, idesc, 1u);
-  }
-}
 
 // The tile tasks of step k, in this order:
 //   kind 2  M row tiles: M_kj = -M_kk G_kj for the columns before block k
@@ -1127,13 +1096,10 @@ namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+}  // namespace
 
-// An np x np fp32 row-major matrix as a 2-D tensor: 128-column x 32-row boxes
-// without swizzle for the reduce-add epilogues (R, G^T), 32-column x 128-row
-// boxes with 128-byte swizzle for the operand loads (L, M^T; the tensor
-// core's K-major layout).
-bool make_r_map(CUtensorMap* m, float* R, int64_t np_, uint32_t box_x = 128, uint32_t box_y = 32,
-                CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
+bool encode_f32_2d(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld, uint32_t box_x,
+                   uint32_t box_y, bool swizzle128) {
   static EncodeTiledFn fn = [] {
     void* f = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -1143,12 +1109,23 @@ bool make_r_map(CUtensorMap* m, float* R, int64_t np_, uint32_t box_x = 128, uin
     return (EncodeTiledFn)f;
   }();
   if (!fn) return false;
-  cuuint64_t gdim[2] = {(cuuint64_t)np_, (cuuint64_t)np_};
-  cuuint64_t gstride[1] = {(cuuint64_t)(np_ * 4)};
+  cuuint64_t gdim[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t gstride[1] = {(cuuint64_t)(ld * 4)};
   cuuint32_t box[2] = {box_x, box_y};
   cuuint32_t estride[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, R, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+// An np x np fp32 row-major matrix as a 2-D tensor: 128-column x 32-row boxes
+// without swizzle for the reduce-add epilogues (R, G^T), 32-column x 128-row
+// boxes with 128-byte swizzle for the operand loads (L, M^T; the tensor
+// core's K-major layout).
+bool make_r_map(CUtensorMap* m, float* R, int64_t np_, uint32_t box_x = 128, uint32_t box_y = 32,
+                bool swz = false) {
+  return encode_f32_2d(m, R, np_, np_, np_, box_x, box_y, swz);
 }
 }  // namespace
 
@@ -1190,7 +1167,7 @@ cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, 
   CUtensorMap rmap, gmap;
   if (!make_r_map(&rmap, R, np_) || !make_r_map(&gmap, Gt, np_)) return cudaErrorInvalidValue;
   OpMaps om;
-  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  const bool sw = true;
   if (!make_r_map(&om.lh, Lh, np_, 32, 128, sw) || !make_r_map(&om.ll, Ll, np_, 32, 128, sw) ||
       !make_r_map(&om.mth, Mth, np_, 32, 128, sw) || !make_r_map(&om.mtl, Mtl, np_, 32, 128, sw) ||
       !make_r_map(&om.mth64, Mth, np_, 32, 64, sw) || !make_r_map(&om.mtl64, Mtl, np_, 32, 64, sw))

@@ -162,6 +162,28 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// 2-D tiled bulk tensor reduce-add shared -> global (bulk-group completion),
+// clipped at the tensor map's bounds.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* smem_src, int32_t x,
+                                                  int32_t y) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+// 2-D tiled bulk tensor store shared -> global (bulk-group completion), clipped
+// at the tensor map's bounds.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* smem_src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+               "r"(smem_u32(smem_src)), "r"(x), "r"(y)
+               : "memory");
+}
+
+// Order this thread's async-proxy global writes (bulk copies it waited for)
+// before its later generic-proxy operations.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* smem_result, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -287,6 +309,11 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, uint32_t M
   return (1u << 4) | (ab_format << 7) | (ab_format << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
+// Byte offset of 16-byte unit u (0..7) of row r in a 128-byte-swizzled
+// K-major chunk (the layout TMA's 128-byte swizzle produces): the unit index
+// is XOR-ed with the row's position inside its 8-row, 1024-byte group.
+__device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+
 // ----------------------------------------------------------------- misc math
 // Split an fp32 value into hi (rounded to tf32, low 13 mantissa bits zero)
 // and lo = v - hi (exact).  hi + lo == v, |lo| <= 2^-11 |v|.
@@ -295,6 +322,21 @@ __device__ __forceinline__ void split_tf32(float v, float& hi, float& lo) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(h) : "f"(v));
   hi = __uint_as_float(h);
   lo = v - hi;
+}
+
+
+// 12 MMAs: D (+)= A B^T over one K chunk of 32 with split operands (hi hi + hi
+// lo + lo hi); accumulate == false starts the accumulator.
+__device__ __forceinline__ void issue_mma_chunk(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
+                                                uint32_t b_lo, uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint64_t ah = smem_desc_k_sw128(a_hi + kk * 32), al = smem_desc_k_sw128(a_lo + kk * 32);
+    const uint64_t bh = smem_desc_k_sw128(b_hi + kk * 32), bl = smem_desc_k_sw128(b_lo + kk * 32);
+    umma_tf32(d, ah, bh, idesc, (accumulate || kk) ? 1u : 0u);
+    umma_tf32(d, ah, bl, idesc, 1u);
+    umma_tf32(d, al, bh, idesc, 1u);
+  }
 }
 
 }  // namespace gptq

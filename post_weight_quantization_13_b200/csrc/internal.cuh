@@ -82,12 +82,28 @@ size_t chol_sync_bytes(int64_t np_);
 cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, float* Ml, float* Mth, float* Mtl,
                         float* Gt, unsigned* sync, uint32_t* status, int sms, cudaStream_t st);
 
+// A 2-D tensor map over a row-major fp32 matrix (cols x rows, row stride ld
+// elements) with boxes of box_x columns by box_y rows; swizzle128 selects the
+// 128-byte swizzle (the tensor core's K-major operand layout).
+bool encode_f32_2d(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld, uint32_t box_x,
+                   uint32_t box_y, bool swizzle128);
+
 // Make the driver load every kernel gptq_quantize_layer can launch on the
 // current device now, instead of at their first launch.
 cudaError_t preload_quantize_kernels();
 
-// Lazy-batch width actually used for a configuration (multiple of 128,
-// compatible with group_size, at most 1024).
-int64_t outer_block(const gptq_config_t* cfg);
+// The sweep and its updates (solve.cu).  Wp (out x np, processing order) is
+// updated in place; Uh/Ul = split U^T (np x np); Ud = solve_pack_ud's
+// diagonal blocks; Eh/El (out x np) receive the split -E; sync:
+// solve_sync_bytes scratch.  Writes codes_p (out x np, processing order),
+// scales, zeros and loss (zeroed by the caller).
+size_t solve_ud_bytes(int64_t np_);
+size_t solve_sync_bytes(int64_t out, int64_t np_);
+cudaError_t solve_pack_ud(const float* U, int64_t in, int64_t np_, float* Ud, cudaStream_t st);
+cudaError_t solve_quantize(float* Wp, int64_t out, int64_t in, int64_t np_, const float* Uh, const float* Ul,
+                           const float* Ud, float* Eh, float* El, const gptq_config_t* cfg, float* scales,
+                           int32_t* zeros, uint8_t* codes_p, float* loss, void* sync, uint32_t* status, int sms,
+                           cudaStream_t st);
+cudaError_t preload_solve_kernels();
 
 }  // namespace gptq

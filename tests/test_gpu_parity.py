@@ -261,37 +261,39 @@ import numpy as np
 import torch
 sys.path.insert(0, sys.argv[1])
 import post_weight_quantization_13_b200 as g
-S32 = np.load(sys.argv[2])
-n, in_ = int(sys.argv[3]), S32.shape[0]
-cfg = g.GptqConfig(bits=4, group_size=128, desc_act=True)
-ws = torch.empty(g.gptq_workspace_bytes(0, in_, cfg), dtype=torch.uint8, device="cuda")
-U = torch.empty((in_, in_), dtype=torch.float32, device="cuda")
-perm = torch.empty(in_, dtype=torch.int32, device="cuda")
-dead = torch.empty(in_, dtype=torch.uint8, device="cuda")
-g.gptq_prepare_hinv(torch.from_numpy(S32).cuda(), n, cfg, U, perm, dead, ws)
-np.save(sys.argv[4], U.cpu().numpy().T)
-np.save(sys.argv[5], perm.cpu().numpy())
+X = torch.from_numpy(np.load(sys.argv[2])).cuda()
+S = torch.zeros((X.shape[0], X.shape[0]), dtype=torch.float32, device="cuda")
+g.gptq_hessian_accumulate(S, X)
+np.save(sys.argv[3], S.cpu().numpy())
 """
 
 
 def test_tensor_core_and_cuda_core_paths_agree(lib, tmp_path):
-    """The prepare's GEMMs on the tensor cores against the same GEMMs on the
+    """The Hessian's SYRK on the tensor cores against the same product on the
     CUDA cores.  The library reads GPTQ_FORCE_SIMT once per process, so the
-    CUDA-core run happens in a child process started with it set."""
+    CUDA-core run happens in a child process started with it set.  Both
+    accumulate exact products in fp32 from the same fp16 X: they differ by
+    rounding order only, and each stays within the header's 5e-5 bound of
+    the exact S."""
     import subprocess
     import sys
-    S32, n = _prep_inputs(93, 640, 2000, "correlated")
-    cfg = _cfg(lib, bits=4, group_size=128, desc_act=True)
-    U1, p1, _ = _run_prepare(lib, S32, n, cfg)
-    np.save(tmp_path / "S.npy", S32)
+
+    import torch
+    rng = np.random.default_rng(93)
+    X = (rng.standard_normal((640, 3000)) * 0.5).astype(np.float16)
+    S1 = torch.zeros((640, 640), dtype=torch.float32, device="cuda")
+    lib.gptq_hessian_accumulate(S1, torch.from_numpy(X).cuda())
+    np.save(tmp_path / "X.npy", X)
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     env = dict(os.environ, GPTQ_FORCE_SIMT="1")
-    subprocess.run([sys.executable, "-c", _SIMT_CHILD, root, str(tmp_path / "S.npy"), str(n),
-                    str(tmp_path / "U.npy"), str(tmp_path / "p.npy")], env=env, check=True, timeout=300)
-    U2 = np.load(tmp_path / "U.npy")
-    p2 = np.load(tmp_path / "p.npy")
-    assert np.array_equal(p1, p2)
-    assert rel_fro(U1, U2) < 1e-5
+    subprocess.run([sys.executable, "-c", _SIMT_CHILD, root, str(tmp_path / "X.npy"),
+                    str(tmp_path / "S.npy")], env=env, check=True, timeout=300)
+    S2 = np.load(tmp_path / "S.npy")
+    S1 = S1.cpu().numpy()
+    assert rel_fro(S1, S2) < 5e-5
+    Xd = X.astype(np.float64)
+    assert rel_fro(np.triu(S1), np.triu(Xd @ Xd.T)) < 5e-5
+    assert rel_fro(np.triu(S2), np.triu(Xd @ Xd.T)) < 5e-5
 
 
 def test_act_order_exact_on_near_tie_diagonals(lib):
