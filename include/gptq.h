@@ -314,6 +314,20 @@ gptq_status_t gptq_export_checkpoint(const uint32_t* qweight,
  */
 gptq_status_t gptq_selftest_wait_timeout(uint64_t limit_ns, void* stream);
 
+/*
+ * Diagnostic with no counterpart in the method: the sweep decides each code
+ * from x / scale rounded to nearest, computed without a divide (a
+ * reciprocal and two fma corrections, Markstein's method).  This call checks
+ * that quotient against the IEEE division on n pseudo-random pairs drawn from
+ * seed (a quarter with random magnitudes, the rest within 8 units in the last
+ * place of a half-integer multiple of the scale).  *checked receives the
+ * pairs inside the method's range (the sweep takes an exact fallback
+ * outside it), *mismatches those whose quotient differed in any bit.
+ * Synchronises the stream.
+ */
+gptq_status_t gptq_selftest_quotient(uint64_t n, uint64_t seed, uint64_t* checked, uint64_t* mismatches,
+                                     void* stream);
+
 /* Size of the fixed device scratch used by gptq_quantize_layer_noalloc:
  * 32 MiB, enough for layers up to 1024 x 1024. */
 #define GPTQ_STATIC_SCRATCH_BYTES ((size_t)32 << 20)

@@ -26,6 +26,7 @@ __all__ = [
     "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "GPTQ_STATIC_SCRATCH_BYTES",
     "gptq_workspace_status", "gptq_quantize_layer_noalloc_status",
     "gptq_dequantize_layer", "gptq_export_checkpoint", "gptq_selftest_wait_timeout",
+    "gptq_selftest_quotient",
     "solve_layer", "solve_block", "export_checkpoint", "STATUS_NAMES",
 ]
 
@@ -90,6 +91,9 @@ lib.gptq_export_checkpoint.restype = ctypes.c_int
 
 lib.gptq_selftest_wait_timeout.argtypes = [ctypes.c_uint64, _p]
 lib.gptq_selftest_wait_timeout.restype = ctypes.c_int
+lib.gptq_selftest_quotient.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64),
+                                       ctypes.POINTER(ctypes.c_uint64), _p]
+lib.gptq_selftest_quotient.restype = ctypes.c_int
 
 # bytes of the library's static scratch (GPTQ_STATIC_SCRATCH_BYTES in gptq.h)
 GPTQ_STATIC_SCRATCH_BYTES = 32 << 20
@@ -247,6 +251,14 @@ def gptq_export_checkpoint(qweight, scales, zeros, out: int, in_: int, bits: int
     _check(lib.gptq_export_checkpoint(_ptr(qweight), _ptr(scales), _ptr(zeros), int(out), int(in_),
                                       int(bits), int(ngroups), int(zero_offset), _ptr(qweight_t),
                                       _ptr(qzeros), _ptr(scales_h), _stream(stream)))
+
+
+def gptq_selftest_quotient(n: int, seed: int = 1, stream=None) -> tuple[int, int]:
+    """Check the sweep's divide-free quotient against IEEE division on n
+    pseudo-random pairs; returns (pairs checked, mismatches)."""
+    c, m = ctypes.c_uint64(0), ctypes.c_uint64(0)
+    _check(lib.gptq_selftest_quotient(int(n), int(seed), ctypes.byref(c), ctypes.byref(m), _stream(stream)))
+    return c.value, m.value
 
 
 def gptq_selftest_wait_timeout(limit_ns: int, stream=None) -> int:

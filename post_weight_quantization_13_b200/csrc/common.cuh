@@ -315,6 +315,24 @@ __host__ __device__ constexpr uint32_t make_idesc(uint32_t ab_format, uint32_t M
 __device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
 // ----------------------------------------------------------------- misc math
+// x / s rounded to nearest (IEEE binary32) without a divide, from
+// Markstein's correction step (P. W. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Develop.
+// 34(1), 1990): when y = RN(1/s) and q is within one unit in the last place
+// of x/s, RN(q + (x - s q) y) = RN(x/s), the residual x - s q being exact in
+// one fma.  q0 = RN(x y) can be 1.5 units off; a first correction brings it
+// within one, the second rounds correctly.  Valid while no step overflows or
+// leaves the normal range, which quot_in_range guarantees.
+__device__ __forceinline__ float quot_rn(float x, float s, float inv_s) {
+  const float q0 = x * inv_s;
+  const float q1 = fmaf(fmaf(-q0, s, x), inv_s, q0);
+  return fmaf(fmaf(-q1, s, x), inv_s, q1);
+}
+__device__ __forceinline__ bool quot_in_range(float x, float s) {
+  const float ax = fabsf(x);
+  return (ax == 0.f || (ax >= 0x1p-60f && ax <= 0x1p60f)) && s >= 0x1p-60f && s <= 0x1p60f;
+}
+
 // Split an fp32 value into hi (rounded to tf32, low 13 mantissa bits zero)
 // and lo = v - hi (exact).  hi + lo == v, |lo| <= 2^-11 |v|.
 __device__ __forceinline__ void split_tf32(float v, float& hi, float& lo) {

@@ -52,13 +52,16 @@ constexpr uint32_t kUdBytes = kUdFloats * 4;
 // chain CTA shared memory (offsets from a 1024-byte aligned base)
 constexpr uint32_t kCWb = 0;                   // 4 chunks: W of the slab's block
 constexpr uint32_t kCUb = kCWb + 4 * kQChunk;  // 2 slots x (hi, lo): U rows of the block, one K chunk
-constexpr uint32_t kCA = kCUb + 4 * kQChunk;   // (hi, lo): -E of the sub-block
-constexpr uint32_t kCUd = kCA + 2 * kQChunk;   // 2 slots of kUdBytes
+constexpr uint32_t kCUn = kCUb + 4 * kQChunk;  // (hi, lo): U rows of the next block, the same K chunk
+constexpr uint32_t kCA = kCUn + 2 * kQChunk;   // (hi, lo): -E of the sub-block
+constexpr uint32_t kCX = kCA + 2 * kQChunk;    // each row's values at the sub-block's start
+constexpr uint32_t kCUd = kCX + kQChunk;       // 2 slots of kUdBytes
 constexpr uint32_t kChainSmem = kCUd + 2 * kUdBytes;
 // worker CTA
-constexpr uint32_t kWRing = 0;                 // 2 slots x (U hi, U lo, E hi, E lo) chunks
-constexpr int kWStages = 4;                    // epilogue staging tiles, 32 rows x 128 columns fp32
-constexpr uint32_t kWStg = kWRing + 8 * kQChunk;
+constexpr uint32_t kWE = 0;                    // -E of a slab's block: 4 K chunks, hi and lo
+constexpr uint32_t kWRing = kWE + 8 * kQChunk; // 2 slots x (U hi, U lo) chunks
+constexpr int kWStages = 2;                    // epilogue staging tiles, 32 rows x 128 columns fp32
+constexpr uint32_t kWStg = kWRing + 4 * kQChunk;
 constexpr uint32_t kWorkerSmem = kWStg + kWStages * 32 * 128 * 4;
 constexpr uint32_t kSolveSmem = 1024 + (kChainSmem > kWorkerSmem ? kChainSmem : kWorkerSmem);
 static_assert(kSolveSmem <= 232448, "shared memory per CTA");
@@ -70,6 +73,7 @@ struct SolveParams {
   int T;            // column blocks (np / 128)
   int nslab;        // row slabs (ceil(out / 128))
   int nchain;       // chain CTAs (CTAs 0 .. nchain - 1); slab i belongs to chain i % nchain
+  int chain_next;   // the chains apply each block's errors to the slab's next block themselves
   int maxq, sym, gs, ngroups;
   float* scales;
   int32_t* zeros;
@@ -183,6 +187,12 @@ __device__ __forceinline__ void load_row(const uint8_t* chunk, int r, float (&v)
   }
 }
 
+__device__ __forceinline__ void store_row(uint8_t* chunk, int r, const float (&v)[32]) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    *reinterpret_cast<float4*>(chunk + sw128(r, u)) = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+}
+
 __device__ __forceinline__ void add_tmem(uint32_t taddr, float (&v)[32]) {
   float d[32];
   tmem_ld32(taddr, d);
@@ -190,20 +200,174 @@ __device__ __forceinline__ void add_tmem(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] += d[i];
 }
 
+// A 16-byte shared-memory load the compiler keeps where it is written (it
+// would otherwise hoist the U rows of many columns at once and run out of
+// registers).
+__device__ __forceinline__ float4 lds128(const float* p) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ float lds32(const float* p) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_u32(p)));
+  return v;
+}
+__device__ __forceinline__ float elem(const float4& v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+// Zero, in a way the compiler cannot see through: an address plus
+// after(v) is only formed once v is, which keeps a load behind v.
+__device__ __forceinline__ uint32_t after(float v) {
+  uint32_t z;
+  asm volatile("and.b32 %0, %1, 0;" : "=r"(z) : "r"(__float_as_uint(v)));
+  return z;
+}
+
+// One row's 32 columns of a sub-block (x: their current values; ud: the
+// sub-block's U and 1 / U_jj).  For each column: the group's scale and zero
+// at a group start inside the sub-block, the code clamp(rint(x / s) + z, 0,
+// maxq), the error e = (x - s (code - z)) / U_jj (zero past the layer's
+// columns), and x[j'] -= e U[j][j'] for the sub-block's later columns.  On
+// return x holds -e, cw the codes (one byte each).
+//
+// kFast: x / s from the divide-free quotient, with no branch in the column
+// loop; false if any quotient was outside its range (the results are then to
+// be discarded).  U's row j + 1 is read while column j is quantized, so the
+// loads never wait in front of the column's updates.  Otherwise x / s from
+// round_div.
+template <int GSB, bool kFast>
+__device__ __forceinline__ bool sweep32(float (&x)[32], const float* ud, int64_t c0, const SolveParams& p,
+                                        int64_t row, bool live, float fmaxq, float& s_, float& z_, float& inv_s,
+                                        float& lsum, uint32_t (&cw)[8]) {
+  bool in_range = true;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) cw[i] = 0u;
+  float4 ucur[8], unext[8];
+  float rcur = 0.f, rnext = 0.f;
+  if (kFast) {
+#pragma unroll
+    for (int a = 0; a < 8; ++a) ucur[a] = lds128(ud + 4 * a);
+    rcur = lds32(ud + SB * SB);
+  }
+#pragma unroll
+  for (int j = 0; j < SB; ++j) {
+    if (kFast && j + 1 < SB) {
+      // U's row j + 1, once column j is final (not earlier: registers)
+      const float* un = ud + after(x[j]);
+#pragma unroll
+      for (int a = (j + 2) >> 2; a < 8; ++a) unext[a] = lds128(un + (j + 1) * SB + 4 * a);
+      rnext = lds32(un + SB * SB + j + 1);
+    }
+    if (GSB <= SB && j % GSB == 0 && c0 + j < p.in) {
+      float lo = INFINITY, hi = -INFINITY, am = 0.f;
+#pragma unroll
+      for (int i = j; i < j + (GSB <= SB ? GSB : 1); ++i) minmax(x[i], lo, hi, am);
+      group_params(lo, hi, am, p.sym, fmaxq, s_, z_);
+      inv_s = __frcp_rn(s_);
+      if (live) {
+        p.scales[row * p.ngroups + (c0 + j) / GSB] = s_;
+        p.zeros[row * p.ngroups + (c0 + j) / GSB] = (int32_t)z_;
+      }
+    }
+    const float xv = x[j];
+    float qf;
+    if (kFast) {
+      qf = rintf(quot_rn(xv, s_, inv_s)) + z_;
+      in_range &= quot_in_range(xv, s_);
+    } else {
+      qf = round_div(xv, s_, inv_s) + z_;
+    }
+    qf = fminf(fmaxf(qf, 0.f), fmaxq);
+    const float deq = s_ * (qf - z_);
+    float e = (xv - deq) * (kFast ? rcur : ud[SB * SB + j]);
+    e = c0 + j < p.in ? e : 0.f;
+    lsum = fmaf(e, e, lsum);
+    cw[j >> 2] |= (uint32_t)qf << (8 * (j & 3));
+    x[j] = -e;
+    // the sub-block's later columns: x[j'] -= e U[j][j'], the next one first
+    if (kFast) {
+#pragma unroll
+      for (int jp = j + 1; jp < SB; ++jp) x[jp] = fmaf(-e, elem(ucur[jp >> 2], jp & 3), x[jp]);
+#pragma unroll
+      for (int a = 0; a < 8; ++a) ucur[a] = unext[a];
+      rcur = rnext;
+    } else {
+      const float* ur = ud + j * SB;
+#pragma unroll
+      for (int a = (j + 1) >> 2; a < 8; ++a) {
+        const float4 u = *reinterpret_cast<const float4*>(ur + 4 * a);
+        if (4 * a + 0 > j) x[4 * a + 0] = fmaf(-e, u.x, x[4 * a + 0]);
+        if (4 * a + 1 > j) x[4 * a + 1] = fmaf(-e, u.y, x[4 * a + 1]);
+        if (4 * a + 2 > j) x[4 * a + 2] = fmaf(-e, u.z, x[4 * a + 2]);
+        if (4 * a + 3 > j) x[4 * a + 3] = fmaf(-e, u.w, x[4 * a + 3]);
+      }
+    }
+  }
+  return in_range;
+}
+
+// A row's 32 codes of a sub-block (one byte each, 16-byte aligned).
+__device__ __forceinline__ void store_codes(const SolveParams& p, int64_t row, int64_t c0, bool live,
+                                            const uint32_t (&cw)[8]) {
+  if (!live) return;
+  uint4* dst = reinterpret_cast<uint4*>(p.codes_p + row * p.np_ + c0);
+  dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+  dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+}
+
+struct RowState {
+  float s, z, inv_s, lsum;
+};
+
+// The sub-block again with round_div, from the row's values at its start
+// (in Xs, where the results, -e, go back too).  Kept out of line: it runs
+// only for quotients outside quot_in_range, and inlined it would take
+// registers from the main loop.
+template <int GSB>
+__device__ __noinline__ RowState replay32(uint8_t* Xs, int rl, const float* ud, int64_t c0, const SolveParams& p,
+                                          int64_t row, bool live, float fmaxq, RowState st) {
+  float x[32];
+  uint32_t cw[8];
+  load_row(Xs, rl, x);
+  sweep32<GSB, false>(x, ud, c0, p, row, live, fmaxq, st.s, st.z, st.inv_s, st.lsum, cw);
+  store_row(Xs, rl, x);
+  store_codes(p, row, c0, live, cw);
+  return st;
+}
+
 // ------------------------------------------------------------------ chain CTA
 // Threads 0-127: one row each (warp w reads tensor-memory lanes 32w..32w+31,
 // its own quarter).  Thread 128: loads, MMAs, the -E stores and the
 // publication.  Threads 129-255 have nothing to do.
+//
+// With p.chain_next (at most two slabs per chain) the chain also applies a
+// block's errors to the slab's next block: each slab keeps two 128-column
+// accumulators, D_cur for the block being swept and D_next for the one after
+// it, and every sub-block's MMAs add to both.  Block k + 1 then starts from
+// W (with the workers' contributions of blocks up to k - 1) plus D_next, and
+// the workers take only the blocks two and more ahead.  Without it the
+// workers take every later block and the chain's one accumulator starts
+// afresh with each block.
 template <int GSB>
 __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams& p, uint8_t* sm) {
   uint8_t* Wb = sm + kCWb;
   uint8_t* Ub = sm + kCUb;
+  uint8_t* Un = sm + kCUn;
   uint8_t* Ab = sm + kCA;
+  uint8_t* Xs = sm + kCX;
   float* Udb = reinterpret_cast<float*>(sm + kCUd);
-  __shared__ uint64_t wb_full[4], wb_empty[4], ub_full[2], ud_full[2], ud_empty[2];
+  __shared__ uint64_t wb_full[4], wb_empty[4], ub_full[2], un_full, ud_full[2], ud_empty[2];
   __shared__ uint64_t a_full, a_empty, mma_next, mma_done, drain;
   __shared__ uint32_t tslot;
   const int warp = threadIdx.x >> 5;
+  const int64_t np = p.np_;
+  const int T = p.T;
+  const bool cn = p.chain_next != 0;
+  // items: (block k, slab) for k = 0 .. T - 1, this chain's slabs in turn
+  const int spc = (p.nslab - (int)blockIdx.x + p.nchain - 1) / p.nchain;
+  const int nitems = T * spc;
+  const uint32_t tcols = cn ? (spc > 1 ? 512u : 256u) : 128u;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 4; ++i) {
       mbar_init(&wb_full[i], 1);
@@ -214,6 +378,7 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
       mbar_init(&ud_full[i], 1);
       mbar_init(&ud_empty[i], 128);
     }
+    mbar_init(&un_full, 1);
     mbar_init(&a_full, 128);
     mbar_init(&a_empty, 1);
     mbar_init(&mma_next, 1);
@@ -222,20 +387,23 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&tslot, 128);
+    tmem_alloc(&tslot, tcols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tslot;
-  const int64_t np = p.np_;
-  const int T = p.T;
-  // items: (block k, slab) for k = 0 .. T - 1, this chain's slabs in turn
-  const int spc = (p.nslab - (int)blockIdx.x + p.nchain - 1) / p.nchain;
-  const int nitems = T * spc;
   auto item_k = [&](int it) { return it / spc; };
   auto item_slab = [&](int it) { return (int)blockIdx.x + (it % spc) * p.nchain; };
+  // accumulator of item it's block (cur = 0) or of the block after it (cur = 1)
+  auto acc = [&](int it, int nxt) -> uint32_t {
+    return cn ? tbase + 256u * (uint32_t)(it % spc) + 128u * (uint32_t)((item_k(it) + nxt) & 1) : tbase;
+  };
+  // contributions to a slab's block k the workers make (the rest come from D)
+  auto worker_count = [&](int k) { return cn ? (k > 0 ? k - 1 : 0) : k; };
+  // sub-block g of the launch's sequence has a next-block product
+  auto has_next = [&](int g) { return cn && g < 4 * nitems && item_k(g >> 2) + 1 < T; };
   bool ok = true;
 
   if (threadIdx.x == 128) {
@@ -245,8 +413,8 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
     tma_prefetch_desc(&mp.ul);
     tma_prefetch_desc(&mp.eh);
     tma_prefetch_desc(&mp.el);
-    // U rows of block k, K chunk s (use u = 3 it + s: the three sub-blocks
-    // with MMAs), into slot u & 1
+    // U rows of block k, K chunk s (use u = 3 it + s: the sub-blocks with
+    // products inside the block), into slot u & 1
     auto load_ub = [&](int u) {
       const int it = u / 3, s = u % 3;
       const int k = item_k(it);
@@ -255,6 +423,14 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
       tma_load_2d(dst, &mp.uh, &ub_full[u & 1], QB * k + SB * s, QB * k);
       tma_load_2d(dst + kQChunk, &mp.ul, &ub_full[u & 1], QB * k + SB * s, QB * k);
     };
+    // U rows of block k + 1, K chunk s of block k, for sub-block g
+    auto load_un = [&](int g) {
+      const int it = g >> 2, s = g & 3;
+      const int k = item_k(it);
+      mbar_arrive_expect_tx(&un_full, 2 * kQChunk);
+      tma_load_2d(Un, &mp.uh, &un_full, QB * k + SB * s, QB * (k + 1));
+      tma_load_2d(Un + kQChunk, &mp.ul, &un_full, QB * k + SB * s, QB * (k + 1));
+    };
     // U of sub-block g (4 per item) into slot g & 1
     auto load_ud = [&](int g) {
       const int it = g >> 2, s = g & 3;
@@ -262,26 +438,39 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
       mbar_arrive_expect_tx(&ud_full[g & 1], kUdBytes);
       bulk_load(Udb + (g & 1) * kUdFloats, p.Ud + (int64_t)(4 * k + s) * kUdFloats, kUdBytes, &ud_full[g & 1]);
     };
-    // W of item it's block, once every earlier contribution has landed
-    auto load_wb = [&](int it) {
-      const int k = item_k(it), slab = item_slab(it);
-      if (!q_wait_ge(p, &p.cnt[(int64_t)slab * T + k], k)) return false;
-      fence_proxy_async_global();
-      for (int c = 0; c < 4; ++c) {
-        if (it > 0 && !q_mbar_wait(p, &wb_empty[c], (it - 1) & 1)) return false;
-        mbar_arrive_expect_tx(&wb_full[c], kQChunk);
-        tma_load_2d(Wb + c * kQChunk, &mp.wld, &wb_full[c], QB * k + SB * c, QB * slab);
-      }
+    // chunk c of item it's W, once the workers' contributions have landed
+    // (wait: block until they have; else give up at once if they have not)
+    auto wb_ready = [&](int it, bool wait) {
+      const int* f = &p.cnt[(int64_t)item_slab(it) * T + item_k(it)];
+      const int need = worker_count(item_k(it));
+      if (wait) return q_wait_ge(p, f, need);
+      if (*(volatile const int*)f < need) return false;
+      __threadfence();
       return true;
+    };
+    auto load_wb = [&](int it, int c) {
+      const int k = item_k(it), slab = item_slab(it);
+      mbar_arrive_expect_tx(&wb_full[c], kQChunk);
+      tma_load_2d(Wb + c * kQChunk, &mp.wld, &wb_full[c], QB * k + SB * c, QB * slab);
     };
     load_ud(0);
     if (4 * nitems > 1) load_ud(1);
     load_ub(0);
     if (3 * nitems > 1) load_ub(1);
-    ok = load_wb(0);
+    if (has_next(0)) load_un(0);
+    int un_used = 0;
+    ok = wb_ready(0, true);
+    if (ok) {
+      fence_proxy_async_global();
+      for (int c = 0; c < 4; ++c) load_wb(0, c);
+    }
     const uint32_t ah = smem_u32(Ab), al = ah + kQChunk;
     for (int it = 0; ok && it < nitems; ++it) {
       const int k = item_k(it), slab = item_slab(it);
+      const uint32_t dcur = acc(it, 0), dnext = acc(it, 1);
+      // in-block products add to what D_cur holds unless it starts afresh
+      const bool fresh = !(cn && k > 0);
+      int wb_next = 0;  // chunks of item it + 1's W already requested
       for (int s = 0; s < 4; ++s) {
         const int g = 4 * it + s;
         if (!q_mbar_wait(p, &a_full, g & 1)) {
@@ -289,35 +478,52 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
           break;
         }
         if (s < 3) {
-          // D[r][c] += sum_j A[r][j] U[j][c] for the block's columns after
-          // this sub-block: first the next sub-block's 32 (the chain waits
-          // for them), then the rest
           const int u = 3 * it + s;
           if (!q_mbar_wait(p, &ub_full[u & 1], (u >> 1) & 1)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t bh = smem_u32(Ub) + 2 * (u & 1) * kQChunk, bl = bh + kQChunk;
-          const uint32_t cn = SB * (s + 1), cr = SB * (s + 2);
-          issue_mma_chunk(tbase + cn, ah, al, bh + cn * 128, bl + cn * 128, make_idesc(2, 128, SB), s > 0);
-          umma_commit(&mma_next);
-          if (cr < QB)
-            issue_mma_chunk(tbase + cr, ah, al, bh + cr * 128, bl + cr * 128, make_idesc(2, 128, QB - cr), s > 0);
-          umma_commit(&mma_done);
         }
+        const bool nx = has_next(g);
+        if (nx) {
+          if (!q_mbar_wait(p, &un_full, un_used & 1)) {
+            ok = false;
+            break;
+          }
+          ++un_used;
+        }
+        tc_fence_after();
+        // D_cur[r][c] += sum_j A[r][j] U[j][c] for the block's columns after
+        // this sub-block (first the next sub-block's 32, which the rows wait
+        // for, then the rest), and D_next for all of the next block
+        const bool accum = s > 0 || !fresh;
+        if (s < 3) {
+          const int u = 3 * it + s;
+          const uint32_t bh = smem_u32(Ub) + 2 * (u & 1) * kQChunk, bl = bh + kQChunk;
+          const uint32_t c1 = SB * (s + 1), c2 = SB * (s + 2);
+          issue_mma_chunk(dcur + c1, ah, al, bh + c1 * 128, bl + c1 * 128, make_idesc(2, 128, SB), accum);
+          umma_commit(&mma_next);
+          if (c2 < QB)
+            issue_mma_chunk(dcur + c2, ah, al, bh + c2 * 128, bl + c2 * 128, make_idesc(2, 128, QB - c2), accum);
+        } else {
+          umma_commit(&mma_next);
+        }
+        if (nx) {
+          const uint32_t nh = smem_u32(Un);
+          issue_mma_chunk(dnext, ah, al, nh, nh + kQChunk, make_idesc(2, 128, QB), s > 0);
+        }
+        umma_commit(&mma_done);
         // the sub-block's -E (hi, lo) for the workers
         tma_store_2d(&mp.eh, Ab, QB * k + SB * s, QB * slab);
         tma_store_2d(&mp.el, Ab + kQChunk, QB * k + SB * s, QB * slab);
         bulk_commit();
-        if (s < 3) {
-          const int u = 3 * it + s;
-          if (!q_mbar_wait(p, &mma_done, u & 1)) {
-            ok = false;
-            break;
-          }
-          if (u + 2 < 3 * nitems) load_ub(u + 2);
+        if (!q_mbar_wait(p, &mma_done, g & 1)) {
+          ok = false;
+          break;
         }
+        if (s < 3 && 3 * it + s + 2 < 3 * nitems) load_ub(3 * it + s + 2);
+        // (the items without a next block are the last ones of the launch)
+        if (has_next(g + 1)) load_un(g + 1);
         bulk_wait_read<0>();
         mbar_arrive(&a_empty);
         if (g + 2 < 4 * nitems) {
@@ -327,6 +533,19 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
           }
           load_ud(g + 2);
         }
+        // item it + 1's W, chunk by chunk as the rows finish with this item's
+        // (requested early when its earlier contributions are already in)
+        if (it + 1 < nitems && wb_next <= s && wb_ready(it + 1, false)) {
+          fence_proxy_async_global();
+          for (; wb_next <= s; ++wb_next) {
+            if (!q_mbar_wait(p, &wb_empty[wb_next], it & 1)) {
+              ok = false;
+              break;
+            }
+            load_wb(it + 1, wb_next);
+          }
+        }
+        if (!ok) break;
       }
       if (!ok) break;
       // block k of the slab: its -E has landed
@@ -334,19 +553,34 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
       fence_proxy_async_global();
       __threadfence();
       atomicExch(&p.sdone[slab], k + 1);
-      if (it + 1 < nitems && !load_wb(it + 1)) ok = false;
+      if (it + 1 < nitems && wb_next < 4) {
+        if (!wb_ready(it + 1, true)) {
+          ok = false;
+          break;
+        }
+        fence_proxy_async_global();
+        for (; wb_next < 4; ++wb_next) {
+          if (!q_mbar_wait(p, &wb_empty[wb_next], it & 1)) {
+            ok = false;
+            break;
+          }
+          load_wb(it + 1, wb_next);
+        }
+      }
     }
     if (!ok) q_give_up(p);
   } else if (threadIdx.x < 128) {
     // ------------------------------------------------------------ the rows
     const int rl = threadIdx.x;
-    const uint32_t tl_addr = tbase + ((uint32_t)(warp * 32) << 16);
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float fmaxq = (float)p.maxq;
     for (int it = 0; ok && it < nitems; ++it) {
       const int k = item_k(it), slab = item_slab(it);
       const int64_t row = (int64_t)slab * QB + rl;
       const bool live = row < p.out;
       const int64_t kB = (int64_t)QB * k;
+      const uint32_t dcur = acc(it, 0) + lane_off;
+      const bool dprev = cn && k > 0;  // D_cur already holds the previous block's product
       float s_ = 1.f, z_ = 0.f, lsum = 0.f;
       const bool gstart0 = GSB == QB && (p.gs == -1 ? k == 0 : kB % p.gs == 0);
       if (GSB == QB && !gstart0 && live) {
@@ -356,6 +590,7 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
         z_ = (float)p.zeros[row * p.ngroups + gi];
       }
       float inv_s = __frcp_rn(s_);
+#pragma unroll 1
       for (int s = 0; s < 4; ++s) {
         const int g = 4 * it + s;
         const int64_t c0 = kB + SB * s;  // first column of the sub-block
@@ -364,26 +599,26 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
           ok = false;
           break;
         }
-        if (s > 0) {
-          if (!q_mbar_wait(p, &mma_next, (3 * it + s - 1) & 1)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        // every product into this sub-block's columns has completed: the
+        // previous sub-block's (s > 0) or all of the previous item's (s = 0)
+        if (g > 0 && !q_mbar_wait(p, s > 0 ? &mma_next : &mma_done, (g - 1) & 1)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
         load_row(Wb + s * kQChunk, rl, x);
-        if (s > 0) add_tmem(tl_addr + SB * s, x);
+        if (s > 0 || dprev) add_tmem(dcur + SB * s, x);
         mbar_arrive(&wb_empty[s]);
         // group starts whose group reaches past this sub-block
         if (GSB == 64 && (s & 1) == 0 && c0 < p.in) {
-          if (!q_mbar_wait(p, &wb_full[s + 1], it & 1) || (s > 0 && !q_mbar_wait(p, &mma_done, (3 * it + s - 1) & 1))) {
+          if (!q_mbar_wait(p, &wb_full[s + 1], it & 1) || (s > 0 && !q_mbar_wait(p, &mma_done, (g - 1) & 1))) {
             ok = false;
             break;
           }
           tc_fence_after();
           float y[32];
           load_row(Wb + (s + 1) * kQChunk, rl, y);
-          if (s > 0) add_tmem(tl_addr + SB * (s + 1), y);
+          if (s > 0 || dprev) add_tmem(dcur + SB * (s + 1), y);
           float lo = INFINITY, hi = -INFINITY, am = 0.f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
@@ -398,9 +633,8 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
           }
         }
         if (GSB == QB && s == 0 && gstart0) {
-          // the whole block (no update has reached it yet in this block), and
-          // the group's columns past it: those need every earlier block's
-          // contribution, as this block has
+          // the whole block as it stands, and the group's columns past it:
+          // those need every earlier block's contribution, as this block has
           float lo = INFINITY, hi = -INFINITY, am = 0.f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) minmax(x[i], lo, hi, am);
@@ -411,6 +645,7 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
             }
             float y[32];
             load_row(Wb + c * kQChunk, rl, y);
+            if (dprev) add_tmem(dcur + SB * c, y);
 #pragma unroll
             for (int i = 0; i < 32; ++i) minmax(y[i], lo, hi, am);
           }
@@ -439,47 +674,21 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
         }
         const float* ud = Udb + (g & 1) * kUdFloats;
         uint32_t cw[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) cw[i] = 0u;
-#pragma unroll
-        for (int j = 0; j < SB; ++j) {
-          if (GSB <= SB && j % GSB == 0 && c0 + j < p.in) {
-            float lo = INFINITY, hi = -INFINITY, am = 0.f;
-#pragma unroll
-            for (int i = j; i < j + (GSB <= SB ? GSB : 1); ++i) minmax(x[i], lo, hi, am);
-            group_params(lo, hi, am, p.sym, fmaxq, s_, z_);
-            inv_s = __frcp_rn(s_);
-            if (live) {
-              p.scales[row * p.ngroups + (c0 + j) / GSB] = s_;
-              p.zeros[row * p.ngroups + (c0 + j) / GSB] = (int32_t)z_;
-            }
-          }
-          const float xv = x[j];
-          float qf = round_div(xv, s_, inv_s) + z_;
-          qf = fminf(fmaxf(qf, 0.f), fmaxq);
-          const float deq = s_ * (qf - z_);
-          float e = (xv - deq) * ud[SB * SB + j];
-          e = c0 + j < p.in ? e : 0.f;
-          lsum = fmaf(e, e, lsum);
-          cw[j >> 2] |= (uint32_t)qf << (8 * (j & 3));
-          x[j] = -e;
-          // the sub-block's later columns: x[j'] -= e U[j][j']
-          const float* ur = ud + j * SB;
-#pragma unroll
-          for (int a = (j + 1) >> 2; a < 8; ++a) {
-            const float4 u = *reinterpret_cast<const float4*>(ur + 4 * a);
-            if (4 * a + 0 > j) x[4 * a + 0] = fmaf(-e, u.x, x[4 * a + 0]);
-            if (4 * a + 1 > j) x[4 * a + 1] = fmaf(-e, u.y, x[4 * a + 1]);
-            if (4 * a + 2 > j) x[4 * a + 2] = fmaf(-e, u.z, x[4 * a + 2]);
-            if (4 * a + 3 > j) x[4 * a + 3] = fmaf(-e, u.w, x[4 * a + 3]);
+        {
+          // the sub-block's columns with the divide-free quotient; a row
+          // that met a quotient outside its range replays them with the
+          // divide (its values at the sub-block's start wait in Xs for that)
+          store_row(Xs, rl, x);
+          RowState st{s_, z_, inv_s, lsum};
+          if (sweep32<GSB, true>(x, ud, c0, p, row, live, fmaxq, s_, z_, inv_s, lsum, cw)) {
+            store_codes(p, row, c0, live, cw);
+          } else {
+            st = replay32<GSB>(Xs, rl, ud, c0, p, row, live, fmaxq, st);
+            s_ = st.s, z_ = st.z, inv_s = st.inv_s, lsum = st.lsum;
+            load_row(Xs, rl, x);
           }
         }
         mbar_arrive(&ud_empty[g & 1]);
-        if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(p.codes_p + row * np + c0);
-          dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-          dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-        }
         // -E of the sub-block, split, as the MMA operand (row rl, K-major)
         if (g > 0 && !q_mbar_wait(p, &a_empty, (g - 1) & 1)) {
           ok = false;
@@ -516,42 +725,63 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tbase, 128);
+    tmem_dealloc(tbase, tcols);
   }
 }
 
 // ------------------------------------------------------------------ workers
-// Task t (all workers, in order): block k, then the column block c = k + 1,
-// k + 2, ..., then the slab.  Thread 0 loads, thread 96 issues the MMAs,
+// A task is one slab's block k applied to a run of up to kRun consecutive
+// column blocks c (from k + 1, or k + 2 when the chains take the next
+// block): W[slab, c] += (-E[slab, k]) U[k, c]^T for each c of the run.  The
+// slab's -E (128 x 128, split) stays in shared memory for the whole run and
+// only U's tiles stream through a two-slot ring of K chunks, so a tile costs
+// 128 KB of operand reads rather than 256 KB.  Tasks go in order of k, then
+// run (nearest first), then slab.  Thread 0 loads, thread 96 issues the MMAs,
 // threads 128-255 run the epilogue; two tensor-memory accumulators let a
-// task's epilogue overlap the next task's MMAs.
+// tile's epilogue overlap the next tile's MMAs.
+constexpr int kRun = 4;
+
 struct QTask {
-  int k, c, slab;
+  int k, c0, c1, slab;  // column blocks [c0, c1)
 };
 
+__host__ __device__ __forceinline__ int runs_of_block(int T, int k, int first) {
+  const int later = T - k - first;  // column blocks k + first .. T - 1
+  return later > 0 ? (later + kRun - 1) / kRun : 0;
+}
+
+__host__ __device__ __forceinline__ int64_t total_tasks(int64_t nslab, int T, int first) {
+  int64_t n = 0;
+  for (int k = 0; k < T; ++k) n += nslab * runs_of_block(T, k, first);
+  return n;
+}
+
 struct TaskWalk {
-  int k;
+  int k, first;
   int64_t base, count;
-  __device__ explicit TaskWalk(const SolveParams& p) : k(0), base(0), count((int64_t)p.nslab * (p.T - 1)) {}
+  __device__ explicit TaskWalk(const SolveParams& p)
+      : k(0), first(1 + p.chain_next), base(0), count((int64_t)p.nslab * runs_of_block(p.T, 0, 1 + p.chain_next)) {}
   __device__ QTask at(int64_t t, const SolveParams& p) {
     while (t >= base + count) {
       base += count;
       ++k;
-      count = (int64_t)p.nslab * (p.T - 1 - k);
+      count = (int64_t)p.nslab * runs_of_block(p.T, k, first);
     }
     const int64_t idx = t - base;
     QTask q;
     q.k = k;
-    q.c = k + 1 + (int)(idx / p.nslab);
+    q.c0 = k + first + kRun * (int)(idx / p.nslab);
+    q.c1 = q.c0 + kRun < p.T ? q.c0 + kRun : p.T;
     q.slab = (int)(idx % p.nslab);
     return q;
   }
 };
 
 __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParams& p, uint8_t* sm) {
-  uint8_t* ring = sm + kWRing;
+  uint8_t* Eb = sm + kWE;      // -E of the task's slab and block: 4 chunks hi, then 4 lo
+  uint8_t* ring = sm + kWRing; // 2 slots x (U hi, U lo) chunks
   float* stg = reinterpret_cast<float*>(sm + kWStg);
-  __shared__ uint64_t st_full[2], st_empty[2], acc_full[2], acc_empty[2], drain;
+  __shared__ uint64_t st_full[2], st_empty[2], acc_full[2], acc_empty[2], e_full, e_empty, drain;
   __shared__ uint32_t tslot;
   __shared__ int epi_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -562,6 +792,8 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    mbar_init(&e_full, 1);
+    mbar_init(&e_empty, 1);
     mbar_init(&drain, 1);
     epi_abort = 0;
     fence_mbar_init();
@@ -576,7 +808,7 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
   const uint32_t tbase = tslot;
   const int T = p.T;
   const int W = (int)gridDim.x - p.nchain, slot = (int)blockIdx.x - p.nchain;
-  const int64_t total = (int64_t)p.nslab * T * (T - 1) / 2;
+  const int64_t total = total_tasks(p.nslab, T, 1 + p.chain_next);
   const uint32_t idesc = make_idesc(2, 128, 128);
   if (threadIdx.x == 0) {
     // ------------------------------------------------------------ loader
@@ -586,57 +818,75 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
     tma_prefetch_desc(&mp.el);
     TaskWalk tw(p);
     bool ok = true;
-    int tl = 0;
-    for (int64_t t = slot; ok && t < total; t += W, ++tl) {
-      const QTask q = tw.at(t, p);
-      for (int ch = 0; ch < 4; ++ch) {
-        const int g = 4 * tl + ch, rs = g & 1;
-        if (g >= 2 && !q_mbar_wait(p, &st_empty[rs], ((g >> 1) - 1) & 1)) {
-          ok = false;
-          break;
-        }
-        uint8_t* dst = ring + 4 * rs * kQChunk;
-        const int32_t xk = QB * q.k + SB * ch;
-        mbar_arrive_expect_tx(&st_full[rs], 4 * kQChunk);
-        tma_load_2d(dst, &mp.uh, &st_full[rs], xk, QB * q.c);
-        tma_load_2d(dst + kQChunk, &mp.ul, &st_full[rs], xk, QB * q.c);
-        if (ch == 0) {
-          // the slab's block k: its -E published by the chain
-          if (!q_wait_ge(p, &p.sdone[q.slab], q.k + 1)) {
+    int g = 0;  // U chunks loaded so far
+    int q = 0;  // tasks so far
+    for (int64_t t = slot; ok && t < total; t += W, ++q) {
+      const QTask x = tw.at(t, p);
+      for (int c = x.c0; ok && c < x.c1; ++c) {
+        for (int ch = 0; ch < 4; ++ch, ++g) {
+          const int rs = g & 1;
+          if (g >= 2 && !q_mbar_wait(p, &st_empty[rs], ((g >> 1) - 1) & 1)) {
             ok = false;
             break;
           }
-          fence_proxy_async_global();
+          uint8_t* dst = ring + 2 * rs * kQChunk;
+          const int32_t xk = QB * x.k + SB * ch;
+          mbar_arrive_expect_tx(&st_full[rs], 2 * kQChunk);
+          tma_load_2d(dst, &mp.uh, &st_full[rs], xk, QB * c);
+          tma_load_2d(dst + kQChunk, &mp.ul, &st_full[rs], xk, QB * c);
+          if (c == x.c0 && ch == 0) {
+            // the slab's -E for block k, published by its chain, once the
+            // previous task's products are done with the buffer
+            if ((q > 0 && !q_mbar_wait(p, &e_empty, (q - 1) & 1)) ||
+                !q_wait_ge(p, &p.sdone[x.slab], x.k + 1)) {
+              ok = false;
+              break;
+            }
+            fence_proxy_async_global();
+            mbar_arrive_expect_tx(&e_full, 8 * kQChunk);
+            for (int ec = 0; ec < 4; ++ec) {
+              tma_load_2d(Eb + ec * kQChunk, &mp.eh, &e_full, QB * x.k + SB * ec, QB * x.slab);
+              tma_load_2d(Eb + (4 + ec) * kQChunk, &mp.el, &e_full, QB * x.k + SB * ec, QB * x.slab);
+            }
+          }
         }
-        tma_load_2d(dst + 2 * kQChunk, &mp.eh, &st_full[rs], xk, QB * q.slab);
-        tma_load_2d(dst + 3 * kQChunk, &mp.el, &st_full[rs], xk, QB * q.slab);
       }
     }
     if (!ok) q_give_up(p);
   } else if (threadIdx.x == 96) {
     // ------------------------------------------------------------ MMA issue
+    TaskWalk tw(p);
     bool ok = true;
-    int tl = 0;
-    for (int64_t t = slot; ok && t < total; t += W, ++tl) {
-      const int buf = tl & 1, use = tl >> 1;
-      if (use > 0 && !q_mbar_wait(p, &acc_empty[buf], (use - 1) & 1)) {
+    int g = 0, tl = 0, q = 0;
+    const uint32_t eb = smem_u32(Eb);
+    for (int64_t t = slot; ok && t < total; t += W, ++q) {
+      const QTask x = tw.at(t, p);
+      if (!q_mbar_wait(p, &e_full, q & 1)) {
         ok = false;
         break;
       }
-      const uint32_t d = tbase + (uint32_t)buf * 128;
-      for (int ch = 0; ch < 4; ++ch) {
-        const int g = 4 * tl + ch, rs = g & 1;
-        if (!q_mbar_wait(p, &st_full[rs], (g >> 1) & 1)) {
+      for (int c = x.c0; ok && c < x.c1; ++c, ++tl) {
+        const int buf = tl & 1, use = tl >> 1;
+        if (use > 0 && !q_mbar_wait(p, &acc_empty[buf], (use - 1) & 1)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint32_t base = smem_u32(ring) + 4 * rs * kQChunk;
-        // D[c][r] (+)= sum_j U^T[c][j] (-E)[r][j]: lanes are W's columns
-        issue_mma_chunk(d, base, base + kQChunk, base + 2 * kQChunk, base + 3 * kQChunk, idesc, ch > 0);
-        umma_commit(&st_empty[rs]);
+        const uint32_t d = tbase + (uint32_t)buf * 128;
+        for (int ch = 0; ch < 4; ++ch, ++g) {
+          const int rs = g & 1;
+          if (!q_mbar_wait(p, &st_full[rs], (g >> 1) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ub = smem_u32(ring) + 2 * rs * kQChunk;
+          // D[c][r] (+)= sum_j U^T[c][j] (-E)[r][j]: lanes are W's columns
+          issue_mma_chunk(d, ub, ub + kQChunk, eb + ch * kQChunk, eb + (4 + ch) * kQChunk, idesc, ch > 0);
+          umma_commit(&st_empty[rs]);
+        }
+        if (ok) umma_commit(&acc_full[buf]);
       }
-      if (ok) umma_commit(&acc_full[buf]);
+      if (ok) umma_commit(&e_empty);
     }
     if (!ok) q_give_up(p);
   } else if (threadIdx.x >= 128) {
@@ -645,44 +895,50 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
     const int cl = quarter * 32 + lane;
     TaskWalk tw(p);
     int tl = 0, epi_pass = 0;
-    for (int64_t t = slot; t < total; t += W, ++tl) {
-      const QTask q = tw.at(t, p);
-      const int buf = tl & 1;
-      bool ok = q_mbar_wait(p, &acc_full[buf], (tl >> 1) & 1, true);
-      if (threadIdx.x == 128 && ok) {
-        // contributions reach a tile in order of k
-        ok = q_wait_ge(p, &p.cnt[(int64_t)q.slab * T + q.c], q.k);
-        fence_proxy_async_global();
-      }
-      if (!ok) epi_abort = 1;
-      named_bar_sync(2, 128);
-      if (epi_abort) break;  // the same decision in all 128 threads
-      tc_fence_after();
-      const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
-#pragma unroll 1
-      for (int pz = 0; pz < 4; ++pz) {
-        float v[32];
-        tmem_ld32(taddr + (uint32_t)(32 * pz), v);
-        float* sb = stg + (epi_pass % kWStages) * (32 * 128);
-        if (threadIdx.x == 128) bulk_wait_read<kWStages - 1>();  // the reduce that last read sb is done
-        named_bar_sync(2, 128);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) sb[j * 128 + cl] = v[j];
-        fence_proxy_async_smem();
-        named_bar_sync(2, 128);
-        if (threadIdx.x == 128) {
-          tma_reduce_add_2d(&mp.wred, sb, QB * q.c, QB * q.slab + 32 * pz);
-          bulk_commit();
+    bool stop = false;
+    for (int64_t t = slot; !stop && t < total; t += W) {
+      const QTask x = tw.at(t, p);
+      for (int c = x.c0; c < x.c1; ++c, ++tl) {
+        const int buf = tl & 1;
+        bool ok = q_mbar_wait(p, &acc_full[buf], (tl >> 1) & 1, true);
+        if (threadIdx.x == 128 && ok) {
+          // contributions reach a tile in order of k
+          ok = q_wait_ge(p, &p.cnt[(int64_t)x.slab * T + c], x.k);
+          fence_proxy_async_global();
         }
-        ++epi_pass;
-      }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
-      if (threadIdx.x == 128) {
-        bulk_wait_all();
-        fence_proxy_async_global();
-        __threadfence();
-        atomicExch(&p.cnt[(int64_t)q.slab * T + q.c], q.k + 1);
+        if (!ok) epi_abort = 1;
+        named_bar_sync(2, 128);
+        if (epi_abort) {  // the same decision in all 128 threads
+          stop = true;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+        for (int pz = 0; pz < 4; ++pz) {
+          float v[32];
+          tmem_ld32(taddr + (uint32_t)(32 * pz), v);
+          float* sb = stg + (epi_pass % kWStages) * (32 * 128);
+          if (threadIdx.x == 128) bulk_wait_read<kWStages - 1>();  // the reduce that last read sb is done
+          named_bar_sync(2, 128);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) sb[j * 128 + cl] = v[j];
+          fence_proxy_async_smem();
+          named_bar_sync(2, 128);
+          if (threadIdx.x == 128) {
+            tma_reduce_add_2d(&mp.wred, sb, QB * c, QB * x.slab + 32 * pz);
+            bulk_commit();
+          }
+          ++epi_pass;
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
+        if (threadIdx.x == 128) {
+          bulk_wait_all();
+          fence_proxy_async_global();
+          __threadfence();
+          atomicExch(&p.cnt[(int64_t)x.slab * T + c], x.k + 1);
+        }
       }
     }
   }
@@ -779,7 +1035,9 @@ cudaError_t solve_quantize(float* Wp, int64_t out, int64_t in, int64_t np_, cons
   const int cap = std::max(1, gmax / 4);
   const int spc = (nslab + cap - 1) / cap;
   const int nchain = (nslab + spc - 1) / spc;
-  const int64_t ntask = (int64_t)nslab * T * (T - 1) / 2;
+  // up to two slabs per chain, the chains also take each slab's next block
+  const int chain_next = spc <= 2 ? 1 : 0;
+  const int64_t ntask = total_tasks(nslab, T, 1 + chain_next);
   const int nworker = ntask > 0 ? (int)std::min<int64_t>(gmax - nchain, ntask) : 0;
   if (ntask > 0 && nworker < 1) return cudaErrorInvalidConfiguration;
   e = cudaMemsetAsync(sync, 0, solve_sync_bytes(out, np_), st);
@@ -793,6 +1051,7 @@ cudaError_t solve_quantize(float* Wp, int64_t out, int64_t in, int64_t np_, cons
   p.T = T;
   p.nslab = nslab;
   p.nchain = nchain;
+  p.chain_next = chain_next;
   p.maxq = (1 << cfg->bits) - 1;
   p.sym = cfg->sym;
   p.gs = gs;

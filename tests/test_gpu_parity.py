@@ -242,6 +242,40 @@ def test_diagonal_hessian_gives_round_to_nearest_exactly(lib):
         assert np.array_equal(g["zeros"], z)
 
 
+def test_divide_free_quotient_matches_ieee_division(lib):
+    """The sweep's x / scale without a divide (reciprocal and two fma
+    corrections) against CUDA's IEEE division, bit for bit, on 2^30 pairs,
+    three quarters of them next to a half-integer quotient."""
+    n = 1 << 30
+    checked, bad = lib.gptq_selftest_quotient(n, seed=20261203)
+    assert checked > 0.9 * n, checked
+    assert bad == 0, bad
+
+
+@pytest.mark.parametrize("gs,sym", [(128, False), (32, True), (-1, False)])
+def test_tiny_weights_take_the_divide_and_scale_exactly(lib, gs, sym):
+    """Weights scaled by 2^-70 put every x / scale outside the divide-free
+    quotient's range, so every sub-block is replayed with the divide.  A
+    power-of-two scale is exact in fp32 and leaves every quotient as it was:
+    codes and zeros must equal the unscaled layer's, scales be 2^-70 times
+    theirs, and both match the oracle."""
+    import torch
+    S32, n = _prep_inputs(95, 384, 900, "correlated")
+    W32, _ = gen.small_case(96, 130, 384, 8)
+    W_t, W64 = exact_values(W32, "float32")
+    cfg = _cfg(lib, bits=4, group_size=gs, sym=sym, desc_act=True)
+    g1, ref = _check_quantize(lib, W_t.cuda(), W64, S32, n, cfg)
+    tiny = 2.0 ** -70
+    Wt2 = (W_t * tiny).contiguous()
+    Ucm = np.ascontiguousarray(ref["U"].T).astype(np.float32)
+    g2 = _run_quantize(lib, Wt2.cuda(), Ucm, ref["perm"], ref["dead"], cfg)
+    g1b = _run_quantize(lib, W_t.cuda(), Ucm, ref["perm"], ref["dead"], cfg)
+    assert np.array_equal(g2["codes"], g1b["codes"])
+    assert np.array_equal(g2["zeros"], g1b["zeros"])
+    assert np.array_equal(g2["scales"], (g1b["scales"].astype(np.float64) * tiny).astype(np.float32))
+    assert torch.all(torch.isfinite(torch.from_numpy(g2["loss"])))
+
+
 def test_block_size_variants_agree(lib):
     S32, n = _prep_inputs(91, 512, 1500, "correlated")
     W32, _ = gen.small_case(92, 64, 512, 8)
