@@ -58,10 +58,10 @@ constexpr uint32_t kCX = kCA + 2 * kQChunk;    // each row's values at the sub-b
 constexpr uint32_t kCUd = kCX + kQChunk;       // 2 slots of kUdBytes
 constexpr uint32_t kChainSmem = kCUd + 2 * kUdBytes;
 // worker CTA
-constexpr uint32_t kWE = 0;                    // -E of a slab's block: 4 K chunks, hi and lo
-constexpr uint32_t kWRing = kWE + 8 * kQChunk; // 2 slots x (U hi, U lo) chunks
-constexpr int kWStages = 2;                    // epilogue staging tiles, 32 rows x 128 columns fp32
-constexpr uint32_t kWStg = kWRing + 4 * kQChunk;
+constexpr int kWSlots = 2;                     // operand ring: K chunks of (U hi, U lo, E hi, E lo)
+constexpr uint32_t kWRing = 0;
+constexpr int kWStages = 4;                    // epilogue staging tiles, 32 rows x 128 columns fp32
+constexpr uint32_t kWStg = kWRing + 4 * kWSlots * kQChunk;
 constexpr uint32_t kWorkerSmem = kWStg + kWStages * 32 * 128 * 4;
 constexpr uint32_t kSolveSmem = 1024 + (kChainSmem > kWorkerSmem ? kChainSmem : kWorkerSmem);
 static_assert(kSolveSmem <= 232448, "shared memory per CTA");
@@ -473,6 +473,20 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
       int wb_next = 0;  // chunks of item it + 1's W already requested
       for (int s = 0; s < 4; ++s) {
         const int g = 4 * it + s;
+        // item it + 1's W, chunk by chunk as the rows take this item's chunk
+        // (they do at the start of sub-block s), once the next item's earlier
+        // contributions are in: then the chunk lands during this sub-block
+        if (it + 1 < nitems && wb_next <= s && wb_ready(it + 1, false)) {
+          fence_proxy_async_global();
+          for (; wb_next <= s; ++wb_next) {
+            if (!q_mbar_wait(p, &wb_empty[wb_next], it & 1)) {
+              ok = false;
+              break;
+            }
+            load_wb(it + 1, wb_next);
+          }
+          if (!ok) break;
+        }
         if (!q_mbar_wait(p, &a_full, g & 1)) {
           ok = false;
           break;
@@ -533,19 +547,6 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
           }
           load_ud(g + 2);
         }
-        // item it + 1's W, chunk by chunk as the rows finish with this item's
-        // (requested early when its earlier contributions are already in)
-        if (it + 1 < nitems && wb_next <= s && wb_ready(it + 1, false)) {
-          fence_proxy_async_global();
-          for (; wb_next <= s; ++wb_next) {
-            if (!q_mbar_wait(p, &wb_empty[wb_next], it & 1)) {
-              ok = false;
-              break;
-            }
-            load_wb(it + 1, wb_next);
-          }
-        }
-        if (!ok) break;
       }
       if (!ok) break;
       // block k of the slab: its -E has landed
@@ -730,70 +731,65 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
 }
 
 // ------------------------------------------------------------------ workers
-// A task is one slab's block k applied to a run of up to kRun consecutive
-// column blocks c (from k + 1, or k + 2 when the chains take the next
-// block): W[slab, c] += (-E[slab, k]) U[k, c]^T for each c of the run.  The
-// slab's -E (128 x 128, split) stays in shared memory for the whole run and
-// only U's tiles stream through a two-slot ring of K chunks, so a tile costs
-// 128 KB of operand reads rather than 256 KB.  Tasks go in order of k, then
-// run (nearest first), then slab.  Thread 0 loads, thread 96 issues the MMAs,
-// threads 128-255 run the epilogue; two tensor-memory accumulators let a
-// tile's epilogue overlap the next tile's MMAs.
-constexpr int kRun = 4;
-
+// A task is one 128 x 128 tile: W[slab, c] += (-E[slab, k]) U[k, c]^T, K =
+// 128, for a column block c from k + 1 on (k + 2 on when the chains take the
+// next block).  Tasks go in order of k, then c (nearest first), then slab.
+// The split operands (U^T and -E, hi and lo) stream through a ring of
+// kWSlots K chunks of 32 (64 KB each); the epilogue stages four 32-row
+// passes, so a tile's reduce-adds do not wait for one another's reads.
+// Thread 0 loads, thread 96 issues the MMAs, threads 128-255 run the
+// epilogue; two tensor-memory accumulators let a tile's epilogue overlap the
+// next tile's MMAs.
 struct QTask {
-  int k, c0, c1, slab;  // column blocks [c0, c1)
+  int k, c, slab;
 };
 
-__host__ __device__ __forceinline__ int runs_of_block(int T, int k, int first) {
+__host__ __device__ __forceinline__ int64_t tasks_of_block(int64_t nslab, int T, int k, int first) {
   const int later = T - k - first;  // column blocks k + first .. T - 1
-  return later > 0 ? (later + kRun - 1) / kRun : 0;
+  return later > 0 ? nslab * later : 0;
 }
 
 __host__ __device__ __forceinline__ int64_t total_tasks(int64_t nslab, int T, int first) {
-  int64_t n = 0;
-  for (int k = 0; k < T; ++k) n += nslab * runs_of_block(T, k, first);
-  return n;
+  const int64_t m = T - first;  // sum over k of (T - k - first)
+  return m > 0 ? nslab * m * (m + 1) / 2 : 0;
 }
 
 struct TaskWalk {
   int k, first;
   int64_t base, count;
   __device__ explicit TaskWalk(const SolveParams& p)
-      : k(0), first(1 + p.chain_next), base(0), count((int64_t)p.nslab * runs_of_block(p.T, 0, 1 + p.chain_next)) {}
+      : k(0), first(1 + p.chain_next), base(0), count(tasks_of_block(p.nslab, p.T, 0, 1 + p.chain_next)) {}
   __device__ QTask at(int64_t t, const SolveParams& p) {
     while (t >= base + count) {
       base += count;
       ++k;
-      count = (int64_t)p.nslab * runs_of_block(p.T, k, first);
+      count = tasks_of_block(p.nslab, p.T, k, first);
     }
     const int64_t idx = t - base;
     QTask q;
     q.k = k;
-    q.c0 = k + first + kRun * (int)(idx / p.nslab);
-    q.c1 = q.c0 + kRun < p.T ? q.c0 + kRun : p.T;
+    q.c = k + first + (int)(idx / p.nslab);
     q.slab = (int)(idx % p.nslab);
     return q;
   }
 };
 
 __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParams& p, uint8_t* sm) {
-  uint8_t* Eb = sm + kWE;      // -E of the task's slab and block: 4 chunks hi, then 4 lo
-  uint8_t* ring = sm + kWRing; // 2 slots x (U hi, U lo) chunks
+  uint8_t* ring = sm + kWRing;
   float* stg = reinterpret_cast<float*>(sm + kWStg);
-  __shared__ uint64_t st_full[2], st_empty[2], acc_full[2], acc_empty[2], e_full, e_empty, drain;
+  __shared__ uint64_t st_full[kWSlots], st_empty[kWSlots], acc_full[2], acc_empty[2], drain;
   __shared__ uint32_t tslot;
   __shared__ int epi_abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kWSlots; ++b) {
       mbar_init(&st_full[b], 1);
       mbar_init(&st_empty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
-    mbar_init(&e_full, 1);
-    mbar_init(&e_empty, 1);
     mbar_init(&drain, 1);
     epi_abort = 0;
     fence_mbar_init();
@@ -818,75 +814,57 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
     tma_prefetch_desc(&mp.el);
     TaskWalk tw(p);
     bool ok = true;
-    int g = 0;  // U chunks loaded so far
-    int q = 0;  // tasks so far
-    for (int64_t t = slot; ok && t < total; t += W, ++q) {
-      const QTask x = tw.at(t, p);
-      for (int c = x.c0; ok && c < x.c1; ++c) {
-        for (int ch = 0; ch < 4; ++ch, ++g) {
-          const int rs = g & 1;
-          if (g >= 2 && !q_mbar_wait(p, &st_empty[rs], ((g >> 1) - 1) & 1)) {
+    int g = 0;  // K chunks loaded so far
+    for (int64_t t = slot; ok && t < total; t += W) {
+      const QTask q = tw.at(t, p);
+      for (int ch = 0; ch < 4; ++ch, ++g) {
+        const int rs = g % kWSlots, use = g / kWSlots;
+        if (use > 0 && !q_mbar_wait(p, &st_empty[rs], (use - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        uint8_t* dst = ring + 4 * rs * kQChunk;
+        const int32_t xk = QB * q.k + SB * ch;
+        mbar_arrive_expect_tx(&st_full[rs], 4 * kQChunk);
+        tma_load_2d(dst, &mp.uh, &st_full[rs], xk, QB * q.c);
+        tma_load_2d(dst + kQChunk, &mp.ul, &st_full[rs], xk, QB * q.c);
+        if (ch == 0) {
+          // the slab's block k: its -E published by the chain
+          if (!q_wait_ge(p, &p.sdone[q.slab], q.k + 1)) {
             ok = false;
             break;
           }
-          uint8_t* dst = ring + 2 * rs * kQChunk;
-          const int32_t xk = QB * x.k + SB * ch;
-          mbar_arrive_expect_tx(&st_full[rs], 2 * kQChunk);
-          tma_load_2d(dst, &mp.uh, &st_full[rs], xk, QB * c);
-          tma_load_2d(dst + kQChunk, &mp.ul, &st_full[rs], xk, QB * c);
-          if (c == x.c0 && ch == 0) {
-            // the slab's -E for block k, published by its chain, once the
-            // previous task's products are done with the buffer
-            if ((q > 0 && !q_mbar_wait(p, &e_empty, (q - 1) & 1)) ||
-                !q_wait_ge(p, &p.sdone[x.slab], x.k + 1)) {
-              ok = false;
-              break;
-            }
-            fence_proxy_async_global();
-            mbar_arrive_expect_tx(&e_full, 8 * kQChunk);
-            for (int ec = 0; ec < 4; ++ec) {
-              tma_load_2d(Eb + ec * kQChunk, &mp.eh, &e_full, QB * x.k + SB * ec, QB * x.slab);
-              tma_load_2d(Eb + (4 + ec) * kQChunk, &mp.el, &e_full, QB * x.k + SB * ec, QB * x.slab);
-            }
-          }
+          fence_proxy_async_global();
         }
+        tma_load_2d(dst + 2 * kQChunk, &mp.eh, &st_full[rs], xk, QB * q.slab);
+        tma_load_2d(dst + 3 * kQChunk, &mp.el, &st_full[rs], xk, QB * q.slab);
       }
     }
     if (!ok) q_give_up(p);
   } else if (threadIdx.x == 96) {
     // ------------------------------------------------------------ MMA issue
-    TaskWalk tw(p);
     bool ok = true;
-    int g = 0, tl = 0, q = 0;
-    const uint32_t eb = smem_u32(Eb);
-    for (int64_t t = slot; ok && t < total; t += W, ++q) {
-      const QTask x = tw.at(t, p);
-      if (!q_mbar_wait(p, &e_full, q & 1)) {
+    int tl = 0, g = 0;
+    for (int64_t t = slot; ok && t < total; t += W, ++tl) {
+      const int buf = tl & 1, use = tl >> 1;
+      if (use > 0 && !q_mbar_wait(p, &acc_empty[buf], (use - 1) & 1)) {
         ok = false;
         break;
       }
-      for (int c = x.c0; ok && c < x.c1; ++c, ++tl) {
-        const int buf = tl & 1, use = tl >> 1;
-        if (use > 0 && !q_mbar_wait(p, &acc_empty[buf], (use - 1) & 1)) {
+      const uint32_t d = tbase + (uint32_t)buf * 128;
+      for (int ch = 0; ch < 4; ++ch, ++g) {
+        const int rs = g % kWSlots;
+        if (!q_mbar_wait(p, &st_full[rs], (g / kWSlots) & 1)) {
           ok = false;
           break;
         }
-        const uint32_t d = tbase + (uint32_t)buf * 128;
-        for (int ch = 0; ch < 4; ++ch, ++g) {
-          const int rs = g & 1;
-          if (!q_mbar_wait(p, &st_full[rs], (g >> 1) & 1)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t ub = smem_u32(ring) + 2 * rs * kQChunk;
-          // D[c][r] (+)= sum_j U^T[c][j] (-E)[r][j]: lanes are W's columns
-          issue_mma_chunk(d, ub, ub + kQChunk, eb + ch * kQChunk, eb + (4 + ch) * kQChunk, idesc, ch > 0);
-          umma_commit(&st_empty[rs]);
-        }
-        if (ok) umma_commit(&acc_full[buf]);
+        tc_fence_after();
+        const uint32_t base = smem_u32(ring) + 4 * rs * kQChunk;
+        // D[c][r] (+)= sum_j U^T[c][j] (-E)[r][j]: lanes are W's columns
+        issue_mma_chunk(d, base, base + kQChunk, base + 2 * kQChunk, base + 3 * kQChunk, idesc, ch > 0);
+        umma_commit(&st_empty[rs]);
       }
-      if (ok) umma_commit(&e_empty);
+      if (ok) umma_commit(&acc_full[buf]);
     }
     if (!ok) q_give_up(p);
   } else if (threadIdx.x >= 128) {
@@ -895,50 +873,44 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
     const int cl = quarter * 32 + lane;
     TaskWalk tw(p);
     int tl = 0, epi_pass = 0;
-    bool stop = false;
-    for (int64_t t = slot; !stop && t < total; t += W) {
-      const QTask x = tw.at(t, p);
-      for (int c = x.c0; c < x.c1; ++c, ++tl) {
-        const int buf = tl & 1;
-        bool ok = q_mbar_wait(p, &acc_full[buf], (tl >> 1) & 1, true);
-        if (threadIdx.x == 128 && ok) {
-          // contributions reach a tile in order of k
-          ok = q_wait_ge(p, &p.cnt[(int64_t)x.slab * T + c], x.k);
-          fence_proxy_async_global();
-        }
-        if (!ok) epi_abort = 1;
-        named_bar_sync(2, 128);
-        if (epi_abort) {  // the same decision in all 128 threads
-          stop = true;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
+    for (int64_t t = slot; t < total; t += W, ++tl) {
+      const QTask q = tw.at(t, p);
+      const int buf = tl & 1;
+      bool ok = q_mbar_wait(p, &acc_full[buf], (tl >> 1) & 1, true);
+      if (threadIdx.x == 128 && ok) {
+        // contributions reach a tile in order of k
+        ok = q_wait_ge(p, &p.cnt[(int64_t)q.slab * T + q.c], q.k);
+        fence_proxy_async_global();
+      }
+      if (!ok) epi_abort = 1;
+      named_bar_sync(2, 128);
+      if (epi_abort) break;  // the same decision in all 128 threads
+      tc_fence_after();
+      const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
-        for (int pz = 0; pz < 4; ++pz) {
-          float v[32];
-          tmem_ld32(taddr + (uint32_t)(32 * pz), v);
-          float* sb = stg + (epi_pass % kWStages) * (32 * 128);
-          if (threadIdx.x == 128) bulk_wait_read<kWStages - 1>();  // the reduce that last read sb is done
-          named_bar_sync(2, 128);
+      for (int pz = 0; pz < 4; ++pz) {
+        float v[32];
+        tmem_ld32(taddr + (uint32_t)(32 * pz), v);
+        float* sb = stg + (epi_pass % kWStages) * (32 * 128);
+        if (threadIdx.x == 128) bulk_wait_read<kWStages - 1>();  // the reduce that last read sb is done
+        named_bar_sync(2, 128);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) sb[j * 128 + cl] = v[j];
-          fence_proxy_async_smem();
-          named_bar_sync(2, 128);
-          if (threadIdx.x == 128) {
-            tma_reduce_add_2d(&mp.wred, sb, QB * c, QB * x.slab + 32 * pz);
-            bulk_commit();
-          }
-          ++epi_pass;
-        }
-        tc_fence_before();
-        mbar_arrive(&acc_empty[buf]);
+        for (int j = 0; j < 32; ++j) sb[j * 128 + cl] = v[j];
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
         if (threadIdx.x == 128) {
-          bulk_wait_all();
-          fence_proxy_async_global();
-          __threadfence();
-          atomicExch(&p.cnt[(int64_t)x.slab * T + c], x.k + 1);
+          tma_reduce_add_2d(&mp.wred, sb, QB * q.c, QB * q.slab + 32 * pz);
+          bulk_commit();
         }
+        ++epi_pass;
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      if (threadIdx.x == 128) {
+        bulk_wait_all();
+        fence_proxy_async_global();
+        __threadfence();
+        atomicExch(&p.cnt[(int64_t)q.slab * T + q.c], q.k + 1);
       }
     }
   }
