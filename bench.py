@@ -181,26 +181,34 @@ def oracle_setup(wl, layer, q, W, X):
 
 # The one sampling recipe both oracle legs use (the GPU line's cpu_baseline
 # and the reference arm): the Hessian over SAMPLE_TOKENS tokens, the whole
-# prepare, and the sweep of SAMPLE_ROWS rows over all columns.
-SAMPLE_TOKENS = 16384
-SAMPLE_ROWS = 512
+# prepare, and the sweep of SAMPLE_ROWS rows over all columns, each part
+# scaled to the whole layer.  The reference arm times the prepare (which has
+# no smaller sample) once and shrinks the other two parts when many steps
+# are asked for, so that its whole run stays within REFERENCE_BUDGET_S.
+SAMPLE_TOKENS = 32768
+SAMPLE_ROWS = 2048
+REFERENCE_BUDGET_S = 150.0
 
 
-def oracle_sample(wl, layer, q, W, X, setup, tokens=SAMPLE_TOKENS, rows=SAMPLE_ROWS):
+def oracle_sample(wl, layer, q, W, X, setup, tokens=SAMPLE_TOKENS, rows=SAMPLE_ROWS, t_prepare=None):
     """The float64 oracle, as it stands, on a bounded sample of one layer
     solve, scaled to the whole layer: the Hessian over ``tokens`` tokens
-    (x all/tokens), the whole prepare (unscaled), and the column sweep of
-    ``rows`` rows over all columns (x out/rows).  Returns (weights/s,
-    detail)."""
+    (x all/tokens), the whole prepare (unscaled; timed here unless its time
+    ``t_prepare`` is given), and the column sweep of ``rows`` rows over all
+    columns (x out/rows).  Returns (weights/s, detail)."""
     import numpy as np
     import oracle as O
     n = wl.tokens
+    tokens = min(tokens, X.shape[1], n)
     t0 = time.perf_counter()
     O.hessian([np.asarray(X[:, :tokens])])
     t_h = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    O.prepare(setup["S"], setup["nt"], q.damp_percent, q.desc_act)
-    t_p = time.perf_counter() - t0
+    if t_prepare is None:
+        t0 = time.perf_counter()
+        O.prepare(setup["S"], setup["nt"], q.damp_percent, q.desc_act)
+        t_p = time.perf_counter() - t0
+    else:
+        t_p = t_prepare
     r = min(rows, layer.out)
     Wp = np.asarray(W[:r], dtype=np.float64)[:, setup["perm"]]
     t0 = time.perf_counter()
@@ -209,11 +217,17 @@ def oracle_sample(wl, layer, q, W, X, setup, tokens=SAMPLE_TOKENS, rows=SAMPLE_R
     sh, ss = n / tokens, layer.out / r
     total = t_h * sh + t_p + t_s * ss
     sample = (f"Hessian over {tokens} of {n} tokens (x{sh:.0f}), the whole {layer.in_}x{layer.in_} "
-              f"prepare (x1), sweep of {r} of {layer.out} rows (x{ss:.0f}); "
-              f"{t_h + t_p + t_s:.2f} s measured")
+              f"prepare (x1{', timed once' if t_prepare is not None else ''}), sweep of {r} of "
+              f"{layer.out} rows (x{ss:.0f}); {t_h + t_s + (0 if t_prepare is not None else t_p):.2f} s measured")
     return layer.out * layer.in_ / total, dict(
         cores=_blas_threads(), sample=sample, est_s_per_layer=total,
         split_s=dict(hessian=t_h * sh, prepare=t_p, sweep=t_s * ss))
+
+
+def O_prepare_once(setup, q):
+    """One oracle prepare of the layer (the reference arm times it once)."""
+    import oracle as O
+    O.prepare(setup["S"], setup["nt"], q.damp_percent, q.desc_act)
 
 
 def oracle_unsampled(wl, layer, q, W, X):
@@ -270,12 +284,23 @@ def run_reference(args):
                           "recipe_estimate_s": d_est["est_s_per_layer"], "recipe_split_s": d_est["split_s"],
                           "recipe_sample": d_est["sample"]}), flush=True)
         return
-    X = gen.x_full(wl, layer.site, tokens=SAMPLE_TOKENS)
+    X = gen.x_full(wl, layer.site, tokens=min(SAMPLE_TOKENS, wl.tokens))
     setup = oracle_setup(wl, layer, q, W, X)
     vals, detail = [], None
     t_run = time.perf_counter()
-    for i in range(args.warmup + args.steps):
-        v, detail = oracle_sample(wl, layer, q, W, X, setup)
+    t0 = time.perf_counter()
+    O_prepare_once(setup, q)
+    t_prep = time.perf_counter() - t0
+    tokens, rows = SAMPLE_TOKENS, SAMPLE_ROWS
+    n_samples = args.warmup + args.steps
+    for i in range(n_samples):
+        t0 = time.perf_counter()
+        v, detail = oracle_sample(wl, layer, q, W, X, setup, tokens, rows, t_prepare=t_prep)
+        if i == 0 and n_samples > 1:
+            # the rest of the run within the budget: shrink tokens and rows
+            left = REFERENCE_BUDGET_S - (time.perf_counter() - t_run)
+            f = min(1.0, max(left, 0.0) / ((n_samples - 1) * (time.perf_counter() - t0)))
+            tokens, rows = max(1024, int(SAMPLE_TOKENS * f)), max(16, int(SAMPLE_ROWS * f))
         if i >= args.warmup:
             vals.append(v)
     t_run = time.perf_counter() - t_run
