@@ -186,7 +186,7 @@ def oracle_setup(wl, layer, q, W, X):
 # no smaller sample) once and shrinks the other two parts when many steps
 # are asked for, so that its whole run stays within REFERENCE_BUDGET_S.
 SAMPLE_TOKENS = 32768
-SAMPLE_ROWS = 2048
+SAMPLE_ROWS = 4096
 REFERENCE_BUDGET_S = 150.0
 
 

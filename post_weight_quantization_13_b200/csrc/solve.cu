@@ -236,10 +236,16 @@ __device__ __forceinline__ uint32_t after(float v) {
 // be discarded).  U's row j + 1 is read while column j is quantized, so the
 // loads never wait in front of the column's updates.  Otherwise x / s from
 // round_div.
-template <int GSB, bool kFast>
+//
+// kRagged: some of the 32 columns lie past the layer's (the last block of a
+// layer whose width is not a multiple of 128); their errors are forced to
+// zero.  A per-column bound check costs a quarter of the loop, so the other
+// sub-blocks run without it.
+template <int GSB, bool kFast, bool kRagged>
 __device__ __forceinline__ bool sweep32(float (&x)[32], const float* ud, int64_t c0, const SolveParams& p,
                                         int64_t row, bool live, float fmaxq, float& s_, float& z_, float& inv_s,
                                         float& lsum, uint32_t (&cw)[8]) {
+  const int nvalid = kRagged ? (int)(p.in - c0 < SB ? p.in - c0 : SB) : SB;
   bool in_range = true;
 #pragma unroll
   for (int i = 0; i < 8; ++i) cw[i] = 0u;
@@ -259,7 +265,7 @@ __device__ __forceinline__ bool sweep32(float (&x)[32], const float* ud, int64_t
       for (int a = (j + 2) >> 2; a < 8; ++a) unext[a] = lds128(un + (j + 1) * SB + 4 * a);
       rnext = lds32(un + SB * SB + j + 1);
     }
-    if (GSB <= SB && j % GSB == 0 && c0 + j < p.in) {
+    if (GSB <= SB && j % GSB == 0 && (!kRagged || j < nvalid)) {
       float lo = INFINITY, hi = -INFINITY, am = 0.f;
 #pragma unroll
       for (int i = j; i < j + (GSB <= SB ? GSB : 1); ++i) minmax(x[i], lo, hi, am);
@@ -281,7 +287,7 @@ __device__ __forceinline__ bool sweep32(float (&x)[32], const float* ud, int64_t
     qf = fminf(fmaxf(qf, 0.f), fmaxq);
     const float deq = s_ * (qf - z_);
     float e = (xv - deq) * (kFast ? rcur : ud[SB * SB + j]);
-    e = c0 + j < p.in ? e : 0.f;
+    if (kRagged) e = j < nvalid ? e : 0.f;
     lsum = fmaf(e, e, lsum);
     cw[j >> 2] |= (uint32_t)qf << (8 * (j & 3));
     x[j] = -e;
@@ -330,7 +336,7 @@ __device__ __noinline__ RowState replay32(uint8_t* Xs, int rl, const float* ud, 
   float x[32];
   uint32_t cw[8];
   load_row(Xs, rl, x);
-  sweep32<GSB, false>(x, ud, c0, p, row, live, fmaxq, st.s, st.z, st.inv_s, st.lsum, cw);
+  sweep32<GSB, false, true>(x, ud, c0, p, row, live, fmaxq, st.s, st.z, st.inv_s, st.lsum, cw);
   store_row(Xs, rl, x);
   store_codes(p, row, c0, live, cw);
   return st;
@@ -681,7 +687,10 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
           // divide (its values at the sub-block's start wait in Xs for that)
           store_row(Xs, rl, x);
           RowState st{s_, z_, inv_s, lsum};
-          if (sweep32<GSB, true>(x, ud, c0, p, row, live, fmaxq, s_, z_, inv_s, lsum, cw)) {
+          const bool fast = c0 + SB <= p.in
+                                ? sweep32<GSB, true, false>(x, ud, c0, p, row, live, fmaxq, s_, z_, inv_s, lsum, cw)
+                                : sweep32<GSB, true, true>(x, ud, c0, p, row, live, fmaxq, s_, z_, inv_s, lsum, cw);
+          if (fast) {
             store_codes(p, row, c0, live, cw);
           } else {
             st = replay32<GSB>(Xs, rl, ud, c0, p, row, live, fmaxq, st);
