@@ -60,8 +60,9 @@ constexpr uint32_t kChainSmem = kCUd + 2 * kUdBytes;
 // worker CTA
 constexpr int kWSlots = 2;                     // operand ring: K chunks of (U hi, U lo, E hi, E lo)
 constexpr uint32_t kWRing = 0;
-constexpr int kWStages = 4;                    // epilogue staging tiles, 32 rows x 128 columns fp32
-constexpr uint32_t kWStg = kWRing + 4 * kWSlots * kQChunk;
+constexpr uint32_t kWStageBytes = 6 * kQChunk; // U 128 rows + E 256 rows, hi and lo
+constexpr int kWStages = 2;                    // epilogue staging tiles, 32 rows x 128 columns fp32
+constexpr uint32_t kWStg = kWRing + kWSlots * kWStageBytes;
 constexpr uint32_t kWorkerSmem = kWStg + kWStages * 32 * 128 * 4;
 constexpr uint32_t kSolveSmem = 1024 + (kChainSmem > kWorkerSmem ? kChainSmem : kWorkerSmem);
 static_assert(kSolveSmem <= 232448, "shared memory per CTA");
@@ -88,9 +89,10 @@ struct SolveParams {
 // Tensor maps, all fp32 2-D row-major: the chain's W loads (32-column x
 // 128-row boxes, 128-byte swizzle), the workers' reduce-adds into W (128 x 32,
 // no swizzle), split U^T (Uh/Ul[c][j] = U[j][c]) and split -E (32 x 128, 128-byte
-// swizzle: the tensor core's K-major operand layout).
+// swizzle: the tensor core's K-major operand layout; eh2/el2 with 256-row
+// boxes, a pair of slabs).
 struct SolveMaps {
-  CUtensorMap wld, wred, uh, ul, eh, el;
+  CUtensorMap wld, wred, uh, ul, eh, el, eh2, el2;
 };
 
 __device__ __forceinline__ bool q_aborted(const SolveParams& p) { return *(volatile unsigned*)p.abort_flag != 0; }
@@ -740,45 +742,49 @@ __device__ __forceinline__ void chain_cta(const SolveMaps& mp, const SolveParams
 }
 
 // ------------------------------------------------------------------ workers
-// A task is one 128 x 128 tile: W[slab, c] += (-E[slab, k]) U[k, c]^T, K =
-// 128, for a column block c from k + 1 on (k + 2 on when the chains take the
-// next block).  Tasks go in order of k, then c (nearest first), then slab.
-// The split operands (U^T and -E, hi and lo) stream through a ring of
-// kWSlots K chunks of 32 (64 KB each); the epilogue stages four 32-row
-// passes, so a tile's reduce-adds do not wait for one another's reads.
-// Thread 0 loads, thread 96 issues the MMAs, threads 128-255 run the
-// epilogue; two tensor-memory accumulators let a tile's epilogue overlap the
-// next tile's MMAs.
+// A task is one column block c of two slabs (rows 256 pair .. + 255, the
+// second slab absent past the last): W[slab, c] += (-E[slab, k]) U[k, c]^T
+// for both, as one 128 x 256 x 128 product, so one U tile serves two output
+// tiles.  c runs from k + 1 on (k + 2 on when the chains take the next
+// block); tasks go in order of k, then c (nearest first), then pair.  The
+// split operands (U^T: 128 rows, -E: 256 rows; hi and lo) stream through a
+// ring of kWSlots K chunks of 32 (96 KB each); the epilogue stages eight
+// 32-row passes through kWStages buffers.  Thread 0 loads, thread 96 issues
+// the MMAs, threads 128-255 run the epilogue; two tensor-memory accumulators
+// (256 columns each) let a task's epilogue overlap the next task's MMAs.
 struct QTask {
-  int k, c, slab;
+  int k, c, pair;
 };
 
-__host__ __device__ __forceinline__ int64_t tasks_of_block(int64_t nslab, int T, int k, int first) {
+__host__ __device__ __forceinline__ int pairs_of(int nslab) { return (nslab + 1) / 2; }
+
+__host__ __device__ __forceinline__ int64_t tasks_of_block(int64_t npair, int T, int k, int first) {
   const int later = T - k - first;  // column blocks k + first .. T - 1
-  return later > 0 ? nslab * later : 0;
+  return later > 0 ? npair * later : 0;
 }
 
-__host__ __device__ __forceinline__ int64_t total_tasks(int64_t nslab, int T, int first) {
+__host__ __device__ __forceinline__ int64_t total_tasks(int64_t npair, int T, int first) {
   const int64_t m = T - first;  // sum over k of (T - k - first)
-  return m > 0 ? nslab * m * (m + 1) / 2 : 0;
+  return m > 0 ? npair * m * (m + 1) / 2 : 0;
 }
 
 struct TaskWalk {
-  int k, first;
+  int k, first, npair;
   int64_t base, count;
   __device__ explicit TaskWalk(const SolveParams& p)
-      : k(0), first(1 + p.chain_next), base(0), count(tasks_of_block(p.nslab, p.T, 0, 1 + p.chain_next)) {}
+      : k(0), first(1 + p.chain_next), npair(pairs_of(p.nslab)), base(0),
+        count(tasks_of_block(pairs_of(p.nslab), p.T, 0, 1 + p.chain_next)) {}
   __device__ QTask at(int64_t t, const SolveParams& p) {
     while (t >= base + count) {
       base += count;
       ++k;
-      count = tasks_of_block(p.nslab, p.T, k, first);
+      count = tasks_of_block(npair, p.T, k, first);
     }
     const int64_t idx = t - base;
     QTask q;
     q.k = k;
-    q.c = k + first + (int)(idx / p.nslab);
-    q.slab = (int)(idx % p.nslab);
+    q.c = k + first + (int)(idx / npair);
+    q.pair = (int)(idx % npair);
     return q;
   }
 };
@@ -804,7 +810,7 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(&tslot, 256);
+    tmem_alloc(&tslot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -813,40 +819,43 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
   const uint32_t tbase = tslot;
   const int T = p.T;
   const int W = (int)gridDim.x - p.nchain, slot = (int)blockIdx.x - p.nchain;
-  const int64_t total = total_tasks(p.nslab, T, 1 + p.chain_next);
-  const uint32_t idesc = make_idesc(2, 128, 128);
+  const int64_t total = total_tasks(pairs_of(p.nslab), T, 1 + p.chain_next);
+  const uint32_t idesc = make_idesc(2, 128, 256);
+  // a stage: U hi, U lo (128 rows each), then -E hi, -E lo (256 rows each)
+  constexpr uint32_t kEOff = 2 * kQChunk, kEChunk = 2 * kQChunk, kStage = kEOff + 2 * kEChunk;
   if (threadIdx.x == 0) {
     // ------------------------------------------------------------ loader
     tma_prefetch_desc(&mp.uh);
     tma_prefetch_desc(&mp.ul);
-    tma_prefetch_desc(&mp.eh);
-    tma_prefetch_desc(&mp.el);
+    tma_prefetch_desc(&mp.eh2);
+    tma_prefetch_desc(&mp.el2);
     TaskWalk tw(p);
     bool ok = true;
     int g = 0;  // K chunks loaded so far
     for (int64_t t = slot; ok && t < total; t += W) {
       const QTask q = tw.at(t, p);
+      const int s0 = 2 * q.pair, s1 = s0 + 1;
       for (int ch = 0; ch < 4; ++ch, ++g) {
         const int rs = g % kWSlots, use = g / kWSlots;
         if (use > 0 && !q_mbar_wait(p, &st_empty[rs], (use - 1) & 1)) {
           ok = false;
           break;
         }
-        uint8_t* dst = ring + 4 * rs * kQChunk;
+        uint8_t* dst = ring + rs * kStage;
         const int32_t xk = QB * q.k + SB * ch;
-        mbar_arrive_expect_tx(&st_full[rs], 4 * kQChunk);
+        mbar_arrive_expect_tx(&st_full[rs], kStage);
         tma_load_2d(dst, &mp.uh, &st_full[rs], xk, QB * q.c);
         tma_load_2d(dst + kQChunk, &mp.ul, &st_full[rs], xk, QB * q.c);
         if (ch == 0) {
-          // the slab's block k: its -E published by the chain
-          if (!q_wait_ge(p, &p.sdone[q.slab], q.k + 1)) {
+          // both slabs' block k: -E published by their chains
+          if (!q_wait_ge(p, &p.sdone[s0], q.k + 1) || (s1 < p.nslab && !q_wait_ge(p, &p.sdone[s1], q.k + 1))) {
             ok = false;
             break;
           }
           fence_proxy_async_global();
         }
-        tma_load_2d(dst + 2 * kQChunk, &mp.eh, &st_full[rs], xk, QB * q.slab);
-        tma_load_2d(dst + 3 * kQChunk, &mp.el, &st_full[rs], xk, QB * q.slab);
+        tma_load_2d(dst + kEOff, &mp.eh2, &st_full[rs], xk, QB * s0);
+        tma_load_2d(dst + kEOff + kEChunk, &mp.el2, &st_full[rs], xk, QB * s0);
       }
     }
     if (!ok) q_give_up(p);
@@ -860,7 +869,7 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
         ok = false;
         break;
       }
-      const uint32_t d = tbase + (uint32_t)buf * 128;
+      const uint32_t d = tbase + (uint32_t)buf * 256;
       for (int ch = 0; ch < 4; ++ch, ++g) {
         const int rs = g % kWSlots;
         if (!q_mbar_wait(p, &st_full[rs], (g / kWSlots) & 1)) {
@@ -868,9 +877,10 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
           break;
         }
         tc_fence_after();
-        const uint32_t base = smem_u32(ring) + 4 * rs * kQChunk;
-        // D[c][r] (+)= sum_j U^T[c][j] (-E)[r][j]: lanes are W's columns
-        issue_mma_chunk(d, base, base + kQChunk, base + 2 * kQChunk, base + 3 * kQChunk, idesc, ch > 0);
+        const uint32_t base = smem_u32(ring) + rs * kStage;
+        // D[c][r] (+)= sum_j U^T[c][j] (-E)[r][j]: lanes are W's columns,
+        // tensor-memory columns the pair's 256 rows
+        issue_mma_chunk(d, base, base + kQChunk, base + kEOff, base + kEOff + kEChunk, idesc, ch > 0);
         umma_commit(&st_empty[rs]);
       }
       if (ok) umma_commit(&acc_full[buf]);
@@ -884,20 +894,23 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
     int tl = 0, epi_pass = 0;
     for (int64_t t = slot; t < total; t += W, ++tl) {
       const QTask q = tw.at(t, p);
+      const int s0 = 2 * q.pair, s1 = s0 + 1;
       const int buf = tl & 1;
       bool ok = q_mbar_wait(p, &acc_full[buf], (tl >> 1) & 1, true);
       if (threadIdx.x == 128 && ok) {
         // contributions reach a tile in order of k
-        ok = q_wait_ge(p, &p.cnt[(int64_t)q.slab * T + q.c], q.k);
+        ok = q_wait_ge(p, &p.cnt[(int64_t)s0 * T + q.c], q.k) &&
+             (s1 >= p.nslab || q_wait_ge(p, &p.cnt[(int64_t)s1 * T + q.c], q.k));
         fence_proxy_async_global();
       }
       if (!ok) epi_abort = 1;
       named_bar_sync(2, 128);
       if (epi_abort) break;  // the same decision in all 128 threads
       tc_fence_after();
-      const uint32_t taddr = tbase + (uint32_t)buf * 128 + ((uint32_t)(quarter * 32) << 16);
+      const uint32_t taddr = tbase + (uint32_t)buf * 256 + ((uint32_t)(quarter * 32) << 16);
+      const int npass = s1 < p.nslab ? 8 : 4;
 #pragma unroll 1
-      for (int pz = 0; pz < 4; ++pz) {
+      for (int pz = 0; pz < npass; ++pz) {
         float v[32];
         tmem_ld32(taddr + (uint32_t)(32 * pz), v);
         float* sb = stg + (epi_pass % kWStages) * (32 * 128);
@@ -908,7 +921,7 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
         fence_proxy_async_smem();
         named_bar_sync(2, 128);
         if (threadIdx.x == 128) {
-          tma_reduce_add_2d(&mp.wred, sb, QB * q.c, QB * q.slab + 32 * pz);
+          tma_reduce_add_2d(&mp.wred, sb, QB * q.c, QB * s0 + 32 * pz);
           bulk_commit();
         }
         ++epi_pass;
@@ -919,7 +932,8 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
         bulk_wait_all();
         fence_proxy_async_global();
         __threadfence();
-        atomicExch(&p.cnt[(int64_t)q.slab * T + q.c], q.k + 1);
+        atomicExch(&p.cnt[(int64_t)s0 * T + q.c], q.k + 1);
+        if (s1 < p.nslab) atomicExch(&p.cnt[(int64_t)s1 * T + q.c], q.k + 1);
       }
     }
   }
@@ -932,7 +946,7 @@ __device__ __forceinline__ void worker_cta(const SolveMaps& mp, const SolveParam
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, 512);
   }
 }
 
@@ -1018,7 +1032,7 @@ cudaError_t solve_quantize(float* Wp, int64_t out, int64_t in, int64_t np_, cons
   const int nchain = (nslab + spc - 1) / spc;
   // up to two slabs per chain, the chains also take each slab's next block
   const int chain_next = spc <= 2 ? 1 : 0;
-  const int64_t ntask = total_tasks(nslab, T, 1 + chain_next);
+  const int64_t ntask = total_tasks(pairs_of(nslab), T, 1 + chain_next);
   const int nworker = ntask > 0 ? (int)std::min<int64_t>(gmax - nchain, ntask) : 0;
   if (ntask > 0 && nworker < 1) return cudaErrorInvalidConfiguration;
   e = cudaMemsetAsync(sync, 0, solve_sync_bytes(out, np_), st);
@@ -1051,7 +1065,9 @@ cudaError_t solve_quantize(float* Wp, int64_t out, int64_t in, int64_t np_, cons
       !encode_f32_2d(&mp.uh, Uh, np_, np_, np_, SB, QB, true) ||
       !encode_f32_2d(&mp.ul, Ul, np_, np_, np_, SB, QB, true) ||
       !encode_f32_2d(&mp.eh, Eh, np_, out, np_, SB, QB, true) ||
-      !encode_f32_2d(&mp.el, El, np_, out, np_, SB, QB, true))
+      !encode_f32_2d(&mp.el, El, np_, out, np_, SB, QB, true) ||
+      !encode_f32_2d(&mp.eh2, Eh, np_, out, np_, SB, 2 * QB, true) ||
+      !encode_f32_2d(&mp.el2, El, np_, out, np_, SB, 2 * QB, true))
     return cudaErrorInvalidValue;
   const int grid = nchain + nworker;
   switch (gsb) {
