@@ -78,6 +78,8 @@ struct CholParams {
   int* t0done;     // [T]: 1 once trailing tile (0, 0) of step k has landed
   int* mrdone;     // [T]: tiles of block row k of M written
   int* gdone;      // [T]: inverse-accumulator tiles of step k whose reduce-adds have landed
+  int* p0done;     // [T]: 1 once panel tile 0 of step k (rows of block k + 2) is written
+  int* lcdone;     // [T]: 1 once CTA 0 has written L_{k+1,k}
   float* Gt;       // np x np: G^T, G_ij = sum over t < (current step) of L_it M_tj
   uint32_t* status;
 };
@@ -229,8 +231,8 @@ __device__ __forceinline__ void publish(int* flag, int j) {
   if ((threadIdx.x & 31) == 0) st_release_cta(flag, j + 1);
 }
 
-// Tiles of the chain's next step, fetched by warp 7 while the leaf runs, once
-// the workers have applied every update to them.
+// Tiles of the chain's next step, fetched by warps 4, 5 and 7 (a third each)
+// while the leaf runs, once the workers have applied every update to them.
 struct NextTiles {
   bool active;
   float *X, *C;               // shared destinations (pitch TP)
@@ -239,18 +241,19 @@ struct NextTiles {
   int tdone_target;           // tiles of step k - 1 that must have landed (0: none)
 };
 
-__device__ void fetch_next_tiles(const NextTiles& nt, int64_t np, const CholParams& p) {
+__device__ void fetch_next_tiles(const NextTiles& nt, int64_t np, const CholParams& p, int part, int nparts) {
   const int lane = threadIdx.x & 31;
-  __shared__ int go;
+  int go = 0;
   if (lane == 0) {
     bool ok = true;
     if (nt.k >= 0) ok = wait_ge(p, &p.t0done[nt.k], 1);
     if (ok && nt.tdone_target > 0) ok = wait_ge(p, &p.tdone[nt.k - 1], nt.tdone_target);
     go = ok;
   }
-  __syncwarp();
+  go = __shfl_sync(0xffffffffu, go, 0);
   if (!go) return;
-  for (int e = lane; e < 2 * FB * FB / 4; e += 32) {
+  // this warp's share of the two tiles' 16-byte pieces
+  for (int e = part * 32 + lane; e < 2 * FB * FB / 4; e += 32 * nparts) {
     const int which = e / (FB * FB / 4), q = e % (FB * FB / 4);
     const int r = q / (FB / 4), t4 = (q % (FB / 4)) * 4;
     cp_async16((which ? nt.C : nt.X) + r * TP + t4, (which ? nt.gC : nt.gX) + (int64_t)r * np + t4);
@@ -357,8 +360,9 @@ __device__ bool leaf64(const float* A, float* M, float* X, float* Lc, float* rdi
     }
   } else if (warp == 5) {
     for (int e = lane; e < 32 * 32; e += 32) M[(e >> 5) * FP + 32 + (e & 31)] = 0.f;
-  } else if (warp == 7 && nt.active) {
-    fetch_next_tiles(nt, p.np_, p);
+    if (nt.active) fetch_next_tiles(nt, p.np_, p, 1, 3);
+  } else if ((warp == 4 || warp == 7) && nt.active) {
+    fetch_next_tiles(nt, p.np_, p, warp == 4 ? 0 : 2, 3);
   }
   if (bad && lane == 0) raise_status(p.status, ST_NOT_PD);
   if (!ok && lane == 0) ok_s = 0;
@@ -526,7 +530,23 @@ __host__ __device__ __forceinline__ StepTasks step_tasks(int64_t np, int k) {
   return st;
 }
 
+// Position t of a worker's step list -> index in the kind order above.  The
+// two tasks the chain's next step waits for come first: panel tile 0 (the
+// rows of block k + 2) and trailing tile (0, 0), which holds the chain's
+// next two tiles; the rest keep the kind order.
+__host__ __device__ __forceinline__ int task_slot(int t, const StepTasks& st) {
+  if (st.npan == 0 || st.ntrail == 0) return t;
+  const int p0 = st.nmrow, t0 = st.nmrow + st.npan;
+  if (t == 0) return p0;
+  if (t == 1) return t0;
+  t -= 2;
+  if (t < p0) return t;
+  if (t < t0 - 1) return t + 1;
+  return t + 2;
+}
+
 __device__ __forceinline__ Task task_of(int64_t np, int k, int t, const StepTasks& st) {
+  t = task_slot(t, st);
   Task x;
   x.diag = 0;
   if (t < st.nmrow) {
@@ -649,7 +669,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       cphase ^= 1;
       tc_fence_after();
     };
-    // the next step's tiles, for warp 7 during the leaf of step k (k = -1:
+    // the next step's tiles, for warps 4, 5 and 7 during the leaf of step k (k = -1:
     // the first diagonal block's leaf, whose next tiles no one updates)
     auto next_tiles = [&](int k) {
       NextTiles nt;
@@ -679,7 +699,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       const float* Cb = Cb2 + (k & 1) * FB * TP;
       // L_{k+1,k} = R_{k+1,k} M_kk^T on the tensor cores: D1[r][c] =
       // sum_t X[r][t] M[c][t], lanes = rows of X (this step's tiles arrived
-      // during the previous leaf: warp 7 waited for its copies before the
+      // during the previous leaf: its fetching warps waited for their copies before the
       // leaf's closing barrier)
       stage_op(OPA, kAChunk, Xb, TP);
       stage_op(OPB, kBChunk, M, FP);
@@ -730,6 +750,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       } else if (threadIdx.x == 32) {
         __threadfence();
         atomicAdd(&p.pdone[k], 1);
+        atomicExch(&p.lcdone[k], 1);
       }
       mma_wait();
       if (reader) {
@@ -797,7 +818,6 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
   for (int k = 0; ok && k < T; ++k) {
     const StepTasks st = step_tasks(np, k);
     const int ntask = st.total();
-    const int t_first_trail = st.nmrow + st.npan;  // task index of trailing tile (0, 0)
     if (warp < 4) {
       // ------------------------------------------------ staging and MMA issue
       // the step's inputs: M_kk published, and every trailing and inverse-
@@ -819,7 +839,16 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       int tl = tcount;
       for (int t = slot; t < ntask && !local_abort; t += W, ++tl) {
         const Task x = task_of(np, k, t, st);
-        if ((x.kind == 1 || x.kind == 3) && !panels_seen) {
+        const bool t00 = x.kind == 1 && x.r0 == (int64_t)FB * (k + 1) && x.c0 == (int64_t)FB * (k + 1);
+        if (t00 && !panels_seen) {
+          // trailing tile (0, 0) reads only L_{k+1,k} and panel tile 0
+          if (threadIdx.x == 0) {
+            if (!wait_ge(p, &p.lcdone[k], 1) || !wait_ge(p, &p.p0done[k], 1)) local_abort = 1;
+            fence_proxy_async_global();
+          }
+          named_bar_sync(1, 128);
+          if (local_abort) break;
+        } else if ((x.kind == 1 || x.kind == 3) && !panels_seen) {
           // every panel tile of the step (by the workers, and one by CTA 0)
           if (threadIdx.x == 0) {
             if (!wait_ge(p, &p.pdone[k], st.npan + 1)) local_abort = 1;
@@ -987,6 +1016,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
             fence_proxy_async_global();
             __threadfence();
             atomicAdd(x.kind == 0 ? &p.pdone[k] : &p.mrdone[k], 1);
+            if (x.kind == 0 && x.r0 == (int64_t)FB * (k + 2)) atomicExch(&p.p0done[k], 1);
           }
         } else {
           // TMA reduce-add in L2, 32 accumulator columns per pass through one
@@ -1039,7 +1069,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
           }
           tc_fence_before();
           mbar_arrive(&acc_empty[buf]);
-          if (t == t_first_trail && threadIdx.x == 128) {
+          if (x.kind == 1 && x.r0 == (int64_t)FB * (k + 1) && x.c0 == (int64_t)FB * (k + 1) && threadIdx.x == 128) {
             // trailing tile (0, 0) holds the chain's next two tiles
             bulk_wait_all();
             fence_proxy_async_global();
@@ -1090,7 +1120,7 @@ size_t chain_smem_bytes() { return kChainOpOffset + kChainOpABytes + kChainOpBBy
 
 size_t chol_smem_bytes() { return 1024 + std::max<size_t>(kWorkerSmem, chain_smem_bytes()); }
 
-size_t chol_sync_bytes(int64_t np_) { return sizeof(int) * (size_t)(5 * (np_ / FB) + 4); }
+size_t chol_sync_bytes(int64_t np_) { return sizeof(int) * (size_t)(7 * (np_ / FB) + 4); }
 
 namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -1162,6 +1192,8 @@ cudaError_t chol_factor(float* R, int64_t np_, float* Lh, float* Ll, float* Mh, 
   p.t0done = p.tdone + T;
   p.mrdone = p.t0done + T;
   p.gdone = p.mrdone + T;
+  p.p0done = p.gdone + T;
+  p.lcdone = p.p0done + T;
   p.Gt = Gt;
   p.status = status;
   CUtensorMap rmap, gmap;
