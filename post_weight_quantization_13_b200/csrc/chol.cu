@@ -7,12 +7,12 @@
 // Right-looking with 64-wide blocks and a look-ahead of one block.  Step k:
 //   CTA 0 (the chain)   L_{k+1,k} = R_{k+1,k} M_kk^T and R_{k+1,k+1} - L L^T
 //                       as 3xTF32 tcgen05 MMAs (M = 128 with zero rows), then
-//                       the leaf of block k+1 on six warps: its Cholesky
-//                       factor in registers (one pivot chain per 32 rows) and
-//                       the factor's inverse M_{k+1,k+1}, pipelined through
-//                       shared memory.  A seventh warp meanwhile fetches the
-//                       next step's two tiles once the workers have updated
-//                       them.
+//                       the leaf of block k+1: its Cholesky factor in
+//                       registers (one pivot chain per 32 rows) and the
+//                       factor's inverse M_{k+1,k+1}, pipelined through shared
+//                       memory.  Three warps with little leaf work meanwhile
+//                       fetch the next step's two tiles once the workers have
+//                       updated them.
 //   CTAs 1.. (workers)  3xTF32 tcgen05 tile tasks (128 x 128 or 128 x 64,
 //                       K = 64):
 //                         M row tiles   M_kj = -M_kk G_kj   (j < k)
