@@ -20,11 +20,12 @@
 //                memory by TMA; once all of block k's -E has landed the slab
 //                publishes it.
 //   worker CTAs  apply a finished block's errors to the later blocks, one
-//                128 x 128 tile per task: W[slab, c] += (-E[slab, k]) U[k, c]
-//                (3xTF32, K = 128), added in L2 by a TMA reduce-add.  The
-//                tasks are taken in order of k, nearest column block first,
-//                and each tile receives its contributions in order of k, so
-//                the result does not depend on timing.
+//                column block of two slabs per task: W[slab, c] += (-E[slab,
+//                k]) U[k, c] (3xTF32, 128 x 256 x 128), added in L2 by TMA
+//                reduce-adds.  The tasks are taken in order of k, nearest
+//                column block first, and each tile receives its
+//                contributions in order of k, so the result does not depend
+//                on timing.
 //
 // A chain starts block k of a slab once all k earlier contributions have
 // landed in that block; the slabs of one chain alternate, so the tile tasks a
