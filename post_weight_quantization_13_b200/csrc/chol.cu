@@ -12,7 +12,10 @@
 //                       factor's inverse M_{k+1,k+1}, pipelined through shared
 //                       memory.  Three warps with little leaf work meanwhile
 //                       fetch the next step's two tiles once the workers have
-//                       updated them.
+//                       updated them.  The leaf's off-diagonal inverse block
+//                       is a forward substitution that follows the second
+//                       half's pivots, so the leaf ends with its last pivot
+//                       chain.
 //   CTAs 1.. (workers)  3xTF32 tcgen05 tile tasks (128 x 128 or 128 x 64,
 //                       K = 64):
 //                         M row tiles   M_kj = -M_kk G_kj   (j < k)
@@ -60,7 +63,7 @@ constexpr int kStages = 4;                           // epilogue staging buffers
 constexpr uint32_t kWorkerSmem = 4 * kRegionBytes + kStages * kStageBytes;  // 192 KB
 constexpr uint32_t kTmemCols = 256;                 // two 128-column accumulators
 // chain CTA: fp32 tiles, then (1024-aligned) the tensor-core operand regions
-constexpr uint32_t kChainFloats = 4 * FB * TP + 2 * FB * FP + 32 * FP + FB * 64 + FB + 4;
+constexpr uint32_t kChainFloats = 4 * FB * TP + 2 * FB * FP + FB * 64 + FB + 4;
 constexpr uint32_t kChainOpOffset = (kChainFloats * 4 + 1023) / 1024 * 1024;
 constexpr uint32_t kChainOpABytes = 2 * 2 * 128 * 128;  // 128 rows x K 64, hi and lo
 constexpr uint32_t kChainOpBBytes = 2 * 2 * 64 * 128;   // 64 rows x K 64, hi and lo
@@ -101,8 +104,12 @@ __device__ bool wait_ge(const CholParams& p, const int* f, int target) {
   volatile const int* vf = f;
   if (vf[0] < target) {
     const uint64_t t0 = globaltimer();
-    while (vf[0] < target) {
-      if (aborted(p)) return false;
+    for (;;) {
+      // both loads are in flight together: one L2 round trip a poll
+      const int v = vf[0];
+      const bool ab = aborted(p);
+      if (v >= target) break;
+      if (ab) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
         give_up(p);
         return false;
@@ -142,26 +149,31 @@ __device__ __forceinline__ int ld_acquire_cta(const int* p) {
 
 // ------------------------------------------------------------------ chain CTA
 // The leaf: A (FB x FB, pitch FP, lower triangle read) -> M = L^-1 (pitch FP,
-// zeros above the diagonal), where A = L L^T.  Six warps, each a chain of
+// zeros above the diagonal), where A = L L^T.  Seven warps, each a chain of
 // pivots over registers, fed through shared memory:
-//   warp 0  factors rows 0..31 (pivots 0..31); lane i keeps row i;
+//   warp 0  factors rows 0..31 (pivots 0..31); lane i keeps row i; then
+//           forms M10 = L11^-1 Y with Y = -L10 M00: Y once L10 and M00 are
+//           complete (lane = column), then forward substitution with L11
+//           behind warp 6;
 //   warp 1  rows 32..63, columns 0..31: forms L[32+i][j] for pivots 0..31
 //           from the pivots warp 0 publishes;
 //   warp 6  rows 32..63, columns 32..63: applies the first 32 pivots' updates
 //           to the trailing block, then factors it (pivots 32..63);
-//   warp 2  inverts L00 (M00 = L00^-1 by forward substitution, lane = column),
-//           trailing warp 0 by a pivot or more;
+//   warp 7  inverts L00 (M00 = L00^-1 by forward substitution, lane =
+//           column), trailing warp 0 by a pivot or more;
 //   warp 3  inverts L11 (M11) behind warp 6;
-//   warp 5  zeroes the upper block of M.
-// Warp w issues on scheduler w % 4: the factor chains (warps 0, 1 and, for
-// pivots 32..63, 6) each have a scheduler to themselves while they run.
-// Then every warp forms M10 = -M11 (L10 M00).  Column j of L goes to Lc[j][.]
-// and 1/L_jj to rdiag[j]; fl[0..2] count the pivots published by warps 0, 1
-// and 6 (release / acquire, once per pass of four pivots).  Each lane keeps a 32-entry window of its row
-// (or column) that slides by four pivots per pass, so every register index is
-// a compile-time constant and the code of one pass serves all passes.  A
-// non-positive or non-finite pivot raises ST_NOT_PD (it is replaced by 1 so
-// the leaf finishes).  False if a wait gave up.
+//   warp 4  zeroes the upper block of M.
+// Warp w issues on scheduler w % 4: warp 6's pivots share theirs with a
+// warp that mostly sleeps (2, fetching the next tiles), and warps 0, 1, 3 and
+// 7 do not run their pivot chains on the same scheduler at the same time.
+// Column j of L goes to Lc[j][.] and 1/L_jj to rdiag[j]; fl[0..2] count the
+// pivots published by warps 0, 1 and 6 (release / acquire, once per pass of
+// four pivots) and fl[3] the rows of M00 (once, at the end).  Each lane keeps
+// a 32-entry window of its row (or column) that slides by four pivots per
+// pass, so every register index is a compile-time constant and the code of
+// one pass serves all passes.  A non-positive or non-finite pivot raises
+// ST_NOT_PD (it is replaced by 1 so the leaf finishes).  False if a wait gave
+// up.
 constexpr int LCP = 64;  // pitch of Lc (one column of L per row)
 
 __device__ __forceinline__ bool wait_count(const int* f, int j) {
@@ -231,14 +243,43 @@ __device__ __forceinline__ void publish(int* flag, int j) {
   if ((threadIdx.x & 31) == 0) st_release_cta(flag, j + 1);
 }
 
-// Tiles of the chain's next step, fetched by warps 4, 5 and 7 (a third each)
+// Forward substitution with L on the pivots o .. o + 31, lane = one column of
+// the right-hand side: x holds that column's rows o + 4m .. o + 4m + 31 at
+// pass m (the window slides by four rows a pass; the rows past o + 31 are
+// never read), and row j of the solution goes to M[j][oc + lane].  Follows
+// the pivots as flag f publishes them.  False if a wait gave up.
+__device__ __forceinline__ bool forward_subst(float (&x)[32], int o, int oc, const int* f, float* M, const float* Lc,
+                                              const float* rdiag) {
+  const int lane = threadIdx.x & 31;
+  bool ok = true;
+#pragma unroll 1
+  for (int m = 0; m < 8 && ok; ++m) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = o + 4 * m + u;
+      if (!wait_count(f, j)) ok = false;
+      const float mj = x[u] * rdiag[j];
+      M[j * FP + oc + lane] = mj;
+      const float* col = Lc + j * LCP + o + 4 * m;
+      switch (u) {
+        case 0: axpy_window<0>(x, mj, col); break;
+        case 1: axpy_window<1>(x, mj, col); break;
+        case 2: axpy_window<2>(x, mj, col); break;
+        default: axpy_window<3>(x, mj, col); break;
+      }
+    }
+    shift4(x);
+  }
+  return ok;
+}
+
+// Tiles of the chain's next step, fetched by warps 1, 2 and 5 (a third each)
 // while the leaf runs, once the workers have applied every update to them.
 struct NextTiles {
   bool active;
   float *X, *C;               // shared destinations (pitch TP)
   const float *gX, *gC;       // R tiles (k+2, k+1) and (k+2, k+2)
   int k;                      // the step whose trailing tile (0, 0) must have landed
-  int tdone_target;           // tiles of step k - 1 that must have landed (0: none)
 };
 
 __device__ void fetch_next_tiles(const NextTiles& nt, int64_t np, const CholParams& p, int part, int nparts) {
@@ -246,8 +287,11 @@ __device__ void fetch_next_tiles(const NextTiles& nt, int64_t np, const CholPara
   int go = 0;
   if (lane == 0) {
     bool ok = true;
+    // trailing tile (0, 0) of step k brings the last update that the chain's
+    // next step needs in both tiles: the worker that wrote it waited, before
+    // its step, for every trailing tile of step k - 1 to land, and those
+    // workers for step k - 2's, and so on
     if (nt.k >= 0) ok = wait_ge(p, &p.t0done[nt.k], 1);
-    if (ok && nt.tdone_target > 0) ok = wait_ge(p, &p.tdone[nt.k - 1], nt.tdone_target);
     go = ok;
   }
   go = __shfl_sync(0xffffffffu, go, 0);
@@ -262,11 +306,11 @@ __device__ void fetch_next_tiles(const NextTiles& nt, int64_t np, const CholPara
   cp_async_wait<0>();
 }
 
-__device__ bool leaf64(const float* A, float* M, float* X, float* Lc, float* rdiag, int* fl, const CholParams& p,
+__device__ bool leaf64(const float* A, float* M, float* Lc, float* rdiag, int* fl, const CholParams& p,
                        const NextTiles& nt) {
   __shared__ int ok_s;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x < 3) fl[threadIdx.x] = 0;
+  if (threadIdx.x < 4) fl[threadIdx.x] = 0;
   if (threadIdx.x == 0) ok_s = 1;
   __syncthreads();
   bool ok = true, bad = false;
@@ -284,6 +328,16 @@ __device__ bool leaf64(const float* A, float* M, float* X, float* Lc, float* rdi
       bad |= factor_pivot<3>(w, dn, 4 * m + 3, 4 * m + 3, 0, Lc, rdiag, col + (4 * m + 3) * LCP);
       publish(&fl[0], 4 * m + 3);
       shift4(w);
+    }
+    // M10: Y = -L10 M00 (x[r] = Y[r][lane]), then L11 M10 = Y
+    float x[32];
+#pragma unroll
+    for (int t = 0; t < 32; ++t) x[t] = 0.f;
+    ok = wait_count(&fl[1], 31) && wait_count(&fl[3], 31);
+    if (ok) {
+#pragma unroll 1
+      for (int t = 0; t < 32; ++t) axpy_window<-1>(x, M[t * FP + lane], Lc + t * LCP + 32);
+      ok = forward_subst(x, 32, 0, &fl[2], M, Lc, rdiag);
     }
   } else if (warp == 1) {
     // rows 32..63, columns 0..31: L[32+i][j] = A'[32+i][j] / L_jj
@@ -310,6 +364,7 @@ __device__ bool leaf64(const float* A, float* M, float* X, float* Lc, float* rdi
       publish(&fl[1], 4 * m + 3);
       shift4(v);
     }
+    if (ok && nt.active) fetch_next_tiles(nt, p.np_, p, 0, 3);
   } else if (warp == 6) {
     float z[32];
 #pragma unroll
@@ -333,74 +388,24 @@ __device__ bool leaf64(const float* A, float* M, float* X, float* Lc, float* rdi
       publish(&fl[2], 32 + 4 * m + 3);
       shift4(z);
     }
-  } else if (warp == 2 || warp == 3) {
-    // forward substitution M = L^-1 on one diagonal 32-block, lane = column
-    const int o = warp == 2 ? 0 : 32;
-    const int* f = warp == 2 ? &fl[0] : &fl[2];
+  } else if (warp == 7 || warp == 3) {
+    // M00 = L00^-1 (warp 7) and M11 = L11^-1 (warp 3): right-hand side I
     float x[32];
 #pragma unroll
     for (int t = 0; t < 32; ++t) x[t] = t == lane ? 1.f : 0.f;
-#pragma unroll 1
-    for (int m = 0; m < 8 && ok; ++m) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = o + 4 * m + u;
-        if (!wait_count(f, j)) ok = false;
-        const float mj = x[u] * rdiag[j];
-        M[j * FP + o + lane] = mj;
-        const float* col = Lc + j * LCP + o + 4 * m;
-        switch (u) {
-          case 0: axpy_window<0>(x, mj, col); break;
-          case 1: axpy_window<1>(x, mj, col); break;
-          case 2: axpy_window<2>(x, mj, col); break;
-          default: axpy_window<3>(x, mj, col); break;
-        }
-      }
-      shift4(x);
+    if (warp == 7) {
+      ok = forward_subst(x, 0, 0, &fl[0], M, Lc, rdiag);
+      publish(&fl[3], 31);
+    } else {
+      ok = forward_subst(x, 32, 32, &fl[2], M, Lc, rdiag);
     }
-  } else if (warp == 5) {
+  } else if (warp == 4) {
     for (int e = lane; e < 32 * 32; e += 32) M[(e >> 5) * FP + 32 + (e & 31)] = 0.f;
-    if (nt.active) fetch_next_tiles(nt, p.np_, p, 1, 3);
-  } else if ((warp == 4 || warp == 7) && nt.active) {
-    fetch_next_tiles(nt, p.np_, p, warp == 4 ? 0 : 2, 3);
+  } else if ((warp == 2 || warp == 5) && nt.active) {
+    fetch_next_tiles(nt, p.np_, p, warp == 2 ? 1 : 2, 3);
   }
   if (bad && lane == 0) raise_status(p.status, ST_NOT_PD);
   if (!ok && lane == 0) ok_s = 0;
-  __syncthreads();
-  // M10 = -M11 (L10 M00): X = L10 M00, then M10 = -M11 X (32 x 32 x 32 each,
-  // 2 x 2 outputs per thread)
-  {
-    const int r0 = (threadIdx.x / 16) * 2, c0 = (threadIdx.x % 16) * 2;
-    float acc[2][2] = {};
-#pragma unroll 4
-    for (int t = 0; t < 32; ++t) {
-      const float a0 = Lc[t * LCP + 32 + r0], a1 = Lc[t * LCP + 33 + r0];  // L[32 + r][t]
-      const float b0 = M[t * FP + c0], b1 = M[t * FP + c0 + 1];
-      acc[0][0] = fmaf(a0, b0, acc[0][0]);
-      acc[0][1] = fmaf(a0, b1, acc[0][1]);
-      acc[1][0] = fmaf(a1, b0, acc[1][0]);
-      acc[1][1] = fmaf(a1, b1, acc[1][1]);
-    }
-    X[r0 * FP + c0] = acc[0][0];
-    X[r0 * FP + c0 + 1] = acc[0][1];
-    X[(r0 + 1) * FP + c0] = acc[1][0];
-    X[(r0 + 1) * FP + c0 + 1] = acc[1][1];
-    __syncthreads();
-    float bcc[2][2] = {};
-#pragma unroll 4
-    for (int t = 0; t < 32; ++t) {
-      const float a0 = M[(32 + r0) * FP + 32 + t], a1 = M[(33 + r0) * FP + 32 + t];
-      const float b0 = X[t * FP + c0], b1 = X[t * FP + c0 + 1];
-      bcc[0][0] = fmaf(a0, b0, bcc[0][0]);
-      bcc[0][1] = fmaf(a0, b1, bcc[0][1]);
-      bcc[1][0] = fmaf(a1, b0, bcc[1][0]);
-      bcc[1][1] = fmaf(a1, b1, bcc[1][1]);
-    }
-    M[(32 + r0) * FP + c0] = -bcc[0][0];
-    M[(32 + r0) * FP + c0 + 1] = -bcc[0][1];
-    M[(33 + r0) * FP + c0] = -bcc[1][0];
-    M[(33 + r0) * FP + c0 + 1] = -bcc[1][1];
-  }
   __syncthreads();
   return ok_s != 0;
 }
@@ -607,8 +612,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
     float* Cb2 = Xb2 + 2 * FB * TP;  // [2][FB][TP] R_{k+1,k+1}
     float* A = Cb2 + 2 * FB * TP;    // [FB][FP]
     float* M = A + FB * FP;          // [FB][FP]
-    float* Xs = M + FB * FP;         // [32][FP] scratch of the leaf's merge
-    float* Lc = Xs + 32 * FP;        // [FB][LCP] columns of L (leaf), 16-byte aligned
+    float* Lc = M + FB * FP;         // [FB][LCP] columns of L (leaf), 16-byte aligned
     float* rdiag = Lc + FB * LCP;    // [FB]
     int* fl = reinterpret_cast<int*>(rdiag + FB);
     // tensor-core operands of the chain's two products (split, 128-byte
@@ -669,7 +673,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       cphase ^= 1;
       tc_fence_after();
     };
-    // the next step's tiles, for warps 4, 5 and 7 during the leaf of step k (k = -1:
+    // the next step's tiles, for warps 1, 2 and 5 during the leaf of step k (k = -1:
     // the first diagonal block's leaf, whose next tiles no one updates)
     auto next_tiles = [&](int k) {
       NextTiles nt;
@@ -680,8 +684,6 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       nt.gX = tile(k + 2, k + 1);
       nt.gC = tile(k + 2, k + 2);
       nt.k = k;
-      nt.tdone_target = 0;
-      if (k >= 1) nt.tdone_target = step_tasks(np, k - 1).ntrail;
       return nt;
     };
     // the first diagonal block
@@ -690,7 +692,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       A[r * FP + c] = __ldcg(p.R + (int64_t)r * np + c);
     }
     __syncthreads();
-    if (!leaf64(A, M, Xs, Lc, rdiag, fl, p, next_tiles(-1))) give_up(p);
+    if (!leaf64(A, M, Lc, rdiag, fl, p, next_tiles(-1))) give_up(p);
     store_diag_m(p, M, 0);
     publish_m(1);
     const uint32_t idesc = make_idesc(2, 128, 64);
@@ -761,7 +763,7 @@ __global__ void __launch_bounds__(FNT, 1) chol_kernel(const __grid_constant__ CU
       }
       tc_fence_before();
       __syncthreads();
-      if (!leaf64(A, M, Xs, Lc, rdiag, fl, p, next_tiles(k))) give_up(p);
+      if (!leaf64(A, M, Lc, rdiag, fl, p, next_tiles(k))) give_up(p);
       store_diag_m(p, M, k + 1);
       publish_m(k + 2);
     }

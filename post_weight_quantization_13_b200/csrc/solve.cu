@@ -108,8 +108,12 @@ __device__ bool q_wait_ge(const SolveParams& p, const int* f, int target) {
   volatile const int* vf = f;
   if (vf[0] < target) {
     const uint64_t t0 = globaltimer();
-    while (vf[0] < target) {
-      if (q_aborted(p)) return false;
+    for (;;) {
+      // both loads are in flight together: one L2 round trip a poll
+      const int v = vf[0];
+      const bool ab = q_aborted(p);
+      if (v >= target) break;
+      if (ab) return false;
       if (globaltimer() - t0 > kWaitLimitNs) {
         q_give_up(p);
         return false;
