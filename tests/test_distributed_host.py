@@ -1,4 +1,4 @@
-"""The sharded layer solve's partition and exchange logic, run as two gloo
+"""The sharded layer solve's partition and exchange logic, run as gloo
 ranks on the host.  Each rank holds a share of the calibration tokens and
 solves a share of the rows; the arithmetic steps are the oracle's (LayerOps
 built from it), so the gathered layer must equal the oracle's single-process
@@ -91,20 +91,21 @@ def _rank_main(rank, world, port, case, q):
 
 
 CASES = [
-    (11, 37, 64, 96, dict(bits=4, group_size=32, desc_act=True)),    # rows 19 + 18
-    (12, 40, 96, 1, dict(bits=3, group_size=-1, sym=True)),          # rank 1 has no tokens
+    (2, (11, 37, 64, 96, dict(bits=4, group_size=32, desc_act=True))),    # rows 19 + 18
+    (2, (12, 40, 96, 1, dict(bits=3, group_size=-1, sym=True))),          # rank 1 has no tokens
+    (3, (13, 23, 64, 2, dict(bits=2, group_size=16, desc_act=True))),     # rows 8 + 8 + 7; rank 2 no tokens
 ]
 
 
-@pytest.mark.parametrize("case", CASES)
-def test_two_gloo_ranks_give_the_single_process_solve(case):
+@pytest.mark.parametrize("world,case", CASES)
+def test_gloo_ranks_give_the_single_process_solve(world, case):
     import torch.multiprocessing as mp
 
     import oracle as O
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, case, q)) for r in range(2)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, case, q)) for r in range(world)]
     for p in procs:
         p.start()
     got = sorted((q.get(timeout=180) for _ in procs), key=lambda t: t[0])
@@ -117,7 +118,8 @@ def test_two_gloo_ranks_give_the_single_process_solve(case):
     full = dict(bits=4, group_size=128, sym=False, desc_act=False, damp_percent=0.01, block_size=128)
     full.update(cfgd)
     ref = O.gptq_layer(W, S, tokens, **full)
-    assert [g[2] for g in got] == [(0, (out + 1) // 2), ((out + 1) // 2, out)]
+    from post_weight_quantization_13_b200.distributed import shard_bounds
+    assert [g[2] for g in got] == [shard_bounds(out, world, r) for r in range(world)]
     for rank, n, rows, k in got:
         assert n == tokens
         assert np.array_equal(k["S"], S)                  # the all-reduced Hessian, exact
