@@ -207,11 +207,11 @@ gptq_status_t gptq_prepare_hinv(const float* S, int64_t n, int64_t in,
  *   loss     fp32[out] or NULL: sum over columns of e^2 for each row (the
  *            quadratic error (W - deq) H (W - deq)^T with the damped H).
  * ws / ws_bytes: workspace from gptq_workspace_bytes(out, in, cfg).
- * Asynchronous.  out == 0 is a no-op.  Inside the call, the kernels of the
- * sweep chain after the first are programmatic dependent launches on the
- * caller's stream.  Each waits for the kernel before it, so the call's
- * work is ordered after everything already queued on the stream and before
- * everything queued after it, as with ordinary launches.
+ * Asynchronous.  out == 0 is a no-op.  Inside the call, every kernel is an
+ * ordinary launch on the caller's stream (the gathers, one cooperative
+ * launch for the sweep and its updates, the inverse permutation and the
+ * packing), so the call's work is ordered after everything already queued
+ * on the stream and before everything queued after it.
  * The call returns before its kernels run, so a failure inside them (a
  * bounded device-side wait that gave up: GPTQ_ERR_TIMEOUT) is not in its
  * return value: it is raised in the status word at the start of ws, which
