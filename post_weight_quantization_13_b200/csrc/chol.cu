@@ -149,7 +149,7 @@ __device__ __forceinline__ int ld_acquire_cta(const int* p) {
 
 // ------------------------------------------------------------------ chain CTA
 // The leaf: A (FB x FB, pitch FP, lower triangle read) -> M = L^-1 (pitch FP,
-// zeros above the diagonal), where A = L L^T.  Seven warps, each a chain of
+// zeros above the diagonal), where A = L L^T.  Five warps run chains of
 // pivots over registers, fed through shared memory:
 //   warp 0  factors rows 0..31 (pivots 0..31); lane i keeps row i; then
 //           forms M10 = L11^-1 Y with Y = -L10 M00: Y once L10 and M00 are
@@ -162,7 +162,8 @@ __device__ __forceinline__ int ld_acquire_cta(const int* p) {
 //   warp 7  inverts L00 (M00 = L00^-1 by forward substitution, lane =
 //           column), trailing warp 0 by a pivot or more;
 //   warp 3  inverts L11 (M11) behind warp 6;
-//   warp 4  zeroes the upper block of M.
+//   warp 4  zeroes the upper block of M;
+//   warps 1 (once L10 is done), 2 and 5 fetch the next step's tiles.
 // Warp w issues on scheduler w % 4: warp 6's pivots share theirs with a
 // warp that mostly sleeps (2, fetching the next tiles), and warps 0, 1, 3 and
 // 7 do not run their pivot chains on the same scheduler at the same time.
